@@ -1,0 +1,216 @@
+"""Python binding of libdsv4 (the C ABI declared in include/dsv4.h).
+
+Argument marshalling only: every function takes torch tensors that already live on
+the CUDA device, checks dtype / shape / contiguity, allocates missing outputs with
+torch (device memory is PyTorch's job here), and calls the C entry point of the same
+name on the current torch stream. All arithmetic happens in the library's CUDA
+kernels. If the library is missing, importing this package fails loudly; there is no
+CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "DSV4Error", "lib", "LIB_PATH", "F32", "BF16", "FP4",
+    "dsv4_compress", "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
+    "dsv4_hybrid_sparse_attn", "dsv4_check_errors",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsv4.so")
+F32, BF16, FP4 = 0, 1, 2
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libdsv4.so not found at {LIB_PATH}: build it with "
+        "`python -m compressed_sparse_mqa_dsv4_b200.build` (nvcc, sm_100a)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P, _I, _L, _F, _S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+lib.dsv4_abi_version.restype = _I
+lib.dsv4_status_string.restype = ctypes.c_char_p
+lib.dsv4_status_string.argtypes = [_I]
+lib.dsv4_last_error_message.restype = ctypes.c_char_p
+lib.dsv4_check_errors.restype = _I
+lib.dsv4_check_errors.argtypes = [_P]
+lib.dsv4_compress.restype = _I
+lib.dsv4_compress.argtypes = [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+lib.dsv4_quantize_fp4.restype = _I
+lib.dsv4_quantize_fp4.argtypes = [_P, _P, _P, _L, _I, _P]
+lib.dsv4_index_topk_workspace_size.restype = _S
+lib.dsv4_index_topk_workspace_size.argtypes = [_I, _I, _I, _I]
+lib.dsv4_index_topk.restype = _I
+lib.dsv4_index_topk.argtypes = [_I, _P, _P, _P, _P, _P, _L, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                _P, _P, _P, _L, _P, _S, _P]
+lib.dsv4_hybrid_sparse_attn.restype = _I
+lib.dsv4_hybrid_sparse_attn.argtypes = [_I, _P, _P, _L, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
+                                        _I, _I, _I, _P, _F, _P, _P, _P]
+
+
+class DSV4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.dsv4_last_error_message().decode(errors="replace")
+        name = lib.dsv4_status_string(status).decode()
+        super().__init__(f"{where}: {name} ({status}): {msg}")
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise DSV4Error(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def _code(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return F32
+    if dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported dtype {dtype}")
+
+
+def dsv4_compress(C: torch.Tensor, Z: torch.Tensor, bias: torch.Tensor, m: int, overlap: bool,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Compressor: C, Z [B, n, S*c], bias fp32 [S, m, c] -> out [B, n//m, c]."""
+    _dev(C, "C"), _dev(Z, "Z", C.dtype), _dev(bias, "bias", torch.float32)
+    B, n, width = C.shape
+    S = 2 if overlap else 1
+    c = width // S
+    if out is None:
+        out = torch.empty(B, n // m, c, dtype=C.dtype, device=C.device)
+    _dev(out, "out", C.dtype)
+    _check(lib.dsv4_compress(_code(C.dtype), _ptr(C), _ptr(Z), _ptr(bias), _ptr(out), B, n, c, m,
+                             1 if overlap else 0, _stream(stream)), "dsv4_compress")
+    return out
+
+
+def dsv4_quantize_fp4(x: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                      scales: Optional[torch.Tensor] = None, stream=None):
+    """bf16 [rows, cols] -> (codes uint8 [rows, cols/2], scales uint8 [rows, cols/16])."""
+    _dev(x, "x", torch.bfloat16)
+    cols = x.shape[-1]
+    rows = x.numel() // max(cols, 1)
+    if codes is None:
+        codes = torch.empty(rows, cols // 2, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(rows, cols // 16, dtype=torch.uint8, device=x.device)
+    _check(lib.dsv4_quantize_fp4(_ptr(x), _ptr(codes), _ptr(scales), rows, cols, _stream(stream)),
+           "dsv4_quantize_fp4")
+    return codes, scales
+
+
+def dsv4_index_topk_workspace_size(B: int, nq: int, max_entries: int, k: int) -> int:
+    return int(lib.dsv4_index_topk_workspace_size(B, nq, max_entries, k))
+
+
+def dsv4_index_topk(qI: torch.Tensor, w: torch.Tensor, KI: torch.Tensor,
+                    kv_row_off: torch.Tensor, q_pos0: torch.Tensor, m: int, k: int,
+                    max_entries: int, qI_scales: Optional[torch.Tensor] = None,
+                    KI_scales: Optional[torch.Tensor] = None, H_I: Optional[int] = None,
+                    c_I: Optional[int] = None, idx: Optional[torch.Tensor] = None,
+                    counts: Optional[torch.Tensor] = None,
+                    scores_out: Optional[torch.Tensor] = None,
+                    workspace: Optional[torch.Tensor] = None, stream=None):
+    """Indexer scores + TopK. Returns (idx int32 [B, nq, k], counts int32 [B, nq]).
+
+    qI: [B, nq, H_I, c_I] fp32/bf16, or FP4 codes uint8 [B, nq, H_I, c_I/2] with qI_scales.
+    KI: [rows, c_I] fp32/bf16, or FP4 codes uint8 [rows, c_I/2] with KI_scales.
+    """
+    fp4 = qI.dtype == torch.uint8
+    _dev(qI, "qI"), _dev(w, "w", torch.float32), _dev(KI, "KI", qI.dtype)
+    _dev(kv_row_off, "kv_row_off", torch.int64), _dev(q_pos0, "q_pos0", torch.int32)
+    B, nq = qI.shape[0], qI.shape[1]
+    H_I = qI.shape[2] if H_I is None else H_I
+    c_I = (qI.shape[3] * (2 if fp4 else 1)) if c_I is None else c_I
+    qd = FP4 if fp4 else _code(qI.dtype)
+    if fp4:
+        _dev(qI_scales, "qI_scales", torch.uint8), _dev(KI_scales, "KI_scales", torch.uint8)
+    ki_rows = KI.shape[0]
+    if idx is None:
+        idx = torch.empty(B, nq, k, dtype=torch.int32, device=qI.device)
+    if counts is None:
+        counts = torch.empty(B, nq, dtype=torch.int32, device=qI.device)
+    ws_bytes = 0
+    scores_ld = 0
+    if scores_out is not None:
+        _dev(scores_out, "scores_out", torch.float32)
+        scores_ld = scores_out.shape[-1]
+    else:
+        ws_bytes = dsv4_index_topk_workspace_size(B, nq, max_entries, k)
+        if workspace is None or workspace.numel() < ws_bytes:
+            workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=qI.device)
+        ws_bytes = workspace.numel()
+    _check(lib.dsv4_index_topk(qd, _ptr(qI), _ptr(qI_scales), _ptr(w), _ptr(KI), _ptr(KI_scales),
+                               ki_rows, _ptr(kv_row_off), _ptr(q_pos0), B, nq, H_I, c_I, m, k,
+                               max_entries, _ptr(idx), _ptr(counts), _ptr(scores_out), scores_ld,
+                               _ptr(workspace) if scores_out is None else None, ws_bytes,
+                               _stream(stream)), "dsv4_index_topk")
+    return idx, counts
+
+
+def dsv4_hybrid_sparse_attn(Q: torch.Tensor, pool: torch.Tensor, kv_row_off: torch.Tensor,
+                            idx: Optional[torch.Tensor], counts: Optional[torch.Tensor],
+                            local: torch.Tensor, q_pos0: torch.Tensor, m: int, w: int,
+                            sink: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                            O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            want_lse: bool = True, stream=None):
+    """Hybrid shared-KV MQA. Q [B, nq, H, c]; pool [rows, c]; local [B, R, c].
+
+    idx/counts: int32 [B, nq, k] / [B, nq] (CSA) or None (HCA dense read with ratio m).
+    Returns (O [B, nq, H, c], lse fp32 [B, nq, H] or None).
+    """
+    _dev(Q, "Q"), _dev(pool, "pool", Q.dtype), _dev(local, "local", Q.dtype)
+    _dev(kv_row_off, "kv_row_off", torch.int64), _dev(q_pos0, "q_pos0", torch.int32)
+    B, nq, H, c = Q.shape
+    R = local.shape[1]
+    k = 0
+    idx_p = None
+    if idx is not None:
+        _dev(idx, "idx", torch.int32), _dev(counts, "counts", torch.int32)
+        k = idx.shape[-1]
+        # k == 0 (window only): torch gives an empty tensor a NULL pointer, which the ABI
+        # reads as the dense mode; hand over a valid pointer that is never dereferenced.
+        idx_p = _ptr(idx) if idx.numel() > 0 else _ptr(counts)
+    if sink is not None:
+        _dev(sink, "sink", torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(c)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty(B, nq, H, dtype=torch.float32, device=Q.device)
+    _check(lib.dsv4_hybrid_sparse_attn(_code(Q.dtype), _ptr(Q), _ptr(pool), pool.shape[0],
+                                       _ptr(kv_row_off), idx_p, _ptr(counts), k, _ptr(local),
+                                       R, _ptr(q_pos0), B, nq, H, c, m, w, _ptr(sink),
+                                       float(scale), _ptr(O), _ptr(lse), _stream(stream)),
+           "dsv4_hybrid_sparse_attn")
+    return O, lse
+
+
+def dsv4_check_errors(stream=None):
+    """Synchronise the stream and raise DSV4Error if a kernel flagged a device-side error."""
+    _check(lib.dsv4_check_errors(_stream(stream)), "dsv4_check_errors")

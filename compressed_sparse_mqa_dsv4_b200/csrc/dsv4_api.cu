@@ -1,0 +1,187 @@
+// C ABI of the dsv4 library: status handling, argument validation and dispatch of the
+// indexer / attention entry points (compress and FP4 quantisation live beside their
+// kernels). Declarations and the contract of every entry point are in include/dsv4.h.
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "attn_common.cuh"
+#include "index_common.cuh"
+
+namespace dsv4 {
+
+__device__ int g_status = 0;
+
+static thread_local std::string t_last_error;
+
+int fail(int status, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return status;
+}
+
+int launch_status(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return DSV4_OK;
+}
+
+static long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
+
+}  // namespace dsv4
+
+using namespace dsv4;
+
+extern "C" int dsv4_abi_version(void) { return 1; }
+
+extern "C" const char* dsv4_status_string(int s) {
+  switch (s) {
+    case DSV4_OK: return "ok";
+    case DSV4_ERR_INVALID_ARG: return "invalid argument";
+    case DSV4_ERR_UNSUPPORTED: return "unsupported";
+    case DSV4_ERR_CUDA: return "CUDA error";
+    case DSV4_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case DSV4_ERR_DEVICE_BOUNDS: return "device-side index out of range (skipped)";
+    case DSV4_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" const char* dsv4_last_error_message(void) { return t_last_error.c_str(); }
+
+extern "C" int dsv4_check_errors(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "dsv4_check_errors: %s", cudaGetErrorString(e));
+  int word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_status, sizeof(int));
+  if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "dsv4_check_errors: %s", cudaGetErrorString(e));
+  if (word != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "dsv4_check_errors: %s", cudaGetErrorString(e));
+    return fail(word, "device status word: %s", dsv4_status_string(word));
+  }
+  return DSV4_OK;
+}
+
+// ----------------------------------------------------------------------------- indexer
+
+static long long scores_ld_for(int max_entries) { return round_up(max_entries > 0 ? max_entries : 1, 4); }
+
+static const long long kScoreChunkBytes = 256ll << 20;
+
+extern "C" size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k) {
+  (void)k;
+  if (B <= 0 || nq <= 0 || max_entries <= 0) return 0;
+  const long long ld = scores_ld_for(max_entries);
+  const long long total = (long long)B * nq;
+  long long rows = kScoreChunkBytes / (ld * 4);
+  if (rows < 1) rows = 1;
+  if (rows > total) rows = total;
+  return (size_t)round_up(rows * ld * 4, 256);
+}
+
+extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_scales,
+                               const float* w, const void* KI, const uint8_t* KI_scales,
+                               int64_t ki_rows, const int64_t* kv_row_off,
+                               const int32_t* q_pos0, int B, int nq, int H_I, int c_I, int m,
+                               int k, int max_entries, int32_t* idx, int32_t* counts,
+                               float* scores_out, int64_t scores_ld, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (qdtype != DSV4_F32 && qdtype != DSV4_BF16 && qdtype != DSV4_FP4)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_index_topk: qdtype %d", qdtype);
+  if (B < 0 || nq < 0 || H_I < 1 || c_I < 16 || c_I % 16 != 0 || m < 1 || k < 0 || k > 4096 ||
+      max_entries < 0 || ki_rows < 0)
+    return fail(DSV4_ERR_INVALID_ARG,
+                "dsv4_index_topk: bad sizes B=%d nq=%d H_I=%d c_I=%d m=%d k=%d max_entries=%d",
+                B, nq, H_I, c_I, m, k, max_entries);
+  if (qdtype == DSV4_FP4 && (c_I % 64 != 0 || !qI_scales || !KI_scales))
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_index_topk: FP4 needs c_I %% 64 == 0 and scale arrays");
+  if ((long long)B * nq == 0 || k == 0) {
+    if ((long long)B * nq > 0 && counts) {
+      cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)B * nq, (cudaStream_t)stream);
+      if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "dsv4_index_topk: %s", cudaGetErrorString(e));
+    }
+    return DSV4_OK;
+  }
+  if (!qI || !w || !KI || !kv_row_off || !q_pos0 || !idx || !counts)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_index_topk: NULL pointer");
+  IndexArgs a;
+  a.qdtype = qdtype; a.qI = qI; a.qI_scales = qI_scales; a.w = w; a.KI = KI;
+  a.KI_scales = KI_scales; a.ki_rows = ki_rows; a.kv_row_off = kv_row_off; a.q_pos0 = q_pos0;
+  a.B = B; a.nq = nq; a.H_I = H_I; a.c_I = c_I; a.m = m; a.k = k; a.max_e = max_entries;
+  a.idx = idx;
+  a.counts = counts;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int total = B * nq;
+  int chunk;
+  if (scores_out) {
+    if (scores_ld < max_entries)
+      return fail(DSV4_ERR_INVALID_ARG, "dsv4_index_topk: scores_ld %lld < max_entries %d",
+                  (long long)scores_ld, max_entries);
+    a.scores = scores_out; a.scores_ld = scores_ld > 0 ? scores_ld : 1;
+    chunk = total;
+  } else {
+    const long long ld = scores_ld_for(max_entries);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+      return fail(DSV4_ERR_WORKSPACE, "dsv4_index_topk: workspace missing or not 256-byte aligned");
+    const long long rows = (long long)workspace_bytes / (ld * 4);
+    if (rows < 1)
+      return fail(DSV4_ERR_WORKSPACE, "dsv4_index_topk: workspace %zu bytes < one score row (%lld)",
+                  workspace_bytes, ld * 4);
+    a.scores = reinterpret_cast<float*>(workspace); a.scores_ld = ld;
+    chunk = (int)(rows < total ? rows : total);
+  }
+  for (int q0 = 0; q0 < total; q0 += chunk) {
+    const int qn = total - q0 < chunk ? total - q0 : chunk;
+    a.score_q0 = scores_out ? 0 : q0;
+    bool used = false;
+    int s = launch_index_scores_tc(a, q0, qn, max_entries, st, &used);
+    if (s != DSV4_OK) return s;
+    if (!used) {
+      s = launch_index_scores_simt(a, q0, qn, max_entries, st);
+      if (s != DSV4_OK) return s;
+    }
+    s = launch_topk(a, q0, qn, st);
+    if (s != DSV4_OK) return s;
+  }
+  return DSV4_OK;
+}
+
+// ----------------------------------------------------------------------------- attention
+
+extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* pool,
+                                       int64_t pool_rows, const int64_t* kv_row_off,
+                                       const int32_t* idx, const int32_t* counts, int k,
+                                       const void* local, int R, const int32_t* q_pos0, int B,
+                                       int nq, int H, int c, int m, int w, const float* sink,
+                                       float scale, void* O, float* lse, void* stream) {
+  if (dtype != DSV4_F32 && dtype != DSV4_BF16)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_hybrid_sparse_attn: dtype %d", dtype);
+  if (B < 0 || nq < 0 || H < 1 || c < 1 || m < 1 || w < 1 || R < 1 || pool_rows < 0 ||
+      (idx && k < 0))
+    return fail(DSV4_ERR_INVALID_ARG,
+                "dsv4_hybrid_sparse_attn: bad sizes B=%d nq=%d H=%d c=%d m=%d w=%d R=%d k=%d", B,
+                nq, H, c, m, w, R, k);
+  if ((dtype == DSV4_BF16 && c % 8 != 0) || (dtype == DSV4_F32 && c % 4 != 0))
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_hybrid_sparse_attn: c=%d not a multiple of the 16-byte vector", c);
+  if ((long long)B * nq == 0) return DSV4_OK;
+  if (!Q || !local || !kv_row_off || !q_pos0 || !O || (idx && !counts) || (!pool && pool_rows > 0))
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_hybrid_sparse_attn: NULL pointer");
+  AttnArgs a;
+  a.Q = Q; a.pool = pool; a.pool_rows = pool_rows; a.kv_row_off = kv_row_off; a.idx = idx;
+  a.counts = counts; a.k = idx ? k : 0; a.local = local; a.R = R; a.q_pos0 = q_pos0; a.B = B;
+  a.nq = nq; a.H = H; a.c = c; a.m = m; a.w = w; a.sink = sink; a.scale = scale; a.O = O;
+  a.lse = lse;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dtype == DSV4_BF16) {
+    bool used = false;
+    int s = launch_attn_tc(a, st, &used);
+    if (s != DSV4_OK || used) return s;
+  }
+  return launch_attn_simt(a, dtype, st);
+}

@@ -1,0 +1,69 @@
+// Shared declarations of the indexer / top-k kernels.
+#pragma once
+#include "dsv4_common.cuh"
+
+namespace dsv4 {
+
+struct IndexArgs {
+  int qdtype;
+  const void* qI;
+  const uint8_t* qI_scales;
+  const float* w;
+  const void* KI;
+  const uint8_t* KI_scales;
+  long long ki_rows;
+  const int64_t* kv_row_off;
+  const int32_t* q_pos0;
+  int B, nq, H_I, c_I, m, k;
+  int max_e;           // score row capacity: queries with more entries are clamped + flagged
+  int32_t* idx;
+  int32_t* counts;
+  float* scores;       // score rows of queries [score_q0, score_q0 + rows)
+  long long scores_ld;
+  int score_q0;        // global query id of score row 0
+};
+
+// Completed entries of query (b, i), clamped to the score-row capacity (flagged).
+__device__ __forceinline__ int visible_entries(const IndexArgs& a, int b, int i) {
+  const long long t = (long long)a.q_pos0[b] + i;
+  long long Et = (t + 1) / a.m;
+  if (Et < 0) Et = 0;
+  if (Et > a.max_e) {
+    flag_status(DSV4_ERR_DEVICE_BOUNDS);
+    Et = a.max_e;
+  }
+  return (int)Et;
+}
+
+// e4m3 byte -> float (exact)
+__device__ __forceinline__ float e4m3_decode(uint32_t b) {
+  const uint32_t e = (b >> 3) & 15u, mt = b & 7u;
+  float v = e == 0 ? (float)mt * 0x1p-9f : (float)(8u + mt) * exp2f((float)e - 10.f);
+  return (b & 0x80u) ? -v : v;
+}
+
+__device__ __forceinline__ float e2m1_decode(uint32_t nib) {
+  const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
+  const float v = mag[nib & 7u];
+  return (nib & 8u) ? -v : v;
+}
+
+// Element d of row `row` of an indexer operand, decoded to fp32.
+template <int QD>
+__device__ __forceinline__ float load_elem(const void* p, const uint8_t* scales, long long row,
+                                           int d, int cols) {
+  if (QD == DSV4_F32) return reinterpret_cast<const float*>(p)[row * cols + d];
+  if (QD == DSV4_BF16)
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[row * cols + d]);
+  const uint8_t byte = reinterpret_cast<const uint8_t*>(p)[row * (cols / 2) + d / 2];
+  const uint32_t nib = (d & 1) ? (byte >> 4) : (byte & 15u);
+  return e2m1_decode(nib) * e4m3_decode(scales[row * (cols / 16) + d / 16]);
+}
+
+int launch_index_scores_simt(const IndexArgs& a, int q_begin, int q_count, int max_e,
+                             cudaStream_t st);
+int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max_e,
+                           cudaStream_t st, bool* used);
+int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
+
+}  // namespace dsv4

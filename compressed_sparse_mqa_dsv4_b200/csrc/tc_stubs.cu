@@ -1,0 +1,14 @@
+// Placeholder tensor-core launchers: report "not used" so the CUDA-core kernels run.
+#include "attn_common.cuh"
+#include "index_common.cuh"
+
+namespace dsv4 {
+int launch_index_scores_tc(const IndexArgs&, int, int, int, cudaStream_t, bool* used) {
+  *used = false;
+  return DSV4_OK;
+}
+int launch_attn_tc(const AttnArgs&, cudaStream_t, bool* used) {
+  *used = false;
+  return DSV4_OK;
+}
+}  // namespace dsv4

@@ -1,0 +1,175 @@
+/*
+ * dsv4.h -- C ABI of the DeepSeek-V4 hybrid CSA/HCA attention hot path on NVIDIA B200
+ * (sm_100a).
+ *
+ * The operations are defined on the page "CSA And HCA: Definition, State, And Cost
+ * Model" (cited below as [CSA-DEF] with its section) and, for the per-query valid-count
+ * idea, on pypto-lib PR #834 ("accelerate DeepSeek V4 Flash prefill sparse attention").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller, densely packed,
+ *    row-major, in the layout stated per argument. The library never frees, keeps or
+ *    aliases them beyond the call's stream-ordered execution.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Every
+ *    call only enqueues work; nothing synchronises the host except dsv4_check_errors.
+ *  - The library allocates no device memory. Scratch space comes from a caller
+ *    workspace sized by the matching *_workspace_size function.
+ *  - Return value: a dsv4_status. Argument errors are detected on the host before any
+ *    launch (nothing is enqueued then). Launch failures return DSV4_ERR_CUDA. Errors
+ *    that only the device can see (an index outside the visible range, a bounded wait
+ *    that gave up) are recorded in a per-device status word that dsv4_check_errors
+ *    reads and clears; the offending element is skipped, never read out of bounds.
+ *    No call aborts, traps or throws across the ABI. dsv4_last_error_message gives a
+ *    human-readable reason for the last failing call on the calling thread.
+ *  - Positions: query i of sequence b sits at position t = q_pos0[b] + i. Prefill uses
+ *    q_pos0 = 0 and nq = n; decode uses nq = 1 and t = L_b - 1.
+ *  - Pools of several sequences are stacked row-wise; sequence b's compressed entry s is
+ *    row kv_row_off[b] + s.
+ */
+#ifndef DSV4_H
+#define DSV4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dsv4_status {
+  DSV4_OK = 0,
+  DSV4_ERR_INVALID_ARG = 1,    /* bad pointer, size, alignment or combination          */
+  DSV4_ERR_UNSUPPORTED = 2,    /* valid request this build has no kernel for           */
+  DSV4_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed                 */
+  DSV4_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait gave up (device word)     */
+  DSV4_ERR_DEVICE_BOUNDS = 5,  /* an index/offset outside its range was skipped        */
+  DSV4_ERR_WORKSPACE = 6       /* workspace pointer/size too small for the request     */
+} dsv4_status;
+
+typedef enum dsv4_dtype {
+  DSV4_F32 = 0,   /* IEEE binary32                                                    */
+  DSV4_BF16 = 1,  /* bfloat16                                                         */
+  DSV4_FP4 = 2    /* e2m1 codes, 2 per byte (element 2j in the low nibble), plus one
+                     E4M3 (fn) scale byte per 16 consecutive elements                 */
+} dsv4_dtype;
+
+/* Version of this ABI (incremented on any incompatible change). */
+int dsv4_abi_version(void);
+
+/* Static description of a status code. Never NULL. */
+const char* dsv4_status_string(int status);
+
+/* Reason for the last non-OK status returned on the calling thread ("" if none). */
+const char* dsv4_last_error_message(void);
+
+/* Synchronises `stream`, then reads and clears the current device's status word.
+ * Returns DSV4_OK, DSV4_ERR_DEVICE_TIMEOUT, DSV4_ERR_DEVICE_BOUNDS or DSV4_ERR_CUDA. */
+int dsv4_check_errors(void* stream);
+
+/*
+ * dsv4_compress -- learned compressor, [CSA-DEF] s2.1 (CSA, overlap = 1) and s2.2
+ * (HCA, overlap = 0); the CSA indexer keys are a second instance ([CSA-DEF] s3.1).
+ *
+ * For every sequence b, entry i < floor(n/m) and channel ch, one softmax over positions
+ * (per channel) of the logits Z + bias, then the weighted sum of the entry stream C:
+ *   positions = block i from stream a (bias[0]) and, when overlap and i > 0, block i-1
+ *   from stream b (bias[1]). For i = 0 the preceding block has zero weight. The
+ *   trailing incomplete block (n mod m tokens) is never pooled.
+ *
+ *   dtype  DSV4_F32 or DSV4_BF16: element type of C, Z and out (math is fp32).
+ *   C, Z   [B, n, S*c] with S = 1 + overlap; columns [0,c) = stream a, [c,2c) = b.
+ *   bias   fp32 [S, m, c]: bias[0] = B^a, bias[1] = B^b.
+ *   out    [B, floor(n/m), c] (dtype).
+ *   Requires B >= 0, n >= 0, c >= 1, m >= 1, overlap in {0,1}. B*n == 0 is a no-op.
+ */
+int dsv4_compress(int dtype, const void* C, const void* Z, const float* bias, void* out,
+                  int B, int n, int c, int m, int overlap, void* stream);
+
+/*
+ * dsv4_quantize_fp4 -- FP4 indexer operands ([CSA-DEF] s3.1 and s8: the indexer Q/K are
+ * multiplied in 4-bit floating point). Per group of 16 consecutive elements of a row:
+ *   scale = RNE_E4M3(amax / 6) (fp32 quotient, saturating at 448);
+ *   code  = RNE_e2m1(x / scale) (fp32 quotient, saturating at +-6; IEEE sign, so a
+ *           negative value that rounds to zero is code 0x8); a zero scale gives codes 0.
+ *
+ *   x       bf16 [rows, cols]; cols % 16 == 0; x 16-byte aligned.
+ *   codes   uint8 [rows, cols/2] (element 2j in the low nibble of byte j).
+ *   scales  uint8 [rows, cols/16] (E4M3 fn bytes).
+ */
+int dsv4_quantize_fp4(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows, int cols,
+                      void* stream);
+
+/* Bytes of workspace dsv4_index_topk needs for this request (0 when scores_out is
+ * given, which then serves as the score buffer). max_entries = the largest number of
+ * completed entries any query of the request can see. */
+size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k);
+
+/*
+ * dsv4_index_topk -- lightning-indexer score and per-query TopK, [CSA-DEF] s3.1:
+ *   I_{t,s} = sum_h w_{t,h} * ReLU(qI_{t,h} . KI_s)    for s < floor((t+1)/m)
+ *   S_t     = TopK_s(I_{t,s}, k)
+ * Scores are accumulated in fp32. k_eff = min(k, floor((t+1)/m)) entries are returned,
+ * ordered by score descending and then entry index ascending; slots k_eff..k-1 hold -1.
+ *
+ *   qdtype     DSV4_F32, DSV4_BF16 or DSV4_FP4: element type of qI and KI.
+ *   qI         [B, nq, H_I, c_I] (FP4: codes [B*nq*H_I, c_I/2] + qI_scales [.., c_I/16]).
+ *   w          fp32 [B, nq, H_I] head weights.
+ *   KI         [ki_rows, c_I] keys of all sequences (FP4: codes + KI_scales).
+ *   kv_row_off int64 [B] first KI row of each sequence.
+ *   q_pos0     int32 [B] position of query 0 of each sequence.
+ *   idx        int32 [B, nq, k] output; counts int32 [B, nq] output (= k_eff).
+ *   scores_out optional fp32 [B, nq, scores_ld]: if non-NULL receives I_{t,s} for
+ *              s < floor((t+1)/m) (other columns untouched); scores_ld >= max_entries.
+ *   workspace  device scratch of >= dsv4_index_topk_workspace_size(...) bytes (256-byte
+ *              aligned), or NULL/0 when scores_out is given.
+ *   Requires c_I % 16 == 0 (FP4: c_I % 64 == 0), H_I >= 1, m >= 1, 0 <= k <= 4096.
+ *   Device-checked: kv_row_off[b] + floor((q_pos0[b]+nq)/m) <= ki_rows.
+ */
+int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_scales, const float* w,
+                    const void* KI, const uint8_t* KI_scales, int64_t ki_rows,
+                    const int64_t* kv_row_off, const int32_t* q_pos0,
+                    int B, int nq, int H_I, int c_I, int m, int k, int max_entries,
+                    int32_t* idx, int32_t* counts, float* scores_out, int64_t scores_ld,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * dsv4_hybrid_sparse_attn -- shared-KV MQA over one candidate list per query,
+ * [CSA-DEF] s3.2, s4, s5.1-s5.3:
+ *   A_t = {pool[s] : s in S_t}            (CSA: idx/counts from dsv4_index_topk)
+ *       or {pool[s] : s < floor((t+1)/m)} (HCA dense read: idx == NULL)
+ *     ++ {local[j mod R] : max(0,t-w+1) <= j <= t}
+ *   z_{h,j} = scale * q_{t,h} . A_j ;  a_{h,j} = exp(z_{h,j}) / (sum_u exp(z_{h,u}) + exp(sink_h))
+ *   O_{t,h} = sum_j a_{h,j} A_j ;       LSE_{t,h} = log(sum_u exp(z_{h,u}) + exp(sink_h))
+ * Each candidate row is both key and value for every head. The sink term is omitted
+ * when sink == NULL. Softmax and accumulation are fp32.
+ *
+ *   dtype      DSV4_F32 or DSV4_BF16: element type of Q, pool, local and O.
+ *   Q          [B, nq, H, c].
+ *   pool       [pool_rows, c] compressed entries of all sequences; kv_row_off int64 [B].
+ *   idx        int32 [B, nq, k] selected entries (first counts[b,i] valid) or NULL.
+ *              With k == 0 and a non-NULL idx (never read) the list is the window only.
+ *   counts     int32 [B, nq] or NULL (required when idx != NULL).
+ *   local      [B, R, c] uncompressed local entries; position j lives in slot j mod R
+ *              (prefill: R = n; decode ring: R >= w).
+ *   q_pos0     int32 [B].
+ *   m          compression ratio used for the dense read (idx == NULL); ignored otherwise.
+ *   w          local window, >= 1 (so every candidate list is non-empty).
+ *   sink       fp32 [H] or NULL.  scale: logit scale (1/sqrt(c) in the model).
+ *   O          [B, nq, H, c] (dtype) output.  lse: fp32 [B, nq, H] output or NULL.
+ *   Requires c % 8 == 0 for bf16 (c % 4 for fp32), R >= min(w, q_pos0+nq).
+ *   Device-checked: every used idx value in [0, floor((t+1)/m_csa)) when `m` > 0, and
+ *   every pool row < pool_rows; out-of-range candidates are skipped and flagged.
+ */
+int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* pool, int64_t pool_rows,
+                            const int64_t* kv_row_off, const int32_t* idx,
+                            const int32_t* counts, int k, const void* local, int R,
+                            const int32_t* q_pos0, int B, int nq, int H, int c, int m, int w,
+                            const float* sink, float scale, void* O, float* lse,
+                            void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSV4_H */

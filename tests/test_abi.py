@@ -1,0 +1,71 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol, and rejects
+bad arguments on the host before touching a device. No kernel is launched here."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "compressed_sparse_mqa_dsv4_b200", "libdsv4.so")
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"\b(dsv4_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from compressed_sparse_mqa_dsv4_b200 import build as b
+        b.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+
+
+def test_status_strings_and_version(lib):
+    lib.dsv4_status_string.restype = ctypes.c_char_p
+    for s in range(7):
+        assert lib.dsv4_status_string(s)
+    assert lib.dsv4_status_string(99) == b"unknown status"
+    assert lib.dsv4_abi_version() == 1
+
+
+def test_host_validation_rejects_bad_arguments(lib):
+    lib.dsv4_last_error_message.restype = ctypes.c_char_p
+    P = ctypes.c_void_p
+    # dsv4_compress with m = 0
+    assert lib.dsv4_compress(1, P(16), P(16), P(16), P(16), 1, 8, 8, 0, 1, None) == 1
+    assert b"bad sizes" in lib.dsv4_last_error_message()
+    # empty request is a no-op (no launch)
+    assert lib.dsv4_compress(1, None, None, None, None, 0, 8, 8, 4, 1, None) == 0
+    # FP4 quantiser needs cols % 16 == 0
+    assert lib.dsv4_quantize_fp4(P(16), P(16), P(16), ctypes.c_int64(4), 24, None) == 1
+    # attention: w < 1 rejected
+    args = [1, P(16), P(16), ctypes.c_int64(4), P(16), None, None, 0, P(16), 8, P(16), 1, 1, 64,
+            512, 4, 0, None, ctypes.c_float(1.0), P(16), None, None]
+    assert lib.dsv4_hybrid_sparse_attn(*args) == 1
+    # index top-k: k above the supported maximum
+    lib.dsv4_index_topk.restype = ctypes.c_int
+    a = [1, P(16), None, P(16), P(16), None, ctypes.c_int64(1), P(16), P(16), 1, 1, 64, 128, 4,
+         5000, 8, P(16), P(16), None, ctypes.c_int64(0), P(256), ctypes.c_size_t(1 << 20), None]
+    assert lib.dsv4_index_topk(*a) == 1
+
+
+def test_workspace_size_is_bounded(lib):
+    lib.dsv4_index_topk_workspace_size.restype = ctypes.c_size_t
+    small = lib.dsv4_index_topk_workspace_size(1, 8192, 2048, 512)
+    assert small == 8192 * 2048 * 4
+    big = lib.dsv4_index_topk_workspace_size(1, 131072, 32768, 1024)
+    assert 0 < big <= (256 << 20) and big % 256 == 0

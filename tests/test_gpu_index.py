@@ -1,0 +1,135 @@
+"""GPU parity: dsv4_index_topk (indexer scores + per-query TopK) against the fp64 oracle.
+
+Stage-isolated: q^I, w and K^I come from the seeded generator (FP4 operands are
+quantised by the oracle), so both sides score the same bytes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from parity_util import check_topk_query, sample_positions
+from workloads import Generator, preset
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(shape, nq, rows, seed):
+    g = Generator(seed)
+    qI, w = g.index_queries(shape, nq)
+    KI = g.index_keys(shape, rows)
+    return qI, w, KI
+
+
+def _score_bound(qI64, w64, KI64, t, m):
+    """Worst-case fp32 accumulation bound per entry: 2e-5 * sum_h w_h sum_d |q_hd k_sd|."""
+    E = (t + 1) // m
+    mag = np.abs(qI64) @ np.abs(KI64[:E]).T            # [H_I, E]
+    return 2e-5 * (w64 @ mag) + 1e-30
+
+
+def _run_and_check(dsv4, qI, w, KI, offs, pos0, m, k, positions, qI_sc=None, KI_sc=None,
+                   qI64=None, KI64=None, c_I=None, what=""):
+    B, nq = w.shape[:2]
+    max_e = max((int(p0) + nq) // m for p0 in pos0)
+    scores = torch.full((B, nq, max(max_e, 1)), float("nan"), device="cuda")
+    idx, counts = dsv4.dsv4_index_topk(
+        qI.cuda(), w.cuda(), KI.cuda(), torch.tensor(offs, dtype=torch.int64).cuda(),
+        torch.tensor(pos0, dtype=torch.int32).cuda(), m, k, max_e,
+        qI_scales=None if qI_sc is None else qI_sc.cuda(),
+        KI_scales=None if KI_sc is None else KI_sc.cuda(), c_I=c_I, scores_out=scores)
+    # the same request through the workspace path must give identical indices
+    idx2, counts2 = dsv4.dsv4_index_topk(
+        qI.cuda(), w.cuda(), KI.cuda(), torch.tensor(offs, dtype=torch.int64).cuda(),
+        torch.tensor(pos0, dtype=torch.int32).cuda(), m, k, max_e,
+        qI_scales=None if qI_sc is None else qI_sc.cuda(),
+        KI_scales=None if KI_sc is None else KI_sc.cuda(), c_I=c_I)
+    dsv4.dsv4_check_errors()
+    assert torch.equal(idx, idx2) and torch.equal(counts, counts2)
+    idx, counts, scores = idx.cpu().numpy(), counts.cpu().numpy(), scores.cpu().numpy()
+    qI64 = O.as_f64(qI) if qI64 is None else qI64
+    KI64 = O.as_f64(KI) if KI64 is None else KI64
+    w64 = O.as_f64(w)
+    ties = 0
+    for b, i in positions:
+        t = int(pos0[b]) + i
+        s64 = O.index_scores_query(qI64[b, i], w64[b, i], KI64[offs[b]:], t, m)
+        bound = _score_bound(qI64[b, i], w64[b, i], KI64[offs[b]:], t, m)
+        ties += check_topk_query(idx[b, i], counts[b, i], s64, k, scores[b, i], bound,
+                                 f"{what} b={b} t={t}")
+    return ties
+
+
+def test_index_tiny_fp32(dsv4):
+    shape = preset("tiny_csa")
+    qI, w, KI = _inputs(shape, shape.n, shape.n // shape.m, 0)
+    pos = [(0, i) for i in range(shape.n)]
+    _run_and_check(dsv4, qI, w, KI, [0], [0], shape.m, shape.k, pos, what="tiny")
+
+
+@pytest.mark.parametrize("n,k,HI,cI", [(300, 8, 4, 32), (523, 64, 8, 64), (97, 200, 2, 16),
+                                       (4 * 300 + 3, 128, 64, 128)])
+def test_index_ragged_bf16(dsv4, n, k, HI, cI):
+    shape = preset("flash_csa_prefill", n=n, k=k, H_I=HI, c_I=cI)
+    qI, w, KI = _inputs(shape, n, n // 4, n + k)
+    pos = [(0, i) for i in range(n)]
+    _run_and_check(dsv4, qI, w, KI, [0], [0], 4, k, pos, what=f"n={n} k={k}")
+
+
+def test_index_batched_offsets_decode_like(dsv4):
+    """Several sequences stacked in one key pool, one query each at the sequence end."""
+    shape = preset("flash_csa_prefill", B=5)
+    lens = [7, 130, 2048 + 3, 4097, 1]
+    rows = [L // 4 for L in lens]
+    offs = list(np.concatenate([[0], np.cumsum(rows)[:-1]]).astype(np.int64))
+    g = Generator(9)
+    qI, w = g.index_queries(shape, 1)
+    KI = g.index_keys(shape, int(sum(rows)) + 1)
+    pos0 = [L - 1 for L in lens]
+    _run_and_check(dsv4, qI, w, KI, offs, pos0, 4, 512, [(b, 0) for b in range(5)],
+                   what="decode-like")
+
+
+def test_index_long_rows_radix_path(dsv4):
+    """Rows far longer than k (radix select) with many exact ties (quantised keys)."""
+    shape = preset("flash_csa_prefill", H_I=4, c_I=16)
+    g = Generator(11)
+    E = 20000
+    KI = (g.normal("KI", (E + 1, 16), 1.0) * 2).round().clamp(-3, 3).to(torch.bfloat16)
+    qI = (g.normal("qI", (1, 2, 4, 16), 1.0)).round().to(torch.bfloat16)
+    w = torch.ones(1, 2, 4)
+    pos0 = [4 * E - 2]
+    _run_and_check(dsv4, qI, w, KI, [0], pos0, 4, 1000, [(0, 0), (0, 1)], what="radix ties")
+
+
+def test_index_flash_full_sampled(dsv4):
+    """V4-Flash shape: n=8192, H_I=64, c_I=128, k=512; every query run, a sample compared."""
+    shape = preset("flash_csa_prefill")
+    qI, w, KI = _inputs(shape, shape.n, shape.n // shape.m, 1)
+    pos = [(0, t) for t in sample_positions(shape.n, 4, extra=[2046, 2047, 2048, 2051, 4095])]
+    _run_and_check(dsv4, qI, w, KI, [0], [0], 4, 512, pos, what="flash")
+
+
+def test_index_fp4(dsv4):
+    """FP4 operands (e2m1 + E4M3 per 16): the oracle scores the same dequantised values."""
+    shape = preset("pro_csa_prefill", n=4 * 700 + 1)
+    n, E = shape.n, shape.n // 4
+    qI, w, KI = _inputs(shape, n, E, 2)
+    qc, qs = O.quantize_fp4(qI.float().reshape(-1, 128))
+    kc, ks = O.quantize_fp4(KI.float())
+    qI64 = O.dequantize_fp4(qc, qs, 128).reshape(1, n, 64, 128)
+    KI64 = O.dequantize_fp4(kc, ks, 128)
+    qc_t = torch.from_numpy(qc).reshape(1, n, 64, 64)
+    pos = [(0, t) for t in sample_positions(n, 4, extra=[1023, 1024, 2799])]
+    _run_and_check(dsv4, qc_t, w, torch.from_numpy(kc), [0], [0], 4, 256, pos,
+                   qI_sc=torch.from_numpy(qs), KI_sc=torch.from_numpy(ks), qI64=qI64,
+                   KI64=KI64, c_I=128, what="fp4")
+
+
+def test_index_k_zero_and_short(dsv4):
+    shape = preset("tiny_csa")
+    qI, w, KI = _inputs(shape, 10, 2, 4)
+    idx, counts = dsv4.dsv4_index_topk(qI.cuda(), w.cuda(), KI.cuda(),
+                                       torch.zeros(1, dtype=torch.int64).cuda(),
+                                       torch.zeros(1, dtype=torch.int32).cuda(), 4, 0, 2)
+    assert idx.numel() == 0 and (counts.cpu() == 0).all()
