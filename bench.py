@@ -1,0 +1,408 @@
+"""Benchmark of the DeepSeek-V4 hybrid CSA/HCA attention hot path on B200.
+
+One step = one V4-Flash CSA prefill layer over one sequence of 8192 tokens (bf16, H=64,
+c=512, m=4, H_I=64, c_I=128, k=512, w=128, per-head sink):
+    compress(main) -> compress(index keys) -> index scores + top-k -> hybrid attention,
+all through the library's C ABI (libdsv4.so) on the current stream, inputs resident
+in HBM. The L2 is flushed (256 MiB write) before every step, outside the step's events.
+
+Prints one JSON line (rank 0). `--impl reference` times the fp64 CPU oracle instead
+(a bounded sample of the same workload on the host cores).
+
+Multi-GPU: the layer has no exchange step at this size, so N GPUs run N independent
+replicas (weak scaling, no data-path collective); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "flash_csa_prefill"
+METRIC = "prefill tokens/s per CSA/HCA layer"
+UNIT = "tokens/s"
+
+# DRAM traffic of the attention kernel per launch, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the attention
+# sources it was measured on; reported as null once those sources change.
+ATTN_TRAFFIC = {"sources_sha1": None, "bytes_per_launch": None}
+
+
+def _attn_sources_sha1() -> str:
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "compressed_sparse_mqa_dsv4_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.startswith("attn") or f.startswith("tc_"):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def attention_flops(n: int, m: int, k: int, w: int, H: int, c: int) -> float:
+    """4*H*c*sum_t N_t with N_t = min(k, floor((t+1)/m)) + min(w, t+1)."""
+    tot = 0
+    for t in range(n):
+        tot += min(k, (t + 1) // m) + min(w, t + 1)
+    return 4.0 * H * c * tot
+
+
+def index_flops(n: int, m: int, HI: int, cI: int) -> float:
+    return 2.0 * HI * cI * sum((t + 1) // m for t in range(n))
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        hi = max(sm)
+        loaded = [s for s in sm if s >= 0.5 * hi] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CUDA arm
+
+
+def run_cuda(args, rank: int, world: int):
+    import torch
+    import compressed_sparse_mqa_dsv4_b200 as dsv4
+    from workloads import Generator, preset
+
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    s = preset(WORKLOAD)
+    E = s.n // s.m
+    gen = Generator(args.seed + rank)
+    C, Z, bias = gen.compressor_inputs(s, "main")
+    CI, ZI, biasI = gen.compressor_inputs(s, "index")
+    qI, w = gen.index_queries(s)
+    Q = gen.queries(s)
+    local = gen.local_kv(s)
+    sink = gen.sink(s)
+    host = dict(C=C, Z=Z, bias=bias, CI=CI, ZI=ZI, biasI=biasI, qI=qI, w=w, Q=Q, local=local,
+                sink=sink)
+    d = {k: v.to(dev) for k, v in host.items()}
+    off = torch.zeros(1, dtype=torch.int64, device=dev)
+    pos0 = torch.zeros(1, dtype=torch.int32, device=dev)
+    pool = torch.empty(1, E, s.c, dtype=torch.bfloat16, device=dev)
+    KI = torch.empty(1, E, s.c_I, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(1, s.n, s.k, dtype=torch.int32, device=dev)
+    counts = torch.empty(1, s.n, dtype=torch.int32, device=dev)
+    ws = torch.empty(dsv4.dsv4_index_topk_workspace_size(1, s.n, E, s.k), dtype=torch.uint8,
+                     device=dev)
+    Out = torch.empty_like(d["Q"])
+    lse = torch.empty(1, s.n, s.H, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    ev = {}
+
+    def step(inp, record=None):
+        if record is not None:
+            record[0].record(stream)
+        dsv4.dsv4_compress(inp["C"], inp["Z"], inp["bias"], s.m, True, out=pool)
+        dsv4.dsv4_compress(inp["CI"], inp["ZI"], inp["biasI"], s.m, True, out=KI)
+        if record is not None:
+            record[1].record(stream)
+        dsv4.dsv4_index_topk(inp["qI"], inp["w"], KI.view(E, s.c_I), off, pos0, s.m, s.k, E,
+                             idx=idx, counts=counts, workspace=ws)
+        if record is not None:
+            record[2].record(stream)
+        dsv4.dsv4_hybrid_sparse_attn(inp["Q"], pool.view(E, s.c), off, idx, counts,
+                                     inp["local"], pos0, s.m, s.w, inp["sink"], O=Out, lse=lse)
+        if record is not None:
+            record[3].record(stream)
+
+    launches_per_step = 2 + 2 * math.ceil(s.n * ((E + 3) // 4 * 4) * 4 / ws.numel()) + 1
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step(d)
+    dsv4.dsv4_check_errors()
+
+    import torch.distributed as dist
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(d, recs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    dsv4.dsv4_check_errors()
+    step_ms = [r[0].elapsed_time(r[3]) for r in recs]
+    comp_ms = [r[0].elapsed_time(r[1]) for r in recs]
+    index_ms = [r[1].elapsed_time(r[2]) for r in recs]
+    attn_ms = [r[2].elapsed_time(r[3]) for r in recs]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens = s.B * s.n * args.steps * world
+    value = tokens / (total_ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies inside the region
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    out_host = torch.empty(Out.shape, dtype=Out.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_host.numel() * out_host.element_size() + lse_host.numel() * lse_host.element_size()
+    e2e_steps = max(1, min(args.steps, 5))
+    dd = {k: torch.empty_like(v) for k, v in d.items()}
+
+    def e2e_step():
+        for k2, v in pinned.items():
+            dd[k2].copy_(v, non_blocking=True)
+        step(dd)
+        out_host.copy_(Out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = s.B * s.n * e2e_steps * world / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant kernel (attention, tensor-core bound by algorithm)
+    peaks, peak_src = _peaks()
+    flops = attention_flops(s.n, s.m, s.k, s.w, s.H, s.c)
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    achieved = flops / (attn_avg / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = None
+    if ATTN_TRAFFIC["sources_sha1"] == _attn_sources_sha1():
+        traffic = ATTN_TRAFFIC["bytes_per_launch"]
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1)/sqrt(dim) activations, N(0,1) gate logits)",
+        "config": {"workload": "flash_csa_prefill: V4-Flash CSA layer prefill, bf16, B=1, "
+                               "n=8192, H=64, c=512, m=4 (2048 entries), H_I=64, c_I=128, "
+                               "k=512, w=128, sink",
+                   "tokens_per_step": s.B * s.n, "parallelism": f"replicas x{world}",
+                   "l2": "flushed (256 MiB write) before every step, outside the step events"},
+        "breakdown_ms": {"compress": round(statistics.mean(comp_ms), 4),
+                         "index_topk": round(statistics.mean(index_ms), 4),
+                         "attention": round(attn_avg, 4)},
+        "roofline": {"kernel": "hybrid_sparse_attn", "bound": "tensor",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_flops_per_launch": flops,
+                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    return res
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_inputs(seed: int):
+    from workloads import Generator, preset
+    s = preset(WORKLOAD)
+    g = Generator(seed)
+    C, Z, bias = g.compressor_inputs(s, "main")
+    CI, ZI, biasI = g.compressor_inputs(s, "index")
+    qI, w = g.index_queries(s)
+    return dict(s=s, C=C, Z=Z, bias=bias, CI=CI, ZI=ZI, biasI=biasI, qI=qI, w=w,
+                Q=g.queries(s), local=g.local_kv(s), sink=g.sink(s))
+
+
+def run_oracle_sample(inp, n_queries: int):
+    """The fp64 oracle on a bounded sample: both compressors in full, then index top-k and
+    attention for `n_queries` positions spread evenly over the sequence. Returns the
+    per-token time extrapolated to the whole layer."""
+    import oracle as O
+    s = inp["s"]
+    t0 = time.perf_counter()
+    pool = O.compress(inp["C"], inp["Z"], inp["bias"], s.m, True)
+    KI = O.compress(inp["CI"], inp["ZI"], inp["biasI"], s.m, True)
+    t1 = time.perf_counter()
+    E = s.n // s.m
+    qs = [(0, int(t)) for t in
+          sorted(set(int(round(x)) for x in
+                     [i * (s.n - 1) / max(n_queries - 1, 1) for i in range(n_queries)]))]
+    idx, counts = O.index_topk(inp["qI"], inp["w"], KI.reshape(E, -1), [0], [0], s.m, s.k,
+                               queries=qs)
+    O.hybrid_attention(inp["Q"], pool.reshape(E, -1), [0], idx, counts, inp["local"], [0],
+                       s.w, inp["sink"], queries=qs)
+    t2 = time.perf_counter()
+    per_token = (t1 - t0) / s.n + (t2 - t1) / len(qs)
+    return per_token, len(qs), (t1 - t0), (t2 - t1)
+
+
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return None
+    nq = max(8, args.oracle_queries // 8)
+    inp = oracle_inputs(args.seed)
+    times = []
+    for _ in range(min(args.warmup, 1)):
+        run_oracle_sample(inp, 8)
+    for _ in range(args.steps):
+        per_token, used, tc, tq = run_oracle_sample(inp, nq)
+        times.append(per_token)
+    per_token = statistics.mean(times)
+    cores = _blas_threads()
+    sample = (f"both compressors over all 8192 tokens + index top-k and attention for {nq} "
+              f"query positions evenly spaced over the sequence, per-token time extrapolated "
+              f"to n=8192")
+    value = 1.0 / per_token
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(per_token * 8192 * 1e3, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": "flash_csa_prefill: V4-Flash CSA layer prefill, bf16 inputs, "
+                               "B=1, n=8192, H=64, c=512, m=4, H_I=64, c_I=128, k=512, w=128, "
+                               "sink", "parallelism": "host cores (rank 0 only)"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--oracle-queries", type=int, default=2048)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world != args.gpus and "RANK" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+        return
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_cuda(args, rank, world)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                per_token, used, tc, tq = run_oracle_sample(oracle_inputs(args.seed),
+                                                            args.oracle_queries)
+                res["cpu_baseline"] = {
+                    "value": round(1.0 / per_token, 3), "unit": UNIT, "cores": _blas_threads(),
+                    "kind": "oracle",
+                    "sample": f"fp64 oracle: both compressors over all 8192 tokens ({tc:.1f} s) + "
+                              f"index top-k and attention for {used} evenly spaced queries "
+                              f"({tq:.1f} s); per-token time extrapolated to n=8192"}
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -209,26 +209,29 @@ def hybrid_attention(Q, pool, kv_row_off, idx, counts, local, q_pos0, w: int,
     counts   [B, nq] valid entries per query (CSA) or None
     local    [B, R, c] local ring (R = n for prefill; slot = position mod R)
     q_pos0   [B]: query i of sequence b sits at position t = q_pos0[b] + i
-    queries  optional list of (b, i) pairs to evaluate; default all
-    returns (O [B, nq, H, c], LSE [B, nq, H]); entries not evaluated are NaN.
+    queries  optional list of (b, i) pairs to evaluate
+    returns (O [B, nq, H, c], LSE [B, nq, H]) for all queries, or, when `queries` is
+    given, (O [len(queries), H, c], LSE [len(queries), H]) in the order listed.
     """
-    Q = as_f64(Q)
     pool = as_f64(pool)
     local = as_f64(local)
     B, nq, H, c = Q.shape
     R = local.shape[1]
-    O = np.full((B, nq, H, c), np.nan)
-    LSE = np.full((B, nq, H), np.nan)
-    if queries is None:
+    listed = queries is not None
+    if not listed:
         queries = [(b, i) for b in range(B) for i in range(nq)]
-    for b, i in queries:
+    O = np.empty((len(queries), H, c))
+    LSE = np.empty((len(queries), H))
+    for q_n, (b, i) in enumerate(queries):
         t = int(q_pos0[b]) + i
         base = int(kv_row_off[b])
         pool_seq = pool[base:]
         row = None if idx is None else np.asarray(idx[b, i])
         cnt = 0 if counts is None else int(counts[b, i])
         A = candidates(pool_seq, row, cnt, local[b], R, t, w, dense_m)
-        O[b, i], LSE[b, i] = attend_query(Q[b, i], A, sink, scale)
+        O[q_n], LSE[q_n] = attend_query(as_f64(Q[b, i]), A, sink, scale)
+    if not listed:
+        return O.reshape(B, nq, H, c), LSE.reshape(B, nq, H)
     return O, LSE
 
 
@@ -240,8 +243,6 @@ def index_topk(qI, w, KI, kv_row_off, q_pos0, m: int, k: int, queries=None,
     row kv_row_off[b]. Returns idx int32 [B, nq, k], counts int32 [B, nq] (and, when
     with_scores, a dict (b, i) -> fp64 score vector over E_t).
     """
-    qI = as_f64(qI)
-    w = as_f64(w)
     KI = as_f64(KI)
     B, nq = qI.shape[:2]
     idx = np.full((B, nq, k), -1, dtype=np.int32)
@@ -251,7 +252,7 @@ def index_topk(qI, w, KI, kv_row_off, q_pos0, m: int, k: int, queries=None,
         queries = [(b, i) for b in range(B) for i in range(nq)]
     for b, i in queries:
         t = int(q_pos0[b]) + i
-        s = index_scores_query(qI[b, i], w[b, i], KI[int(kv_row_off[b]):], t, m)
+        s = index_scores_query(as_f64(qI[b, i]), as_f64(w[b, i]), KI[int(kv_row_off[b]):], t, m)
         idx[b, i], counts[b, i] = topk_select(s, k)
         if with_scores:
             scores[(b, i)] = s
