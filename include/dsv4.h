@@ -134,6 +134,34 @@ int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_scales, const 
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * dsv4_index_topk_noalloc -- the same indexer score + TopK as dsv4_index_topk, for
+ * callers that cannot allocate device memory (a runtime that only hands out buffers it
+ * planned in advance, plain C code without a device allocator, or a serving loop that
+ * must not call cudaMalloc because it can synchronise the device and fail under
+ * fragmentation). The pages have no counterpart of this entry point; it is a property
+ * of this library's interface only.
+ *
+ * Instead of a caller workspace it uses a fixed 8 MiB scratch array compiled into the
+ * library (a __device__ array that every GPU which loads the library keeps until the
+ * process exits). It allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ * library routine. Arguments and outputs are those of dsv4_index_topk without
+ * scores_out, scores_ld, workspace and workspace_bytes.
+ *   - max_entries above 2,097,152 (one score row larger than the scratch) is rejected
+ *     with DSV4_ERR_INVALID_ARG before anything is enqueued.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array. The scratch holds score rows that
+ *     each call writes before it reads them, so nothing needs to start at zero, but two
+ *     calls whose work overlaps on the GPU (different streams, no ordering between them)
+ *     race on the array and may return wrong indices. Order such calls on one stream.
+ */
+int dsv4_index_topk_noalloc(int qdtype, const void* qI, const uint8_t* qI_scales,
+                            const float* w, const void* KI, const uint8_t* KI_scales,
+                            int64_t ki_rows, const int64_t* kv_row_off, const int32_t* q_pos0,
+                            int B, int nq, int H_I, int c_I, int m, int k, int max_entries,
+                            int32_t* idx, int32_t* counts, void* stream);
+
+/*
  * dsv4_hybrid_sparse_attn -- shared-KV MQA over one candidate list per query,
  * [CSA-DEF] s3.2, s4, s5.1-s5.3:
  *   A_t = {pool[s] : s in S_t}            (CSA: idx/counts from dsv4_index_topk)
