@@ -1,0 +1,54 @@
+// Host helpers of the tensor-core kernels: tensor-map encoding through the driver entry
+// point (no link-time dependency on libcuda) and the bounded-wait spin limit.
+#include <cudaTypedefs.h>
+
+#include <cstdlib>
+#include <mutex>
+
+#include "tc_common.cuh"
+
+namespace dsv4 {
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+int encode_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                         int elem_bytes, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                         uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  auto fn = get_encode_fn();
+  if (!fn) return fail(DSV4_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (cuuint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(DSV4_ERR_INVALID_ARG,
+                "cuTensorMapEncodeTiled failed (%d): base %p, %llu x %llu, box %u x %u", (int)r,
+                base, (unsigned long long)rows, (unsigned long long)cols, box_rows, box_cols);
+  return DSV4_OK;
+}
+
+uint32_t spin_limit() {
+  static uint32_t lim = [] {
+    const char* e = std::getenv("DSV4_SPIN_LIMIT");
+    long long v = e ? std::atoll(e) : 0;
+    return v > 0 ? (uint32_t)v : (uint32_t)(1u << 22);
+  }();
+  return lim;
+}
+
+}  // namespace dsv4

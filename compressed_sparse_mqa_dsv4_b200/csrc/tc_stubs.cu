@@ -7,8 +7,4 @@ int launch_index_scores_tc(const IndexArgs&, int, int, int, cudaStream_t, bool* 
   *used = false;
   return DSV4_OK;
 }
-int launch_attn_tc(const AttnArgs&, cudaStream_t, bool* used) {
-  *used = false;
-  return DSV4_OK;
-}
 }  // namespace dsv4

@@ -73,14 +73,22 @@ def test_attn_tiny_fp32_sink(dsv4):
     _case(dsv4, B=2, nq=100, H=4, c=64, m=4, w=16, k=8, dtype="f32", sink=True, what="sink")
 
 
-@pytest.mark.parametrize("H,nq,k,w", [(64, 37, 16, 8), (128, 20, 64, 128), (16, 300, 32, 5)])
-def test_attn_bf16_ragged(dsv4, H, nq, k, w):
+@pytest.fixture(params=["tensor_cores", "cuda_cores"])
+def attn_path(request, monkeypatch):
+    """Run a case on the tcgen05 kernel (bf16, c=512, H%64==0) and on the CUDA-core kernel."""
+    monkeypatch.setenv("DSV4_FORCE_SIMT", "1" if request.param == "cuda_cores" else "0")
+    return request.param
+
+
+@pytest.mark.parametrize("H,nq,k,w", [(64, 37, 16, 8), (128, 20, 64, 128), (16, 300, 32, 5),
+                                      (64, 1, 4, 1), (64, 131, 512, 128)])
+def test_attn_bf16_ragged(dsv4, attn_path, H, nq, k, w):
     _case(dsv4, B=2, nq=nq, H=H, c=512, m=4, w=w, k=k, dtype="bf16", sink=True, seed=H + nq,
-          what=f"H={H} nq={nq}")
+          what=f"{attn_path} H={H} nq={nq}")
 
 
 @pytest.mark.parametrize("scale_mul", [1.0, 4.0])
-def test_attn_bf16_stress_logits(dsv4, scale_mul):
+def test_attn_bf16_stress_logits(dsv4, attn_path, scale_mul):
     """Unscaled N(0,1) activations: logits with std 1 and 4 (peaky softmax)."""
     _case(dsv4, B=1, nq=600, H=64, c=512, m=4, w=128, k=64, dtype="bf16", sink=True,
           q_std=1.0, kv_std=1.0, scale=scale_mul / math.sqrt(512), seed=7,
@@ -91,12 +99,12 @@ def test_attn_k_zero_window_only(dsv4):
     _case(dsv4, B=1, nq=50, H=8, c=64, m=4, w=7, k=0, dtype="f32", what="k=0")
 
 
-def test_attn_hca_dense_bf16(dsv4):
+def test_attn_hca_dense_bf16(dsv4, attn_path):
     _case(dsv4, B=2, nq=128 * 5 + 17, H=64, c=512, m=128, w=128, k=0, dtype="bf16", dense=True,
           q_std=1.0, what="hca dense")
 
 
-def test_attn_decode_ring(dsv4):
+def test_attn_decode_ring(dsv4, attn_path):
     """Decode: one query per sequence at t = L-1, local ring of R = w slots, stacked pools."""
     lens = [1, 5, 127, 128, 129, 3000, 70000]
     B = len(lens)
@@ -106,7 +114,7 @@ def test_attn_decode_ring(dsv4):
           pos0=[L - 1 for L in lens], R=128, q_std=1.0, what="decode hca")
 
 
-def test_attn_flash_full_sampled(dsv4):
+def test_attn_flash_full_sampled(dsv4, attn_path):
     """V4-Flash CSA prefill shape (n=8192, H=64, c=512, k=512, w=128, sink) -- sampled."""
     s = preset("flash_csa_prefill")
     pos = [(0, t) for t in sample_positions(s.n, 4, extra=[2046, 2047, 2048, 127, 128])]
@@ -114,9 +122,9 @@ def test_attn_flash_full_sampled(dsv4):
           kv_std=1 / math.sqrt(512), positions=pos, what="flash full")
 
 
-def test_attn_out_of_range_index_is_flagged(dsv4):
+def test_attn_out_of_range_index_is_flagged(dsv4, attn_path):
     """An index outside the visible range is skipped and reported, never read."""
-    B, nq, H, c = 1, 8, 16, 64
+    B, nq, H, c = 1, 8, 64, 512
     Q = torch.randn(B, nq, H, c, device="cuda").to(torch.bfloat16)
     pool = torch.randn(4, c, device="cuda").to(torch.bfloat16)
     local = torch.randn(B, nq, c, device="cuda").to(torch.bfloat16)
