@@ -67,16 +67,27 @@ def test_index_tiny_fp32(dsv4):
     _run_and_check(dsv4, qI, w, KI, [0], [0], shape.m, shape.k, pos, what="tiny")
 
 
+@pytest.fixture(params=["tensor_cores", "cuda_cores"])
+def index_path(request, monkeypatch):
+    """Run a case on the tcgen05 score kernel (bf16, H_I=64, c_I=128) and the CUDA-core one."""
+    monkeypatch.setenv("DSV4_FORCE_SIMT", "1" if request.param == "cuda_cores" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("n,k,HI,cI", [(300, 8, 4, 32), (523, 64, 8, 64), (97, 200, 2, 16),
-                                       (4 * 300 + 3, 128, 64, 128)])
-def test_index_ragged_bf16(dsv4, n, k, HI, cI):
+                                       (4 * 300 + 3, 128, 64, 128), (4 * 5000 + 2, 300, 64, 128),
+                                       (7, 4, 64, 128)])
+def test_index_ragged_bf16(dsv4, index_path, n, k, HI, cI):
     shape = preset("flash_csa_prefill", n=n, k=k, H_I=HI, c_I=cI)
     qI, w, KI = _inputs(shape, n, n // 4, n + k)
-    pos = [(0, i) for i in range(n)]
-    _run_and_check(dsv4, qI, w, KI, [0], [0], 4, k, pos, what=f"n={n} k={k}")
+    if n <= 2000:
+        pos = [(0, i) for i in range(n)]
+    else:
+        pos = [(0, t) for t in sample_positions(n, 4, extra=[4 * 4096 - 1, 4 * 4096, 4 * k])]
+    _run_and_check(dsv4, qI, w, KI, [0], [0], 4, k, pos, what=f"{index_path} n={n} k={k}")
 
 
-def test_index_batched_offsets_decode_like(dsv4):
+def test_index_batched_offsets_decode_like(dsv4, index_path):
     """Several sequences stacked in one key pool, one query each at the sequence end."""
     shape = preset("flash_csa_prefill", B=5)
     lens = [7, 130, 2048 + 3, 4097, 1]
@@ -102,7 +113,7 @@ def test_index_long_rows_radix_path(dsv4):
     _run_and_check(dsv4, qI, w, KI, [0], pos0, 4, 1000, [(0, 0), (0, 1)], what="radix ties")
 
 
-def test_index_flash_full_sampled(dsv4):
+def test_index_flash_full_sampled(dsv4, index_path):
     """V4-Flash shape: n=8192, H_I=64, c_I=128, k=512; every query run, a sample compared."""
     shape = preset("flash_csa_prefill")
     qI, w, KI = _inputs(shape, shape.n, shape.n // shape.m, 1)
