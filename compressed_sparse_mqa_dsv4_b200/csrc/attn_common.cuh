@@ -78,5 +78,6 @@ __device__ __forceinline__ long long candidate_row(const AttnArgs& a, const Cand
 
 int launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
 int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used);
+int launch_attn_tc2(const AttnArgs& a, cudaStream_t st, bool* used);
 
 }  // namespace dsv4

@@ -180,7 +180,9 @@ extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* poo
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == DSV4_BF16) {
     bool used = false;
-    int s = launch_attn_tc(a, st, &used);
+    int s = launch_attn_tc2(a, st, &used);
+    if (s != DSV4_OK || used) return s;
+    s = launch_attn_tc(a, st, &used);
     if (s != DSV4_OK || used) return s;
   }
   return launch_attn_simt(a, dtype, st);

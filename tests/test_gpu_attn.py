@@ -73,10 +73,12 @@ def test_attn_tiny_fp32_sink(dsv4):
     _case(dsv4, B=2, nq=100, H=4, c=64, m=4, w=16, k=8, dtype="f32", sink=True, what="sink")
 
 
-@pytest.fixture(params=["tensor_cores", "cuda_cores"])
+@pytest.fixture(params=["tc_cluster", "tc_single_cta", "cuda_cores"])
 def attn_path(request, monkeypatch):
-    """Run a case on the tcgen05 kernel (bf16, c=512, H%64==0) and on the CUDA-core kernel."""
+    """Run a case on each attention kernel: the 2-CTA-cluster tcgen05 kernel, the single-CTA
+    tcgen05 kernel (both bf16, c=512, H%64==0) and the CUDA-core kernel."""
     monkeypatch.setenv("DSV4_FORCE_SIMT", "1" if request.param == "cuda_cores" else "0")
+    monkeypatch.setenv("DSV4_ATTN_V1", "1" if request.param == "tc_single_cta" else "0")
     return request.param
 
 
