@@ -1,5 +1,5 @@
 // Hybrid shared-KV MQA on the 5th-generation tensor cores, channel-split over a 2-CTA
-// cluster, persistent.
+// cluster, persistent, with cp.async row gathers.
 //
 // "CSA And HCA: Definition, State, And Cost Model": s3.2/s4 every candidate row is both key
 // and value for all heads; s5.1 one candidate list (selected or all completed compressed
@@ -10,18 +10,23 @@
 // time; CTA r holds channels [256r, 256r+256) of every candidate row and of Q, so each SM
 // keeps half of a 128-slot KV block and can double-buffer it:
 //   GEMM1  S_r^T[128 slots x 64 heads] = KV_r[slots x 256] . Q_r[heads x 256]^T   (partial)
-//   exchange over DSMEM: CTA r owns heads [32r, 32r+32); it sends the peer its partial for
-//          the peer's heads and adds the peer's partial for its own heads
-//   softmax for the 32 owned heads (block max, conditional rescale, exp2), P^T columns of
-//          those heads written to both CTAs' shared memory; rescale factors exchanged
-//   GEMM2  O_r^T[256 channels x 64 heads] += KV_r^T . P^T                             (full)
-// Both GEMMs use M = 128 (full tensor-core rate): slots for GEMM1, channels for GEMM2. The
-// same swizzled KV stage is the K-major A operand of GEMM1 and the MN-major A of GEMM2.
-// GEMM1 of block j+1 overlaps the softmax of block j (two S buffers, two KV stages).
+//   exchange: each CTA sends its partial S (all heads) to the other over DSMEM and adds the
+//          other's, so both hold the identical full S and run the identical softmax; each
+//          writes the full P^T into its own shared memory (no further exchange)
+//   GEMM2  O_r^T[256 channels x 64 heads] += KV_r^T . P^T
+// Both GEMMs use M = 128 (full tensor-core rate). The same swizzled KV stage is the K-major
+// A operand of GEMM1 and the MN-major A operand of GEMM2. GEMM1 of block j+1 overlaps the
+// softmax of block j (two S buffers, two KV stages).
 //
-// Warps: 0-3 softmax/epilogue (thread t = TMEM lane t), 4 producer (Q by 2D TMA, rows by
-// TMA row gather), 5 MMA issuer and TMEM owner. Every wait is bounded; a cluster barrier at
+// Candidate rows are gathered with 16-byte cp.async by three producer warps (one 512-byte
+// half-row per warp instruction): on B200 that moves a gathered block about 3x faster than
+// TMA row gathers. Q uses 2D TMA.
+//
+// Warps: 0-7 softmax/epilogue (warp w reads TMEM lane quadrant w%4 for heads 32(w/4)..+31),
+// 8-10 producer, 11 MMA issuer and TMEM owner (12 warps: 3 per SM sub-partition, so up to
+// 168 registers per thread). Every wait is bounded; a cluster barrier at
 // the end keeps both CTAs alive until neither can touch the other's shared memory.
+#include <cstdio>
 #include <cstdlib>
 
 #include "attn_common.cuh"
@@ -33,30 +38,33 @@ namespace {
 constexpr int A2_C = 512;               // channels of a row
 constexpr int A2_CH = 256;              // channels per CTA
 constexpr int A2_H = 64;                // heads per item
-constexpr int A2_HO = 32;               // heads owned per CTA
 constexpr int A2_BLK = 128;             // candidate slots per block
 constexpr int A2_KCH = A2_CH / 64;      // 64-channel chunks per CTA
-constexpr int A2_THREADS = 192;
+constexpr int A2_SOFT = 256;            // softmax threads (8 warps)
+constexpr int A2_PROD = 96;             // producer threads (3 warps)
+constexpr int A2_THREADS = A2_SOFT + A2_PROD + 32;
 constexpr uint32_t T2_S = 0;            // S buffers at columns 0 and 64
 constexpr uint32_t T2_O = 128;          // O^T tiles at 128 + 64 q
 constexpr uint32_t T2_COLS = 256;
-constexpr float TAU2 = 8.f;
+constexpr float TAU2 = 8.f;             // log2-domain max growth tolerated before rescaling
 constexpr float LOG2E2 = 1.4426950408889634f;
 constexpr float LN2_2 = 0.6931471805599453f;
 
 struct Smem2 {
-  uint8_t q[A2_KCH][A2_H * 128];              // 32 KiB
-  uint8_t kv[2][A2_KCH][A2_BLK * 128];        // 128 KiB
-  uint8_t p[2][A2_BLK * 128];                 // 32 KiB, P^T [slots][64 heads], MN-major SW128
-  float xs[2][A2_BLK][A2_HO];                 // 32 KiB, peer's partial S for my heads
-  float red[4][A2_HO];
-  float mcur[A2_HO];
-  float fac[2][A2_H];
-  float inv[2][A2_H];
+  uint8_t q[A2_KCH][A2_H * 128];              // 32 KiB, K-major SW128 [64 heads][64 ch]
+  uint8_t kv[2][A2_KCH][A2_BLK * 128];        // 128 KiB, [128 slots][64 ch] per chunk
+  uint8_t p[A2_BLK * 128];                    // 16 KiB, P^T [slots][64 heads] MN-major SW128;
+                                              // also the O staging tile of the epilogue
+  float xs[A2_BLK][A2_H];                     // 32 KiB, the peer's partial S (swizzled rows)
+  float red[4][A2_H];
+  float mcur[A2_H];
+  float fac[A2_H];
+  float inv[A2_H];
+  uint64_t rowaddr[A2_BLK];                   // global address of each slot's row (producer)
   uint64_t q_full, q_empty;
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t s_full[2], xs_full[2], fac_full[2], p_full[2];
-  uint64_t o_blk[2], inv_full[2], drain;
+  uint64_t s_full[2], xs_full, xs_empty, p_full;
+  uint64_t o_blk[2], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -67,10 +75,10 @@ static_assert(A2_SMEM <= 232448, "shared memory of the cluster attention kernel"
 // Phase timestamps (clock64) of cluster 0, first 4 items, first 8 blocks: a profiling aid
 // compiled only into traced builds.
 __device__ unsigned long long g_attn_trace[2][4][8][32];
-#define A2_TRACE(ev, k_, j_)                                                   \
-  do {                                                                         \
-    if (cluster_id == 0 && (k_) < 4 && (j_) < 8)                               \
-      g_attn_trace[rank][k_][j_][ev] = clock64();                              \
+#define A2_TRACE(ev, k_, j_)                                   \
+  do {                                                         \
+    if (cluster_id == 0 && (k_) < 4 && (j_) < 8)               \
+      g_attn_trace[rank][k_][j_][ev] = clock64();              \
   } while (0)
 #else
 #define A2_TRACE(ev, k_, j_) \
@@ -91,13 +99,20 @@ __device__ __forceinline__ uint32_t mapa(uint32_t local, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_remote_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
-               "r"(v.z), "r"(v.w)
+__device__ __forceinline__ void st_remote_v4(uint32_t addr, float a, float b, float c, float d) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
                : "memory");
 }
-__device__ __forceinline__ void st_remote_f32(uint32_t addr, float v) {
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+// 16-byte store into the peer CTA's shared memory whose completion is counted (in bytes) on
+// the peer's mbarrier; no release fence is needed for the peer to observe it.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d,
+                                            uint32_t remote_bar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+          addr),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+      : "memory");
 }
 __device__ __forceinline__ void arrive_remote(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster_addr)
@@ -130,9 +145,6 @@ __device__ __forceinline__ bool wait_cluster(uint64_t* bar, uint32_t parity, uin
   *abort = 1;
   return false;
 }
-__device__ __forceinline__ void fence_proxy_async_all() {
-  asm volatile("fence.proxy.async;" ::: "memory");
-}
 __device__ __forceinline__ bool bar_red_or2(uint32_t id, uint32_t threads, bool pred) {
   uint32_t r;
   asm volatile(
@@ -142,6 +154,13 @@ __device__ __forceinline__ bool bar_red_or2(uint32_t id, uint32_t threads, bool 
       : "r"((uint32_t)pred), "r"(id), "r"(threads)
       : "memory");
   return r != 0;
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, uint64_t src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar))
+               : "memory");
 }
 
 // Transposing butterfly over 32 per-lane values: lane L ends with the reduction of value L.
@@ -215,11 +234,9 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int item, int h
   return it;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
-    attn_tc2_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q,
-                    const __grid_constant__ CUtensorMap map_pool,
-                    const __grid_constant__ CUtensorMap map_local, int head_groups, int items,
-                    float scale_log2, uint32_t spin) {
+__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
+    attn_tc2_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q, int head_groups,
+                    int items, float scale_log2, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
   Smem2& s = *reinterpret_cast<Smem2*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                        ~uintptr_t(1023));
@@ -232,22 +249,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
     tc::mbar_init(&s.q_full, 1);
     tc::mbar_init(&s.q_empty, 1);
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&s.kv_full[i], 1);
+      tc::mbar_init(&s.kv_full[i], A2_PROD);
       tc::mbar_init(&s.kv_empty[i], 1);
       tc::mbar_init(&s.s_full[i], 1);
-      tc::mbar_init(&s.xs_full[i], 128);
-      tc::mbar_init(&s.fac_full[i], 128);
-      tc::mbar_init(&s.p_full[i], 256);
-      tc::mbar_init(&s.inv_full[i], 128);
+      tc::mbar_init(&s.o_blk[i], 1);
     }
-    tc::mbar_init(&s.o_blk[0], 1);
-    tc::mbar_init(&s.o_blk[1], 1);
+    tc::mbar_init(&s.xs_full, 1);                   // local expect_tx + the peer's st.async bytes
+    tc::mbar_init(&s.xs_empty, 1);                  // one remote arrive per consumed block
+    tc::mbar_init(&s.p_full, A2_SOFT);
     tc::mbar_init(&s.drain, 1);
     s.abort = 0;
     tc::fence_barrier_init();
   }
-  if (tid < A2_HO) s.mcur[tid] = -INFINITY;
-  if (warp == 5) {
+  if (tid < A2_H) s.mcur[tid] = -INFINITY;
+  if (warp == 11) {
     tc::tmem_alloc(&s.tmem_base, T2_COLS);
     tc::tmem_relinquish();
   }
@@ -257,79 +272,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
   tc::tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------------ producer
-    int issued[2] = {0, 0};
-    int q_issued = 0;
-    if (lane == 0) {
-      tc::prefetch_tensormap(&map_q);
-      tc::prefetch_tensormap(&map_pool);
-      tc::prefetch_tensormap(&map_local);
-    }
+  if (warp >= 8 && warp < 11) {
+    // ------------------------------------------------------------------ producer (4 warps)
+    const int pt = tid - A2_SOFT, pw = pt >> 5;
+    // this lane's 16 bytes of a 512-byte half-row: chunk (64 channels) and piece (8 channels)
+    const int piece = lane & 7, chunk = lane >> 3;
+    const uint64_t my_off = (uint64_t)rank * A2_CH * 2 + chunk * 128 + piece * 16;
+    const uint64_t pool_addr = reinterpret_cast<uint64_t>(a.pool);
+    const uint64_t local_addr = reinterpret_cast<uint64_t>(a.local);
     uint32_t G = 0;
     int k = 0;
     bool ok = true;
+    if (pt == 0) tc::prefetch_tensormap(&map_q);
     for (int item = cluster_id; item < items && ok; item += nclusters, ++k) {
       const ItemInfo it = item_info(a, item, head_groups);
-      if (lane == 0) {
+      if (pt == 0) {
         if (k > 0) ok = tc::mbar_wait(&s.q_empty, (uint32_t)((k - 1) & 1), spin, abort);
         if (ok) {
           tc::mbar_arrive_expect_tx(&s.q_full, A2_KCH * A2_H * 128);
           const int qrow = it.qi * a.H + it.hg * A2_H;
           for (int c = 0; c < A2_KCH; ++c)
             tc::tma_load_2d(s.q[c], &map_q, &s.q_full, (int)rank * A2_CH + 64 * c, qrow);
-          q_issued = k + 1;
         }
       }
-      ok = __shfl_sync(0xffffffffu, (int)ok, 0) != 0;
-      for (int j = 0; j < it.nb && ok; ++j, ++G) {
+      ok = !bar_red_or2(4, A2_PROD, !ok);
+      if (!ok) break;
+      for (int j = 0; j < it.nb; ++j, ++G) {
         const int st = G & 1;
-        Slot r[4];
-        bool any_valid = false, bad = false;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          r[u] = slot_of(a, it.cs, it.nc4, j * A2_BLK + 4 * lane + u);
-          any_valid |= r[u].valid;
-          bad |= r[u].bad;
+        // resolve the block's 128 row addresses (one index load per slot)
+        for (int u = pt; u < A2_BLK; u += A2_PROD) {
+          const Slot sl = slot_of(a, it.cs, it.nc4, j * A2_BLK + u);
+          if (sl.bad && rank == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
+          s.rowaddr[u] =
+              (sl.part == 0 && sl.valid)
+                  ? pool_addr + (uint64_t)sl.row * A2_C * 2
+                  : local_addr + (uint64_t)(sl.part == 1 ? sl.row : it.cs.local_base) * A2_C * 2;
         }
-        if (bad && rank == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
-        const CUtensorMap* map = &map_local;
-        int32_t y[4];
-        if (r[0].part == 0 && any_valid) {
-          map = &map_pool;
-          long long fill = 0;
-#pragma unroll
-          for (int u = 3; u >= 0; --u)
-            if (r[u].valid) fill = r[u].row;
-#pragma unroll
-          for (int u = 0; u < 4; ++u) y[u] = (int32_t)(r[u].valid ? r[u].row : fill);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            y[u] = (int32_t)(r[u].part == 1 ? r[u].row : it.cs.local_base);
-        }
-        int w_ok = 1;
-        if (lane == 0 && G >= 2) w_ok = tc::mbar_wait(&s.kv_empty[st], ((G >> 1) - 1) & 1, spin, abort);
-        if (lane == 0) A2_TRACE(0, k, j);
-        ok = __shfl_sync(0xffffffffu, w_ok, 0) != 0;
+        ok = G >= 2 ? tc::mbar_wait(&s.kv_empty[st], ((G >> 1) - 1) & 1, spin, abort) : true;
+        ok = !bar_red_or2(4, A2_PROD, !ok);             // also publishes rowaddr[]
         if (!ok) break;
-        if (lane == 0) tc::mbar_arrive_expect_tx(&s.kv_full[st], A2_KCH * A2_BLK * 128);
-        __syncwarp();
-#pragma unroll
-        for (int c = 0; c < A2_KCH; ++c)
-          tc::tma_gather4(s.kv[st][c] + 4 * lane * 128, map, &s.kv_full[st],
-                          (int)rank * A2_CH + 64 * c, y[0], y[1], y[2], y[3]);
-        if (lane == 0) A2_TRACE(1, k, j);
-        issued[st] = (int)(G >> 1) + 1;
+        if (pt == 0) A2_TRACE(0, k, j);
+        uint8_t* dst_base = s.kv[st][chunk];
+        // warp pw copies rows pw, pw + 3, ...: one 512-byte half-row per warp instruction
+#pragma unroll 4
+        for (int row = pw; row < A2_BLK; row += A2_PROD / 32) {
+          const uint64_t src = s.rowaddr[row] + my_off;
+          cp_async16(tc::smem_u32(dst_base + row * 128 + ((piece ^ (row & 7)) << 4)), src);
+        }
+        cp_async_arrive_noinc(&s.kv_full[st]);
+        if (pt == 0) A2_TRACE(1, k, j);
+        tc::named_barrier(5, A2_PROD);                  // rowaddr[] is rewritten next block
       }
     }
-    if (*abort) {
-      volatile int never = 0;
-      for (int st = 0; st < 2; ++st)
-        if (issued[st] > 0) tc::mbar_wait(&s.kv_full[st], (uint32_t)((issued[st] - 1) & 1), spin, &never);
-      if (lane == 0 && q_issued > 0) tc::mbar_wait(&s.q_full, (uint32_t)((q_issued - 1) & 1), spin, &never);
-    }
-  } else if (warp == 5) {
+    // let every copy of this thread land before the CTA can exit
+    asm volatile("cp.async.wait_all;" ::: "memory");
+  } else if (warp == 11) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id1 = tc::idesc_bf16_f32(128, A2_H, 0, 0);
@@ -340,6 +337,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
       auto gemm1 = [&](uint32_t g) -> bool {
         const int st = g & 1;
         if (!tc::mbar_wait(&s.kv_full[st], (g >> 1) & 1, spin, abort)) return false;
+        // rows written by cp.async (generic proxy) are read by the tensor core (async proxy)
+        tc::fence_proxy_async_smem();
         tc::tc_fence_after();
 #pragma unroll
         for (int c = 0; c < A2_KCH; ++c) {
@@ -355,7 +354,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
       for (int item = cluster_id; item < items && ok; item += nclusters, ++k) {
         const ItemInfo it = item_info(a, item, head_groups);
         ok = tc::mbar_wait(&s.q_full, (uint32_t)(k & 1), spin, abort);
-        A2_TRACE(25, k, 0);
         if (!ok) break;
         ok = gemm1(G);
         A2_TRACE(3, k, 0);
@@ -368,11 +366,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
             if (j + 2 == it.nb) tc::mma_commit(&s.q_empty);
           }
           const int st = G & 1;
-          ok = wait_cluster(&s.p_full[st], (G >> 1) & 1, spin, abort);
-          A2_TRACE(4, k, j);
+          ok = tc::mbar_wait(&s.p_full, G & 1, spin, abort);
           if (!ok) break;
+          A2_TRACE(4, k, j);
           tc::tc_fence_after();
-          const uint32_t pb = tc::smem_u32(s.p[st]);
+          const uint32_t pb = tc::smem_u32(s.p);
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             const uint32_t kvb = tc::smem_u32(s.kv[st][2 * q]);
@@ -397,77 +395,78 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    const uint32_t r_xs[2] = {mapa(tc::smem_u32(&s.xs[0][tid][0]), peer),
-                              mapa(tc::smem_u32(&s.xs[1][tid][0]), peer)};
-    const uint32_t r_p[2] = {mapa(tc::smem_u32(s.p[0] + tid * 128), peer),
-                             mapa(tc::smem_u32(s.p[1] + tid * 128), peer)};
-    const uint32_t r_fac[2] = {mapa(tc::smem_u32(&s.fac[0][0]), peer),
-                               mapa(tc::smem_u32(&s.fac[1][0]), peer)};
-    const uint32_t r_inv[2] = {mapa(tc::smem_u32(&s.inv[0][0]), peer),
-                               mapa(tc::smem_u32(&s.inv[1][0]), peer)};
-    const uint32_t rb_xs[2] = {mapa(tc::smem_u32(&s.xs_full[0]), peer),
-                               mapa(tc::smem_u32(&s.xs_full[1]), peer)};
-    const uint32_t rb_fac[2] = {mapa(tc::smem_u32(&s.fac_full[0]), peer),
-                                mapa(tc::smem_u32(&s.fac_full[1]), peer)};
-    const uint32_t rb_p[2] = {mapa(tc::smem_u32(&s.p_full[0]), peer),
-                              mapa(tc::smem_u32(&s.p_full[1]), peer)};
-    const uint32_t rb_inv[2] = {mapa(tc::smem_u32(&s.inv_full[0]), peer),
-                                mapa(tc::smem_u32(&s.inv_full[1]), peer)};
-    const int own0 = A2_HO * (int)rank, peer0 = A2_HO * (int)peer;
+    const int quad = warp & 3, half = warp >> 2;        // lane quadrant, head half
+    const int slot = 32 * quad + lane;                  // TMEM lane = slot / channel row
+    const int hb = 32 * half;                           // first head of this thread
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    const uint32_t r_xs = mapa(tc::smem_u32(&s.xs[slot][0]), peer);   // my row in the peer
+    const uint32_t rb_xs_full = mapa(tc::smem_u32(&s.xs_full), peer);
+    const uint32_t rb_xs_empty = mapa(tc::smem_u32(&s.xs_empty), peer);
     uint32_t G = 0;
     int k = 0;
     bool ok = true;
     for (int item = cluster_id; item < items && ok; item += nclusters, ++k) {
       const ItemInfo it = item_info(a, item, head_groups);
-      float l_part[A2_HO], l32[A2_HO];   // sums of bf16-rounded / exact probabilities
+      float lsum[32];                                   // sums of the bf16-rounded weights
 #pragma unroll
-      for (int h = 0; h < A2_HO; ++h) l_part[h] = l32[h] = 0.f;
+      for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
       for (int j = 0; j < it.nb; ++j, ++G) {
         const int st = G & 1;
-        const uint32_t par = (G >> 1) & 1;
-        const Slot sl = slot_of(a, it.cs, it.nc4, j * A2_BLK + tid);   // load overlaps the wait
+        const Slot sl = slot_of(a, it.cs, it.nc4, j * A2_BLK + slot);   // load overlaps the wait
         if (tid == 0) A2_TRACE(6, k, j);
-        ok = tc::mbar_wait(&s.s_full[st], par, spin, abort);
+        ok = tc::mbar_wait(&s.s_full[st], (G >> 1) & 1, spin, abort);
+        ok = !bar_red_or2(3, A2_SOFT, !ok);
+        if (!ok) break;
         if (tid == 0) A2_TRACE(7, k, j);
-        ok = !bar_red_or2(3, 128, !ok);
-        if (!ok) break;
         tc::tc_fence_after();
-        float vo[A2_HO], vp[A2_HO];            // partial S: owned heads, peer's heads
-        tc::tmem_ld32(tmem + lane_base + T2_S + 64 * st + own0, vo);
-        tc::tmem_ld32(tmem + lane_base + T2_S + 64 * st + peer0, vp);
+        float z[32];
+        tc::tmem_ld32(tmem + lane_base + T2_S + 64 * st + hb, z);
         tc::tmem_wait_ld();
-        // the peer's heads -> peer.xs[st][tid][*] (16-byte chunk c at c ^ (tid & 7))
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_remote_v4(r_xs[st] + 16 * (c ^ (tid & 7)),
-                       make_uint4(__float_as_uint(vp[4 * c]), __float_as_uint(vp[4 * c + 1]),
-                                  __float_as_uint(vp[4 * c + 2]), __float_as_uint(vp[4 * c + 3])));
-        arrive_remote(rb_xs[st]);
-        if (tid == 0) A2_TRACE(9, k, j);
-        ok = wait_cluster(&s.xs_full[st], par, spin, abort);
-        if (tid == 0) A2_TRACE(10, k, j);
-        ok = !bar_red_or2(3, 128, !ok);
-        if (!ok) break;
-        float z[A2_HO];
-        const float* xr = s.xs[st][tid];
+        // my partial -> the peer (after it consumed the previous block's partial)
+        if (G > 0) {
+          ok = wait_cluster(&s.xs_empty, (G - 1) & 1, spin, abort);
+          ok = !bar_red_or2(3, A2_SOFT, !ok);
+          if (!ok) break;
+        }
+        // asynchronous remote stores; each one counts its bytes on the peer's xs_full
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          const float4 x4 = *reinterpret_cast<const float4*>(xr + 4 * (c ^ (tid & 7)));
-          z[4 * c] = sl.valid ? (vo[4 * c] + x4.x) * scale_log2 : -INFINITY;
-          z[4 * c + 1] = sl.valid ? (vo[4 * c + 1] + x4.y) * scale_log2 : -INFINITY;
-          z[4 * c + 2] = sl.valid ? (vo[4 * c + 2] + x4.z) * scale_log2 : -INFINITY;
-          z[4 * c + 3] = sl.valid ? (vo[4 * c + 3] + x4.w) * scale_log2 : -INFINITY;
+          const int cc = 8 * half + c;                  // 16-byte chunk within the 256-B row
+          st_async_v4(r_xs + 16 * (cc ^ (slot & 7)), z[4 * c], z[4 * c + 1], z[4 * c + 2],
+                      z[4 * c + 3], rb_xs_full);
         }
-        float red[A2_HO];
+        if (tid == 0) tc::mbar_arrive_expect_tx(&s.xs_full, A2_BLK * A2_H * 4);
+        if (tid == 0) A2_TRACE(9, k, j);
+        ok = wait_cluster(&s.xs_full, G & 1, spin, abort);
+        ok = !bar_red_or2(3, A2_SOFT, !ok);
+        if (!ok) break;
+        if (tid == 0) A2_TRACE(10, k, j);
+        const float* xr = s.xs[slot];
 #pragma unroll
-        for (int h = 0; h < A2_HO; ++h) red[h] = z[h];
-        s.red[warp][lane] = xpose_reduce32<true>(red);
-        tc::named_barrier(1, 128);
+        for (int c = 0; c < 8; ++c) {
+          const int cc = 8 * half + c;
+          const float4 x4 = *reinterpret_cast<const float4*>(xr + 4 * (cc ^ (slot & 7)));
+          z[4 * c] = sl.valid ? (z[4 * c] + x4.x) * scale_log2 : -INFINITY;
+          z[4 * c + 1] = sl.valid ? (z[4 * c + 1] + x4.y) * scale_log2 : -INFINITY;
+          z[4 * c + 2] = sl.valid ? (z[4 * c + 2] + x4.z) * scale_log2 : -INFINITY;
+          z[4 * c + 3] = sl.valid ? (z[4 * c + 3] + x4.w) * scale_log2 : -INFINITY;
+        }
+        // block max per head: butterfly within the warp, then the 4 lane quadrants
+        {
+          float red[32];
+#pragma unroll
+          for (int h = 0; h < 32; ++h) red[h] = z[h];
+          s.red[quad][hb + lane] = xpose_reduce32<true>(red);
+        }
+        tc::named_barrier(1, A2_SOFT);
+        // every thread has read its xs row: the peer may send its next partial
+        if (tid == 0) arrive_remote(rb_xs_empty);
         if (tid == 0) A2_TRACE(11, k, j);
-        if (tid < A2_HO) {
-          const float bm = fmaxf(fmaxf(s.red[0][tid], s.red[1][tid]), fmaxf(s.red[2][tid], s.red[3][tid]));
-          const float mo = s.mcur[tid];
+        bool grow = false;
+        if (quad == 0) {                                // warps 0 and 4 own heads hb + lane
+          const int h = hb + lane;
+          const float bm = fmaxf(fmaxf(s.red[0][h], s.red[1][h]), fmaxf(s.red[2][h], s.red[3][h]));
+          const float mo = s.mcur[h];
           float mn = mo, f = 1.f;
           if (mo == -INFINITY) {
             mn = bm;
@@ -475,145 +474,116 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
           } else if (bm > mo + TAU2) {
             mn = bm;
             f = exp2f(mo - mn);
+            grow = true;
           }
-          s.mcur[tid] = mn;
-          s.fac[st][own0 + tid] = f;
-          st_remote_f32(r_fac[st] + 4 * (own0 + tid), f);
+          s.mcur[h] = mn;
+          s.fac[h] = f;
         }
-        tc::named_barrier(1, 128);
-        arrive_remote(rb_fac[st]);
+        const bool rescale = bar_red_or2(2, A2_SOFT, grow) && j > 0;
         if (tid == 0) A2_TRACE(12, k, j);
-        // probabilities of the owned heads, P^T columns to both CTAs
-        uint32_t packed[A2_HO / 2];
+        // the single P buffer: GEMM2 of the previous block must have read it
+        if (j > 0) {
+          ok = tc::mbar_wait(&s.o_blk[(G - 1) & 1], ((G - 1) >> 1) & 1, spin, abort);
+          ok = !bar_red_or2(3, A2_SOFT, !ok);
+          if (!ok) break;
+        }
+        if (tid == 0) A2_TRACE(14, k, j);
+        uint32_t packed[16];
 #pragma unroll
-        for (int h = 0; h < A2_HO; h += 2) {
-          const float m0 = s.mcur[h], m1 = s.mcur[h + 1];
+        for (int h = 0; h < 32; h += 2) {
+          const float m0 = s.mcur[hb + h], m1 = s.mcur[hb + h + 1];
           const float p0 = exp2f(z[h] - (m0 == -INFINITY ? 0.f : m0));
           const float p1 = exp2f(z[h + 1] - (m1 == -INFINITY ? 0.f : m1));
           __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
           const float2 pr = __bfloat1622float2(pb2);
-          const float f0 = s.fac[st][own0 + h], f1 = s.fac[st][own0 + h + 1];
-          l_part[h] = fmaf(l_part[h], f0, pr.x);
-          l_part[h + 1] = fmaf(l_part[h + 1], f1, pr.y);
-          l32[h] = fmaf(l32[h], f0, p0);
-          l32[h + 1] = fmaf(l32[h + 1], f1, p1);
+          lsum[h] = fmaf(lsum[h], s.fac[hb + h], pr.x);
+          lsum[h + 1] = fmaf(lsum[h + 1], s.fac[hb + h + 1], pr.y);
           packed[h / 2] = *reinterpret_cast<uint32_t*>(&pb2);
         }
-        uint8_t* prow = s.p[st] + tid * 128;
+        uint8_t* prow = s.p + slot * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint32_t off = (uint32_t)(((4 * (int)rank + c) ^ (tid & 7)) << 4);
-          const uint4 val = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-          *reinterpret_cast<uint4*>(prow + off) = val;
-          st_remote_v4(r_p[st] + off, val);
-        }
-        ok = wait_cluster(&s.fac_full[st], par, spin, abort);
-        if (tid == 0) A2_TRACE(14, k, j);
-        ok = !bar_red_or2(3, 128, !ok);
-        if (!ok) break;
-        // rescale O^T (all 64 heads of this CTA's channels) when any head's max grew
-        bool any = false;
-#pragma unroll
-        for (int h = 0; h < A2_H; ++h) any |= (s.fac[st][h] != 1.f);
-        if (any && j > 0) {
-          // GEMM2 of the previous block must be done (its buffer's barrier, see below)
-          ok = tc::mbar_wait(&s.o_blk[(G - 1) & 1], ((G - 1) >> 1) & 1, spin, abort);
-          ok = !bar_red_or2(3, 128, !ok);
-          if (!ok) break;
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (slot & 7)) << 4)) =
+              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        if (rescale) {
           tc::tc_fence_after();
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
+            float o[32];
+            const uint32_t addr = tmem + lane_base + T2_O + 64 * q + hb;
+            tc::tmem_ld32(addr, o);
+            tc::tmem_wait_ld();
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              float o[32];
-              const uint32_t addr = tmem + lane_base + T2_O + 64 * q + 32 * hh;
-              tc::tmem_ld32(addr, o);
-              tc::tmem_wait_ld();
-#pragma unroll
-              for (int u = 0; u < 32; ++u) o[u] *= s.fac[st][32 * hh + u];
-              tc::tmem_st32(addr, o);
-            }
+            for (int u = 0; u < 32; ++u) o[u] *= s.fac[hb + u];
+            tc::tmem_st32(addr, o);
           }
           tc::tmem_wait_st();
         }
-        fence_proxy_async_all();
-        if (tid == 0) A2_TRACE(16, k, j);
+        tc::fence_proxy_async_smem();
         tc::tc_fence_before();
-        tc::mbar_arrive(&s.p_full[st]);
-        arrive_remote(rb_p[st]);
+        tc::mbar_arrive(&s.p_full);
         if (tid == 0) A2_TRACE(17, k, j);
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue
       // GEMM2 of the item's last block (hence every earlier one) is complete. One barrier per
-      // S/KV parity keeps the phase of the waited GEMM2 unambiguous: GEMM1 of block G
-      // completing implies GEMM2 of block G-2 completed (issued before it).
+      // S/KV parity keeps the waited phase unambiguous: GEMM1 of block G completing implies
+      // GEMM2 of block G-2 completed (issued before it).
       ok = tc::mbar_wait(&s.o_blk[(G - 1) & 1], ((G - 1) >> 1) & 1, spin, abort);
-      ok = !bar_red_or2(3, 128, !ok);
-      if (tid == 0) A2_TRACE(20, k, 0);
+      ok = !bar_red_or2(3, A2_SOFT, !ok);
       if (!ok) break;
+      if (tid == 0) A2_TRACE(20, k, 0);
       tc::tc_fence_after();
-      // O is normalised by the sum of the same bf16 weights the PV product used; the LSE
-      // uses the sum of the exact fp32 weights.
-      s.red[warp][lane] = xpose_reduce32<false>(l32);
-      tc::named_barrier(1, 128);
-      float L32 = 0.f;
-      if (tid < A2_HO) L32 = (s.red[0][tid] + s.red[1][tid]) + (s.red[2][tid] + s.red[3][tid]);
-      tc::named_barrier(1, 128);
-      s.red[warp][lane] = xpose_reduce32<false>(l_part);
-      tc::named_barrier(1, 128);
-      const int kb = k & 1;
+      s.red[quad][hb + lane] = xpose_reduce32<false>(lsum);
+      tc::named_barrier(1, A2_SOFT);
       const int h0 = it.hg * A2_H;
-      if (tid < A2_HO) {
-        const float L = (s.red[0][tid] + s.red[1][tid]) + (s.red[2][tid] + s.red[3][tid]);
-        const float m = s.mcur[tid];
-        const int hgl = h0 + own0 + tid;
-        const float s2 = a.sink ? a.sink[hgl] * LOG2E2 : -INFINITY;
+      if (quad == 0) {
+        const int h = hb + lane;
+        const float L = (s.red[0][h] + s.red[1][h]) + (s.red[2][h] + s.red[3][h]);
+        const float m = s.mcur[h];
+        const float s2 = a.sink ? a.sink[h0 + h] * LOG2E2 : -INFINITY;
         const float mf = fmaxf(m, s2);
-        const float sk = a.sink ? exp2f(s2 - mf) : 0.f;
         const float em = m == -INFINITY ? 0.f : exp2f(m - mf);
-        const float den = L * em + sk;
-        const float den32 = L32 * em + sk;
+        const float den = L * em + (a.sink ? exp2f(s2 - mf) : 0.f);
         float inv = 0.f, lse = -INFINITY;
         if (den > 0.f && mf != -INFINITY) {
           inv = em / den;
-          lse = (mf + log2f(den32)) * LN2_2;
+          lse = (mf + log2f(den)) * LN2_2;
         }
-        s.inv[kb][own0 + tid] = inv;
-        st_remote_f32(r_inv[kb] + 4 * (own0 + tid), inv);
-        if (a.lse) a.lse[(long long)it.qi * a.H + hgl] = lse;
-        s.mcur[tid] = -INFINITY;                    // next item starts fresh
+        s.inv[h] = inv;
+        if (a.lse && (int)rank == half) a.lse[(long long)it.qi * a.H + h0 + h] = lse;
+        s.mcur[h] = -INFINITY;                          // the next item starts fresh
       }
-      tc::named_barrier(1, 128);
-      arrive_remote(rb_inv[kb]);
-      ok = wait_cluster(&s.inv_full[kb], (uint32_t)((k >> 1) & 1), spin, abort);
-      if (tid == 0) A2_TRACE(22, k, 0);
-      ok = !bar_red_or2(3, 128, !ok);
-      if (!ok) break;
+      tc::named_barrier(1, A2_SOFT);
+      // O^T tiles -> bf16 [64 heads][128 channels] staging in the P buffer -> 16-byte stores
+      __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(s.p);
       __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(a.O) + ((long long)it.qi * a.H + h0) * A2_C +
                          (int)rank * A2_CH;
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
+        float o[32];
+        tc::tmem_ld32(tmem + lane_base + T2_O + 64 * q + hb, o);
+        tc::tmem_wait_ld();
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          float o[32];
-          tc::tmem_ld32(tmem + lane_base + T2_O + 64 * q + 32 * hh, o);
-          tc::tmem_wait_ld();
+        for (int u = 0; u < 32; ++u)
+          stage[(hb + u) * A2_BLK + slot] = __float2bfloat16_rn(o[u] * s.inv[hb + u]);
+        tc::named_barrier(1, A2_SOFT);
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int h = 32 * hh + u;
-            O[(long long)h * A2_C + 128 * q + tid] = __float2bfloat16_rn(o[u] * s.inv[kb][h]);
-          }
+        for (int e = tid; e < A2_H * A2_BLK / 8; e += A2_SOFT) {
+          const int h = e >> 4, c8 = e & 15;
+          *reinterpret_cast<uint4*>(O + (long long)h * A2_C + 128 * q + 8 * c8) =
+              *reinterpret_cast<const uint4*>(stage + h * A2_BLK + 8 * c8);
         }
+        tc::named_barrier(1, A2_SOFT);
       }
-      if (tid == 0) A2_TRACE(23, k, 0);
       tc::tc_fence_before();
+      if (tid == 0) A2_TRACE(23, k, 0);
     }
   }
   tc::tc_fence_before();
   __syncthreads();
   cluster_sync();                       // no remote access may target an exited peer
-  if (warp == 5) {
+  if (warp == 11) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, T2_COLS);
   }
@@ -624,18 +594,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(A2_THREADS, 1)
 // Returns DSV4_OK with *used = false when the shape or the device does not fit this kernel.
 int launch_attn_tc2(const AttnArgs& a, cudaStream_t st, bool* used) {
   *used = false;
-  const char* off = std::getenv("DSV4_ATTN_V1");
-  if (off && off[0] == '1') return DSV4_OK;
+  // the single-CTA kernel is the default; DSV4_ATTN_CLUSTER=1 selects this one
+  const char* on = std::getenv("DSV4_ATTN_CLUSTER");
+  if (!on || on[0] != '1') return DSV4_OK;
   const char* force = std::getenv("DSV4_FORCE_SIMT");
   if (force && force[0] == '1') return DSV4_OK;
   if (a.c != A2_C || a.H % A2_H != 0) return DSV4_OK;
   if (!aligned16(a.Q) || !aligned16(a.local) || (a.pool && !aligned16(a.pool))) return DSV4_OK;
   const long long nrows_q = (long long)a.B * a.nq * a.H;
-  const long long nrows_local = (long long)a.B * a.R;
   const long long items = (long long)a.B * a.nq * (a.H / A2_H);
-  if (nrows_q >= (1ll << 31) || nrows_local >= (1ll << 31) || a.pool_rows >= (1ll << 31) ||
-      items >= (1ll << 31))
-    return DSV4_OK;
+  if (nrows_q >= (1ll << 31) || items >= (1ll << 31)) return DSV4_OK;
   static int max_clusters = -1;
   if (max_clusters < 0) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -654,29 +622,31 @@ int launch_attn_tc2(const AttnArgs& a, cudaStream_t st, bool* used) {
     cfg.numAttrs = 1;
     int n = 0;
     e = cudaOccupancyMaxActiveClusters(&n, attn_tc2_kernel, &cfg);
+    const char* verbose = std::getenv("DSV4_VERBOSE");
+    if (verbose && verbose[0] == '1')
+      std::fprintf(stderr, "[dsv4] cluster attention: %d co-resident clusters (%s)\n", n,
+                   cudaGetErrorString(e));
     if (e != cudaSuccess) {
       cudaGetLastError();
       n = 0;
     }
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, attn_tc2_kernel, A2_THREADS, A2_SMEM);
+    if (verbose && verbose[0] == '1')
+      std::fprintf(stderr, "[dsv4] cluster attention: %d CTAs per SM (%s)\n", per_sm,
+                   cudaGetErrorString(e));
+    const char* force_n = std::getenv("DSV4_CLUSTERS");
+    if (force_n && std::atoi(force_n) > 0) n = std::atoi(force_n);
     max_clusters = n;
   }
   if (max_clusters <= 0) return DSV4_OK;
-  CUtensorMap mq, mpool, mlocal;
+  CUtensorMap mq;
   int s = encode_tensor_map_2d(&mq, a.Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A2_C, nrows_q, 64,
                                A2_H, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
-  s = encode_tensor_map_2d(&mlocal, a.local, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A2_C,
-                           nrows_local, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != DSV4_OK) return s;
-  if (a.pool && a.pool_rows > 0)
-    s = encode_tensor_map_2d(&mpool, a.pool, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, A2_C,
-                             a.pool_rows, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
-  else
-    mpool = mlocal;
-  if (s != DSV4_OK) return s;
   const long long nclusters = items < max_clusters ? items : max_clusters;
   attn_tc2_kernel<<<(unsigned)(2 * nclusters), A2_THREADS, A2_SMEM, st>>>(
-      a, mq, mpool, mlocal, a.H / A2_H, (int)items, a.scale * LOG2E2, spin_limit());
+      a, mq, a.H / A2_H, (int)items, a.scale * LOG2E2, spin_limit());
   *used = true;
   return launch_status("hybrid attention (tensor cores, 2-CTA cluster)");
 }

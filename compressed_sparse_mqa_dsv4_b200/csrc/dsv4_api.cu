@@ -3,6 +3,7 @@
 // kernels). Declarations and the contract of every entry point are in include/dsv4.h.
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <string>
 
 #include "attn_common.cuh"
@@ -31,6 +32,15 @@ int launch_status(const char* what) {
 }
 
 static long long round_up(long long a, long long b) { return (a + b - 1) / b * b; }
+
+// DSV4_VERBOSE=1: report on stderr which kernel path each entry point takes.
+static void trace_path(const char* what) {
+  static const bool verbose = [] {
+    const char* e = std::getenv("DSV4_VERBOSE");
+    return e && e[0] == '1';
+  }();
+  if (verbose) std::fprintf(stderr, "[dsv4] %s\n", what);
+}
 
 }  // namespace dsv4
 
@@ -181,9 +191,16 @@ extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* poo
   if (dtype == DSV4_BF16) {
     bool used = false;
     int s = launch_attn_tc2(a, st, &used);
-    if (s != DSV4_OK || used) return s;
+    if (s != DSV4_OK || used) {
+      trace_path("hybrid attention: tcgen05, 2-CTA cluster");
+      return s;
+    }
     s = launch_attn_tc(a, st, &used);
-    if (s != DSV4_OK || used) return s;
+    if (s != DSV4_OK || used) {
+      trace_path("hybrid attention: tcgen05, single CTA");
+      return s;
+    }
   }
+  trace_path("hybrid attention: CUDA cores");
   return launch_attn_simt(a, dtype, st);
 }

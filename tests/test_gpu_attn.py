@@ -78,7 +78,7 @@ def attn_path(request, monkeypatch):
     """Run a case on each attention kernel: the 2-CTA-cluster tcgen05 kernel, the single-CTA
     tcgen05 kernel (both bf16, c=512, H%64==0) and the CUDA-core kernel."""
     monkeypatch.setenv("DSV4_FORCE_SIMT", "1" if request.param == "cuda_cores" else "0")
-    monkeypatch.setenv("DSV4_ATTN_V1", "1" if request.param == "tc_single_cta" else "0")
+    monkeypatch.setenv("DSV4_ATTN_CLUSTER", "1" if request.param == "tc_cluster" else "0")
     return request.param
 
 
