@@ -122,6 +122,32 @@ __device__ __forceinline__ float xpose_reduce32(float (&v)[32]) {
   return v[0];
 }
 
+// 8x8 transpose across the 8 lanes of a lane group (r = lane & 7): on entry v[i] is element
+// (row r, column i); on exit v[i] is element (row i, column r). Three exchange stages swap
+// the off-diagonal blocks of size 4, 2 and 1.
+__device__ __forceinline__ void transpose8x8(float (&v)[8], int r) {
+#pragma unroll
+  for (int m = 4; m >= 1; m >>= 1) {
+    const bool hi = (r & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if ((i & m) == 0) {
+        const float send = hi ? v[i] : v[i + m];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+        if (hi)
+          v[i] = recv;
+        else
+          v[i + m] = recv;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
 // Slot g of the query's candidate list: part (0 pool, 1 local), global row, validity.
 struct SlotRow {
   int part;
@@ -175,7 +201,8 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int item, int h
 }
 
 __global__ void __maxnreg__(168)
-    attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q, int head_groups,
+    attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q,
+                   const __grid_constant__ CUtensorMap map_local, int head_groups,
                    int items, float scale_log2, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& s = *reinterpret_cast<AttnSmem*>(
@@ -227,9 +254,26 @@ __global__ void __maxnreg__(168)
       ok = !bar_red_or(4, AT_PROD, !ok);
       if (!ok) break;
       for (int j = 0; j < it.nb && ok; ++j, ++G) {
-        // the block's 128 row addresses (one index load per slot)
-        for (int u = pt; u < AT_BLK; u += AT_PROD) {
-          const SlotRow r = slot_row(a, it.cs, it.nc4, j * AT_BLK + u);
+        // Local-window slots of this block whose rows are contiguous (no ring wrap) and start
+        // on a 32-slot boundary come in by 2D TMA boxes of 32 rows; the rest by cp.async.
+        const int bs = j * AT_BLK;
+        int ls = it.nc4 - bs;
+        if (ls < 0) ls = 0;
+        bool tma_win = false;
+        long long first_row = 0;
+        if (ls < AT_BLK && (ls & 31) == 0) {
+          const long long jl0 = bs + ls - it.nc4;         // window index of slot ls
+          if (jl0 < it.cs.n_local) {
+            const long long p0 = it.cs.win0 + jl0;
+            const long long last = it.cs.win0 + it.cs.n_local - 1;
+            tma_win = (p0 % a.R) + (last - p0) < a.R;
+            first_row = it.cs.local_base + p0 % a.R;
+          }
+        }
+        const int cp_end = tma_win ? ls : AT_BLK;        // slots [0, cp_end) by cp.async
+        // the block's row addresses (one index load per slot)
+        for (int u = pt; u < cp_end; u += AT_PROD) {
+          const SlotRow r = slot_row(a, it.cs, it.nc4, bs + u);
           if (r.bad_index) flag_status(DSV4_ERR_DEVICE_BOUNDS);
           s.rowaddr[u] = (r.part == 0 && r.valid)
                              ? pool_addr + (uint64_t)r.row * AT_C * 2
@@ -237,18 +281,40 @@ __global__ void __maxnreg__(168)
         }
         tc::named_barrier(5, AT_PROD);
         if (pt == 0) A1_TRACE(0, k, j);
+        // this thread's copies of every chunk: rows/pieces e = pt + 96 i (same for each chunk)
+        constexpr int NPER = (AT_BLK * 8 + AT_PROD - 1) / AT_PROD;
+        const int ncopy = cp_end * 8;
+        uint64_t src[NPER];
+        uint32_t dsto[NPER];
+#pragma unroll
+        for (int i = 0; i < NPER; ++i) {
+          const int e = pt + AT_PROD * i;
+          const int row = (e >> 3) & (AT_BLK - 1), piece = e & 7;
+          src[i] = e < ncopy ? s.rowaddr[row] + (uint64_t)(16 * piece) : 0;
+          dsto[i] = (uint32_t)(row * 128 + ((piece ^ (row & 7)) << 4));
+        }
+        const uint32_t kv0 = tc::smem_u32(s.kv[0]);
         for (int c = 0; c < AT_CHUNKS; ++c) {
-          if (G > 0 && (c & 1) == 0) {
-            // GEMM2 of the previous block released chunks c, c+1
-            ok = tc::mbar_wait(&s.ch_empty[c >> 1], (G - 1) & 1, spin, abort);
+          if ((c & 1) == 0) {
+            // GEMM2 of the previous block released chunks c, c+1 (so their full-barrier
+            // phases of that block are complete and the TMA bytes go to this block's phase)
+            ok = G > 0 ? tc::mbar_wait(&s.ch_empty[c >> 1], (G - 1) & 1, spin, abort) : true;
+            if (ok && tma_win && pt == 0) {
+              tc::mbar_expect_tx(&s.ch_full[c], (AT_BLK - ls) * 128);
+              tc::mbar_expect_tx(&s.ch_full[c + 1], (AT_BLK - ls) * 128);
+            }
             ok = !bar_red_or(4, AT_PROD, !ok);
             if (!ok) break;
           }
           uint8_t* dst = s.kv[c];
-          for (int e = pt; e < AT_BLK * 8; e += AT_PROD) {
-            const int row = e >> 3, piece = e & 7;
-            cp_async16(tc::smem_u32(dst + row * 128 + ((piece ^ (row & 7)) << 4)),
-                       s.rowaddr[row] + (uint64_t)(128 * c + 16 * piece));
+#pragma unroll
+          for (int i = 0; i < NPER; ++i)
+            if (pt + AT_PROD * i < ncopy)
+              cp_async16(kv0 + (uint32_t)(c * AT_BLK * 128) + dsto[i], src[i] + (uint64_t)(128 * c));
+          if (tma_win && pt == 0) {
+            for (int r0 = ls; r0 < AT_BLK; r0 += 32)
+              tc::tma_load_2d(dst + r0 * 128, &map_local, &s.ch_full[c], 64 * c,
+                              (int32_t)(first_row + (r0 - ls)));
           }
           cp_async_arrive_noinc(&s.ch_full[c]);
         }
@@ -262,6 +328,12 @@ __global__ void __maxnreg__(168)
     if (lane == 0) {
       const uint32_t id1 = tc::idesc_bf16_f32(128, AT_H, 0, 0);   // A, B K-major
       const uint32_t id2 = tc::idesc_bf16_f32(128, AT_H, 1, 1);   // A, B MN-major
+      // Base descriptors; a K step or a chunk only moves the start address, which is the low
+      // 14-bit field (address >> 4), so the loops just add small constants.
+      const uint64_t d_kv1 = tc::sdesc_sw128(tc::smem_u32(s.kv[0]), 16, 1024);
+      const uint64_t d_q1 = tc::sdesc_sw128(tc::smem_u32(s.q[0]), 16, 1024);
+      const uint64_t d_kv2 = tc::sdesc_sw128(tc::smem_u32(s.kv[0]), AT_BLK * 128, 1024);
+      const uint64_t d_p2 = tc::sdesc_sw128(tc::smem_u32(s.p), AT_BLK * 128, 1024);
       uint32_t G = 0;
       int k = 0;
       bool ok = true;
@@ -269,16 +341,17 @@ __global__ void __maxnreg__(168)
         const ItemInfo it = item_info(a, item, head_groups);
         ok = tc::mbar_wait(&s.q_full, (uint32_t)(k & 1), spin, abort);
         for (int j = 0; j < it.nb && ok; ++j, ++G) {
-          for (int c = 0; c < AT_CHUNKS && ok; ++c) {
+#pragma unroll
+          for (int c = 0; c < AT_CHUNKS; ++c) {
             ok = tc::mbar_wait(&s.ch_full[c], G & 1, spin, abort);
             if (!ok) break;
             tc::fence_proxy_async_smem();          // cp.async (generic) -> tensor core (async)
             tc::tc_fence_after();
-            const uint32_t kvb = tc::smem_u32(s.kv[c]), qb = tc::smem_u32(s.q[c]);
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              tc::mma_bf16_ss(tmem + TM_S, tc::sdesc_sw128(kvb + kk * 32, 16, 1024),
-                              tc::sdesc_sw128(qb + kk * 32, 16, 1024), id1, (c | kk) != 0);
+              tc::mma_bf16_ss(tmem + TM_S, d_kv1 + (uint64_t)(c * (AT_BLK * 128 / 16) + 2 * kk),
+                              d_q1 + (uint64_t)(c * (AT_H * 128 / 16) + 2 * kk), id1,
+                              (c | kk) != 0);
           }
           if (!ok) break;
           tc::mma_commit(&s.s_full);
@@ -288,15 +361,14 @@ __global__ void __maxnreg__(168)
           if (!ok) break;
           A1_TRACE(4, k, j);
           tc::tc_fence_after();
-          const uint32_t pb = tc::smem_u32(s.p);
+          const uint32_t acc0 = j > 0 ? 1u : 0u;
+#pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint32_t kvb = tc::smem_u32(s.kv[2 * q]);
 #pragma unroll
             for (int ks = 0; ks < AT_BLK / 16; ++ks)
               tc::mma_bf16_ss(tmem + TM_O + 64 * q,
-                              tc::sdesc_sw128(kvb + ks * 2048, AT_BLK * 128, 1024),
-                              tc::sdesc_sw128(pb + ks * 2048, AT_BLK * 128, 1024), id2,
-                              (j > 0 || ks > 0) ? 1u : 0u);
+                              d_kv2 + (uint64_t)(2 * q * (AT_BLK * 128 / 16) + ks * 128),
+                              d_p2 + (uint64_t)(ks * 128), id2, ks > 0 ? 1u : acc0);
             tc::mma_commit(&s.ch_empty[q]);
           }
           tc::mma_commit(&s.o_done);
@@ -322,6 +394,8 @@ __global__ void __maxnreg__(168)
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
       const ItemInfo it = item_info(a, item, head_groups);
       float lsum[32];                                  // sums of the bf16-rounded weights
+      // sink logit of the head this thread finalises (loaded early, used in the epilogue)
+      const float sink_h = (quad == 0 && a.sink) ? __ldg(a.sink + it.hg * AT_H + hb + lane) : 0.f;
 #pragma unroll
       for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
       for (int j = 0; j < it.nb; ++j, ++G) {
@@ -412,12 +486,13 @@ __global__ void __maxnreg__(168)
       tc::tc_fence_after();
       s.red[quad][hb + lane] = xpose_reduce32<false>(lsum);
       tc::named_barrier(1, AT_SOFT);
+      if (tid == 0) A1_TRACE(21, k, 0);
       const int h0 = it.hg * AT_H;
       if (quad == 0) {
         const int h = hb + lane;
         const float L = (s.red[0][h] + s.red[1][h]) + (s.red[2][h] + s.red[3][h]);
         const float m = s.mcur[h];
-        const float s2 = a.sink ? a.sink[h0 + h] * LOG2E : -INFINITY;
+        const float s2 = a.sink ? sink_h * LOG2E : -INFINITY;
         const float mf = fmaxf(m, s2);
         const float em = m == -INFINITY ? 0.f : exp2f(m - mf);
         const float den = L * em + (a.sink ? exp2f(s2 - mf) : 0.f);
@@ -431,24 +506,31 @@ __global__ void __maxnreg__(168)
         s.mcur[h] = -INFINITY;                         // the next item starts fresh
       }
       tc::named_barrier(1, AT_SOFT);
-      // O^T tiles -> bf16 [64 heads][128 channels] staging in the P buffer -> 16-byte stores
-      __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(s.p);
-      __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(a.O) + ((long long)it.qi * a.H + h0) * AT_C;
+      if (tid == 0) A1_TRACE(22, k, 0);
+      // O^T tiles: each lane holds one channel for 32 heads; an 8x8 shuffle transpose within
+      // groups of 8 lanes gives each lane 8 consecutive channels of one head -> 16-byte stores
+      // (no shared-memory staging, no barrier).
+      __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(a.O) + ((long long)it.qi * a.H + h0 + hb) * AT_C;
+      const int r8 = lane & 7, g8 = lane >> 3;
       for (int q = 0; q < 4; ++q) {
         float o[32];
         tc::tmem_ld32(tmem + lane_base + TM_O + 64 * q + hb, o);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
-          stage[(hb + u) * AT_BLK + slot] = __float2bfloat16_rn(o[u] * s.inv[hb + u]);
-        tc::named_barrier(1, AT_SOFT);
+        for (int hblk = 0; hblk < 4; ++hblk) {
+          float v[8];
 #pragma unroll
-        for (int e = tid; e < AT_H * AT_BLK / 8; e += AT_SOFT) {
-          const int h = e >> 4, c8 = e & 15;
-          *reinterpret_cast<uint4*>(O + (long long)h * AT_C + 128 * q + 8 * c8) =
-              *reinterpret_cast<const uint4*>(stage + h * AT_BLK + 8 * c8);
+          for (int i = 0; i < 8; ++i) v[i] = o[8 * hblk + i] * s.inv[hb + 8 * hblk + i];
+          transpose8x8(v, r8);
+          // lane (g8, r8) now holds head hb + 8*hblk + r8, channels 32*quad + 8*g8 .. +7
+          uint4 pk;
+          pk.x = pack_bf16(v[0], v[1]);
+          pk.y = pack_bf16(v[2], v[3]);
+          pk.z = pack_bf16(v[4], v[5]);
+          pk.w = pack_bf16(v[6], v[7]);
+          *reinterpret_cast<uint4*>(O + (long long)(8 * hblk + r8) * AT_C + 128 * q + 32 * quad + 8 * g8) = pk;
         }
-        tc::named_barrier(1, AT_SOFT);
+        if (tid == 0) A1_TRACE(24 + q, k, 0);
       }
       tc::tc_fence_before();
       if (tid == 0) A1_TRACE(23, k, 0);
@@ -483,13 +565,19 @@ int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used) {
                                          (int)AT_SMEM);
     if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "attn_tc: %s", cudaGetErrorString(e));
   }
-  CUtensorMap mq;
+  const long long nrows_local = (long long)a.B * a.R;
+  if (nrows_local >= (1ll << 31) || !aligned16(a.O)) return DSV4_OK;
+  CUtensorMap mq, mlocal;
   int s = encode_tensor_map_2d(&mq, a.Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_q, 64,
                                AT_H, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
+  s = encode_tensor_map_2d(&mlocal, a.local, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_local,
+                           64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DSV4_OK) return s;
   const long long grid = items < sms ? items : sms;
-  attn_tc_kernel<<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(a, mq, a.H / AT_H, (int)items,
-                                                             a.scale * LOG2E, spin_limit());
+  attn_tc_kernel<<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(a, mq, mlocal, a.H / AT_H,
+                                                             (int)items, a.scale * LOG2E,
+                                                             spin_limit());
   *used = true;
   return launch_status("hybrid attention (tensor cores)");
 }
