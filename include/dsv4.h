@@ -110,7 +110,8 @@ size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k);
  *   I_{t,s} = sum_h w_{t,h} * ReLU(qI_{t,h} . KI_s)    for s < floor((t+1)/m)
  *   S_t     = TopK_s(I_{t,s}, k)
  * Scores are accumulated in fp32. k_eff = min(k, floor((t+1)/m)) entries are returned,
- * ordered by score descending and then entry index ascending; slots k_eff..k-1 hold -1.
+ * as a set listed in ascending entry order (ties at the k-th score go to the lower entry
+ * index); slots k_eff..k-1 hold -1.
  *
  *   qdtype     DSV4_F32, DSV4_BF16 or DSV4_FP4: element type of qI and KI.
  *   qI         [B, nq, H_I, c_I] (FP4: codes [B*nq*H_I, c_I/2] + qI_scales [.., c_I/16]).

@@ -31,8 +31,8 @@ Readings taken where the pages are silent (each is also listed in the design not
   * i = 0: the preceding block is excluded from the softmax (weight exactly 0).
   * Trailing incomplete block: never pooled; a sequence of n tokens has floor(n/m)
     entries.
-  * Top-k: k_eff = min(k, |E_t|); order by score descending, then index ascending;
-    the k - k_eff unused slots hold -1.
+  * Top-k: S_t is a set: the k_eff = min(k, |E_t|) largest scores, ties going to the
+    lower entry index, listed in ascending entry order; the k - k_eff unused slots hold -1.
   * Softmax scale is an explicit parameter (default 1/sqrt(c)).
   * No de-duplication between compressed and local candidates (different objects).
   * FP4: e2m1 codes with one E4M3 scale per 16 consecutive elements (NVFP4-style),
@@ -137,15 +137,16 @@ def index_scores_query(qI, w, KI, t: int, m: int) -> np.ndarray:
 def topk_select(scores: np.ndarray, k: int):
     """TopK over the eligible entries ([CSA-DEF] s3.1), with the tie/padding reading.
 
-    Returns (idx int32 [k], count): the min(k, len) best entries by score descending,
-    index ascending among equal scores; unused slots are -1.
+    S_t is a set: the min(k, len) entries with the largest scores, equal scores at the
+    threshold going to the lower entry index. Returns (idx int32 [k], count) with the
+    selected entries in ascending entry order; unused slots are -1.
     """
     scores = np.asarray(scores, dtype=np.float64)
     E = scores.shape[0]
     k_eff = min(k, E)
     order = np.lexsort((np.arange(E), -scores))   # primary: -score, secondary: index
     idx = np.full(k, -1, dtype=np.int32)
-    idx[:k_eff] = order[:k_eff]
+    idx[:k_eff] = np.sort(order[:k_eff])
     return idx, k_eff
 
 

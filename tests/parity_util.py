@@ -6,7 +6,7 @@ Tolerances (from the stated targets; written here once):
   * LSE: the same rule as the output of that dtype;
   * integer / byte outputs (FP4 codes, scale bytes, top-k indices, counts): bit-exact,
     except top-k members whose fp64 scores lie within a 1e-6 * max(1, |I_(k)|) gap of
-    the k-th score (ties), and the order of equal fp32 scores (checked for validity).
+    the k-th score (ties). The selected set is listed in ascending entry order.
 """
 from __future__ import annotations
 
@@ -34,9 +34,10 @@ def assert_close(gpu, ref, dtype: str, what: str):
 
 
 def topk_ref_from_scores(scores: np.ndarray, k: int) -> list:
-    """Brute-force TopK (score desc, index asc) of a score vector (used on GPU fp32 scores)."""
+    """Brute-force TopK of a score vector (used on GPU fp32 scores): the k largest, ties to the
+    lower index, as a set listed in ascending entry order."""
     order = sorted(range(len(scores)), key=lambda j: (-float(scores[j]), j))
-    return order[:min(k, len(scores))]
+    return sorted(order[:min(k, len(scores))])
 
 
 def check_topk_query(gpu_idx_row, gpu_count, oracle_scores: np.ndarray, k: int,
@@ -52,8 +53,8 @@ def check_topk_query(gpu_idx_row, gpu_count, oracle_scores: np.ndarray, k: int,
     assert ((sel >= 0) & (sel < E)).all(), f"{what}: index out of range"
     if gpu_scores_row is not None:
         gs = np.asarray(gpu_scores_row[:E], dtype=np.float32)
-        # (i) the GPU's own selection and order are exact w.r.t. its fp32 scores
-        assert sel.tolist() == topk_ref_from_scores(gs, k), f"{what}: order/selection vs own scores"
+        # (i) the GPU's own selection is exact w.r.t. its fp32 scores (ascending entry order)
+        assert sel.tolist() == topk_ref_from_scores(gs, k), f"{what}: selection vs own scores"
         if score_bound is not None:
             err = np.abs(gs.astype(np.float64) - oracle_scores)
             assert (err <= score_bound).all(), f"{what}: score error {err.max():.3e}"

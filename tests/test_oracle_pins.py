@@ -270,14 +270,14 @@ def test_topk_brute_force(E, k):
         if best is None or key < best[0]:
             best = (key, sub)
     assert sorted(chosen) == sorted(best[1])
-    # listed by score descending, index ascending
-    assert [j for _, j in sorted((-s[j], j) for j in chosen)] == chosen
+    # the set is listed in ascending entry order
+    assert chosen == sorted(chosen)
 
 
 def test_topk_ties_prefer_lower_index():
     s = np.array([1.0, 3.0, 3.0, 2.0, 3.0, 0.5])
     idx, cnt = O.topk_select(s, 4)
-    assert idx.tolist() == [1, 2, 4, 3] and cnt == 4
+    assert idx.tolist() == [1, 2, 3, 4] and cnt == 4
 
 
 def test_index_topk_brute_force_tiny():
@@ -299,7 +299,7 @@ def test_index_topk_brute_force_tiny():
             sc.append(tot)
         want = sorted(range(E), key=lambda j: (-sc[j], j))[:k]
         assert counts[0, t] == min(k, E)
-        assert idx[0, t, :counts[0, t]].tolist() == want
+        assert idx[0, t, :counts[0, t]].tolist() == sorted(want)
 
 
 # ----------------------------------------------------------------------------- attention
