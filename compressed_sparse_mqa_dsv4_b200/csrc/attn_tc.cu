@@ -21,9 +21,13 @@
 //         4-quadrant exchange; O^T is rescaled only when a head's max grows by > 2^8;
 //         P^T is written as bf16; the epilogue stages O through shared memory for 16-byte
 //         stores.
-//   8-10  producer: resolves the block's 128 row addresses, then gathers them with 16-byte
+//   8-11  producer (one per sub-partition; each warp instruction moves one 128-byte chunk
+//         of 4 rows): resolves the block's 128 row addresses, then gathers them with 16-byte
 //         cp.async, chunk by chunk as GEMM2 of the previous block releases each chunk pair.
-//   11    MMA issuer and TMEM owner.
+//   12    watcher: waits for GEMM2's chunk releases and the Q buffer on the producers'
+//         behalf and passes them on through named-barrier gates (a producer's own mbarrier
+//         wait would queue behind its cp.async traffic and stall the gather).
+//   13    MMA issuer and TMEM owner; the warp stays converged and elect.sync issues.
 // Candidate slots: [0, round4(n_comp)) compressed, then the local window; slots past a
 // part's count are masked (p = 0) and fetch an in-range row, so every value is finite.
 // All waits are bounded (see tc_common.cuh).
@@ -41,8 +45,11 @@ constexpr int AT_H = 64;
 constexpr int AT_BLK = 128;
 constexpr int AT_CHUNKS = AT_C / 64;
 constexpr int AT_SOFT = 256;
-constexpr int AT_PROD = 96;
-constexpr int AT_THREADS = AT_SOFT + AT_PROD + 32;
+constexpr int AT_PROD = 128;
+constexpr int AT_THREADS = AT_SOFT + AT_PROD + 64;
+// Named barriers: 1-3 softmax warps, 5 producers, and the producer/watcher gates.
+constexpr uint32_t GATE_ITEM = 10;
+constexpr uint32_t GATE_PAIR0 = 6;          // 6..9: chunk pairs 0..3
 constexpr uint32_t TM_S = 0;
 constexpr uint32_t TM_O = 64;
 constexpr uint32_t TM_COLS = 512;
@@ -57,6 +64,7 @@ struct AttnSmem {
                                             // also the O staging tile of the epilogue
   float red[4][AT_H];
   float mcur[AT_H];
+  float moff[AT_H];                         // exp2 offset: mcur, or 0 while mcur = -inf
   float fac[AT_H];
   float inv[AT_H];
   uint64_t rowaddr[AT_BLK];
@@ -73,8 +81,8 @@ static_assert(AT_SMEM <= 232448, "shared memory of the attention kernel");
 __device__ unsigned long long g_attn1_trace[4][8][32];
 #define A1_TRACE(ev, k_, j_)                                 \
   do {                                                       \
-    if (blockIdx.x == 0 && (k_) < 4 && (j_) < 8)             \
-      g_attn1_trace[k_][j_][ev] = clock64();                 \
+    if (blockIdx.x == 0 && (k_) >= 40 && (k_) < 44 && (j_) < 8) \
+      g_attn1_trace[(k_) - 40][j_][ev] = clock64();          \
   } while (0)
 #else
 #define A1_TRACE(ev, k_, j_) \
@@ -91,6 +99,18 @@ __device__ __forceinline__ bool bar_red_or(uint32_t id, uint32_t threads, bool p
       : "r"((uint32_t)pred), "r"(id), "r"(threads)
       : "memory");
   return r != 0;
+}
+// Producer/watcher rendezvous (all producer warps and the watcher warp). gate() blocks both
+// sides and returns the OR of their predicates; pair_arrive / pair_sync are the watcher's
+// non-blocking and the producers' blocking halves of a one-way release.
+__device__ __forceinline__ bool gate(uint32_t id, bool pred) {
+  return bar_red_or(id, AT_PROD + 32, pred);
+}
+__device__ __forceinline__ void pair_arrive(uint32_t id) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(AT_PROD + 32) : "memory");
+}
+__device__ __forceinline__ void pair_sync(uint32_t id) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(AT_PROD + 32) : "memory");
 }
 __device__ __forceinline__ void cp_async16(uint32_t dst, uint64_t src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
@@ -200,7 +220,7 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int item, int h
   return it;
 }
 
-__global__ void __maxnreg__(168)
+__global__ void __maxnreg__(128)
     attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_local, int head_groups,
                    int items, float scale_log2, uint32_t spin) {
@@ -223,7 +243,7 @@ __global__ void __maxnreg__(168)
     tc::fence_barrier_init();
   }
   if (tid < AT_H) s.mcur[tid] = -INFINITY;
-  if (warp == 11) {
+  if (warp == 13) {
     tc::tmem_alloc(&s.tmem_base, TM_COLS);
     tc::tmem_relinquish();
   }
@@ -232,8 +252,8 @@ __global__ void __maxnreg__(168)
   tc::tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
-  if (warp >= 8 && warp < 11) {
-    // ------------------------------------------------------------------ producer (3 warps)
+  if (warp >= 8 && warp < 12) {
+    // ------------------------------------------------------------------ producer (4 warps)
     const int pt = tid - AT_SOFT;
     const uint64_t pool_addr = reinterpret_cast<uint64_t>(a.pool);
     const uint64_t local_addr = reinterpret_cast<uint64_t>(a.local);
@@ -243,16 +263,13 @@ __global__ void __maxnreg__(168)
     if (pt == 0) tc::prefetch_tensormap(&map_q);
     for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
       const ItemInfo it = item_info(a, item, head_groups);
-      if (pt == 0) {
-        if (k > 0) ok = tc::mbar_wait(&s.q_empty, (uint32_t)((k - 1) & 1), spin, abort);
-        if (ok) {
-          tc::mbar_arrive_expect_tx(&s.q_full, AT_CHUNKS * AT_H * 128);
-          const int qrow = it.qi * a.H + it.hg * AT_H;
-          for (int c = 0; c < AT_CHUNKS; ++c) tc::tma_load_2d(s.q[c], &map_q, &s.q_full, 64 * c, qrow);
-        }
-      }
-      ok = !bar_red_or(4, AT_PROD, !ok);
+      ok = !gate(GATE_ITEM, false);                    // the Q buffer is free (or abort)
       if (!ok) break;
+      if (pt == 0) {
+        tc::mbar_arrive_expect_tx(&s.q_full, AT_CHUNKS * AT_H * 128);
+        const int qrow = it.qi * a.H + it.hg * AT_H;
+        for (int c = 0; c < AT_CHUNKS; ++c) tc::tma_load_2d(s.q[c], &map_q, &s.q_full, 64 * c, qrow);
+      }
       for (int j = 0; j < it.nb && ok; ++j, ++G) {
         // Local-window slots of this block whose rows are contiguous (no ring wrap) and start
         // on a 32-slot boundary come in by 2D TMA boxes of 32 rows; the rest by cp.async.
@@ -297,14 +314,15 @@ __global__ void __maxnreg__(168)
         for (int c = 0; c < AT_CHUNKS; ++c) {
           if ((c & 1) == 0) {
             // GEMM2 of the previous block released chunks c, c+1 (so their full-barrier
-            // phases of that block are complete and the TMA bytes go to this block's phase)
-            ok = G > 0 ? tc::mbar_wait(&s.ch_empty[c >> 1], (G - 1) & 1, spin, abort) : true;
-            if (ok && tma_win && pt == 0) {
+            // phases of that block are complete and the TMA bytes go to this block's phase).
+            // The watcher warp saw the release; waiting on the mbarrier here instead would
+            // queue behind this thread's own cp.async traffic and starve the gather.
+            if (G > 0) pair_sync(GATE_PAIR0 + (c >> 1));
+            if (pt == 0) A1_TRACE(8 + (c >> 1), k, j);
+            if (tma_win && pt == 0) {
               tc::mbar_expect_tx(&s.ch_full[c], (AT_BLK - ls) * 128);
               tc::mbar_expect_tx(&s.ch_full[c + 1], (AT_BLK - ls) * 128);
             }
-            ok = !bar_red_or(4, AT_PROD, !ok);
-            if (!ok) break;
           }
           uint8_t* dst = s.kv[c];
 #pragma unroll
@@ -317,15 +335,53 @@ __global__ void __maxnreg__(168)
                               (int32_t)(first_row + (r0 - ls)));
           }
           cp_async_arrive_noinc(&s.ch_full[c]);
+          if (pt == 0 && (c & 1)) A1_TRACE(28 + (c >> 1), k, j);
         }
         if (pt == 0) A1_TRACE(1, k, j);
         tc::named_barrier(5, AT_PROD);                 // rowaddr[] is rewritten next block
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 11) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (pt == 0 && *abort) {
+      // the consumers gave up: let this thread's own bulk copies land before exiting
+      volatile int never = 0;
+      if (k > 0) tc::mbar_wait(&s.q_full, (uint32_t)((k - 1) & 1), spin, &never);
+      if (G > 0)
+        for (int c = 0; c < AT_CHUNKS; ++c) tc::mbar_wait(&s.ch_full[c], (G - 1) & 1, spin, &never);
+    }
+  } else if (warp == 12) {
+    // ------------------------------------------------------------------ watcher
+    // Performs the producers' mbarrier waits and passes each result on; both sides take
+    // the same sequence of gates (one per item, four per block after the first).
+    //  * item gate: a blocking OR-reduction, so both sides take the same abort decision;
+    //  * pair gates: the watcher only arrives (it does not block, so it is already waiting
+    //    for the next release while the producers copy) and the producers sync. A release
+    //    of pair q of block j needs all of block j's copies, so at most one arrival per
+    //    gate is outstanding. After an abort the watcher syncs instead (lock step with the
+    //    producers) until the next item gate ends both loops.
+    auto wwait = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, spin, abort));
+    };
+    uint32_t G = 0;
+    int k = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
+      const ItemInfo it = item_info(a, item, head_groups);
+      if (k > 0) ok = wwait(&s.q_empty, (uint32_t)((k - 1) & 1));
+      ok = !gate(GATE_ITEM, !ok || *abort != 0);
+      for (int j = 0; j < it.nb && ok; ++j, ++G) {
+        if (G == 0) continue;
+        for (int q = 0; q < 4; ++q) {
+          if (wwait(&s.ch_empty[q], (G - 1) & 1))
+            pair_arrive(GATE_PAIR0 + q);
+          else
+            pair_sync(GATE_PAIR0 + q);
+        }
+      }
+    }
+  } else if (warp == 13) {
+    // ------------------------------------------------------------------ MMA issuer (converged)
+    {
       const uint32_t id1 = tc::idesc_bf16_f32(128, AT_H, 0, 0);   // A, B K-major
       const uint32_t id2 = tc::idesc_bf16_f32(128, AT_H, 1, 1);   // A, B MN-major
       // Base descriptors; a K step or a chunk only moves the start address, which is the low
@@ -334,49 +390,54 @@ __global__ void __maxnreg__(168)
       const uint64_t d_q1 = tc::sdesc_sw128(tc::smem_u32(s.q[0]), 16, 1024);
       const uint64_t d_kv2 = tc::sdesc_sw128(tc::smem_u32(s.kv[0]), AT_BLK * 128, 1024);
       const uint64_t d_p2 = tc::sdesc_sw128(tc::smem_u32(s.p), AT_BLK * 128, 1024);
+      // every lane waits (acquire per lane) and the warp takes one decision
+      auto wwait = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, spin, abort));
+      };
       uint32_t G = 0;
       int k = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
         const ItemInfo it = item_info(a, item, head_groups);
-        ok = tc::mbar_wait(&s.q_full, (uint32_t)(k & 1), spin, abort);
+        ok = wwait(&s.q_full, (uint32_t)(k & 1));
         for (int j = 0; j < it.nb && ok; ++j, ++G) {
 #pragma unroll
           for (int c = 0; c < AT_CHUNKS; ++c) {
-            ok = tc::mbar_wait(&s.ch_full[c], G & 1, spin, abort);
+            ok = wwait(&s.ch_full[c], G & 1);
             if (!ok) break;
+            if (lane == 0 && (c & 1)) A1_TRACE(12 + (c >> 1), k, j);
             tc::fence_proxy_async_smem();          // cp.async (generic) -> tensor core (async)
             tc::tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              tc::mma_bf16_ss(tmem + TM_S, d_kv1 + (uint64_t)(c * (AT_BLK * 128 / 16) + 2 * kk),
-                              d_q1 + (uint64_t)(c * (AT_H * 128 / 16) + 2 * kk), id1,
-                              (c | kk) != 0);
+              tc::mma_bf16_ss_warp(tmem + TM_S, d_kv1 + (uint64_t)(c * (AT_BLK * 128 / 16) + 2 * kk),
+                                   d_q1 + (uint64_t)(c * (AT_H * 128 / 16) + 2 * kk), id1,
+                                   (c | kk) != 0);
           }
           if (!ok) break;
-          tc::mma_commit(&s.s_full);
-          A1_TRACE(3, k, j);
-          if (j + 1 == it.nb) tc::mma_commit(&s.q_empty);
-          ok = tc::mbar_wait(&s.p_full, G & 1, spin, abort);
+          tc::mma_commit_warp(&s.s_full);
+          if (lane == 0) A1_TRACE(3, k, j);
+          if (j + 1 == it.nb) tc::mma_commit_warp(&s.q_empty);
+          ok = wwait(&s.p_full, G & 1);
           if (!ok) break;
-          A1_TRACE(4, k, j);
+          if (lane == 0) A1_TRACE(4, k, j);
           tc::tc_fence_after();
           const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
 #pragma unroll
             for (int ks = 0; ks < AT_BLK / 16; ++ks)
-              tc::mma_bf16_ss(tmem + TM_O + 64 * q,
-                              d_kv2 + (uint64_t)(2 * q * (AT_BLK * 128 / 16) + ks * 128),
-                              d_p2 + (uint64_t)(ks * 128), id2, ks > 0 ? 1u : acc0);
-            tc::mma_commit(&s.ch_empty[q]);
+              tc::mma_bf16_ss_warp(tmem + TM_O + 64 * q,
+                                   d_kv2 + (uint64_t)(2 * q * (AT_BLK * 128 / 16) + ks * 128),
+                                   d_p2 + (uint64_t)(ks * 128), id2, ks > 0 ? 1u : acc0);
+            tc::mma_commit_warp(&s.ch_empty[q]);
           }
-          tc::mma_commit(&s.o_done);
-          A1_TRACE(5, k, j);
+          tc::mma_commit_warp(&s.o_done);
+          if (lane == 0) A1_TRACE(5, k, j);
         }
       }
       if (!ok) {
-        tc::mma_commit(&s.drain);
+        tc::mma_commit_warp(&s.drain);
         volatile int never = 0;
         tc::mbar_wait(&s.drain, 0, spin, &never);
       }
@@ -391,15 +452,20 @@ __global__ void __maxnreg__(168)
     uint32_t G = 0;
     int k = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
-      const ItemInfo it = item_info(a, item, head_groups);
+    // The item's description, its sink logit and the validity of this thread's slot in the
+    // next block are loaded one step ahead (global loads queue behind the producers' gather
+    // traffic, so their latency is long).
+    int item = blockIdx.x;
+    ItemInfo it = item_info(a, item < items ? item : 0, head_groups);
+    float sink_h = (quad == 0 && a.sink) ? __ldg(a.sink + it.hg * AT_H + hb + lane) : 0.f;
+    bool vnext = item < items && slot_row(a, it.cs, it.nc4, slot).valid;
+    for (; item < items && ok; item += gridDim.x, ++k) {
       float lsum[32];                                  // sums of the bf16-rounded weights
-      // sink logit of the head this thread finalises (loaded early, used in the epilogue)
-      const float sink_h = (quad == 0 && a.sink) ? __ldg(a.sink + it.hg * AT_H + hb + lane) : 0.f;
 #pragma unroll
       for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
       for (int j = 0; j < it.nb; ++j, ++G) {
-        const SlotRow sr = slot_row(a, it.cs, it.nc4, j * AT_BLK + slot);   // overlaps the wait
+        const bool valid = vnext;
+        if (j + 1 < it.nb) vnext = slot_row(a, it.cs, it.nc4, (j + 1) * AT_BLK + slot).valid;
         if (tid == 0) A1_TRACE(6, k, j);
         ok = tc::mbar_wait(&s.s_full, G & 1, spin, abort);
         ok = !bar_red_or(3, AT_SOFT, !ok);             // all 256 threads take the same branch
@@ -408,15 +474,13 @@ __global__ void __maxnreg__(168)
         tc::tc_fence_after();
         float z[32];
         tc::tmem_ld32(tmem + lane_base + TM_S + hb, z);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld_dep(z);
 #pragma unroll
-        for (int h = 0; h < 32; ++h) z[h] = sr.valid ? z[h] * scale_log2 : -INFINITY;
-        {
-          float red[32];
-#pragma unroll
-          for (int h = 0; h < 32; ++h) red[h] = z[h];
-          s.red[quad][hb + lane] = xpose_reduce32<true>(red);
-        }
+        for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
+        // the butterfly consumes z; the scores are read from TMEM again (S^T is not
+        // overwritten before this block's P is published) while the block max is combined
+        s.red[quad][hb + lane] = xpose_reduce32<true>(z);
+        tc::tmem_ld32(tmem + lane_base + TM_S + hb, z);
         tc::named_barrier(1, AT_SOFT);
         bool grow = false;
         if (quad == 0) {                               // warps 0 and 4 own heads hb + lane
@@ -433,39 +497,55 @@ __global__ void __maxnreg__(168)
             grow = true;
           }
           s.mcur[h] = mn;
+          s.moff[h] = mn == -INFINITY ? 0.f : mn;
           s.fac[h] = f;
         }
         const bool rescale = bar_red_or(2, AT_SOFT, grow) && j > 0;
-        if (tid == 0) A1_TRACE(11, k, j);
-        uint32_t packed[16];
+        tc::tmem_wait_ld_dep(z);
 #pragma unroll
-        for (int h = 0; h < 32; h += 2) {
-          const float m0 = s.mcur[hb + h], m1 = s.mcur[hb + h + 1];
-          const float p0 = exp2f(z[h] - (m0 == -INFINITY ? 0.f : m0));
-          const float p1 = exp2f(z[h + 1] - (m1 == -INFINITY ? 0.f : m1));
-          __nv_bfloat162 pb2 = __floats2bfloat162_rn(p0, p1);
-          // the denominator sums the same bf16-rounded weights the PV product uses
-          const float2 pr = __bfloat1622float2(pb2);
-          lsum[h] = fmaf(lsum[h], s.fac[hb + h], pr.x);
-          lsum[h + 1] = fmaf(lsum[h + 1], s.fac[hb + h + 1], pr.y);
-          packed[h / 2] = *reinterpret_cast<uint32_t*>(&pb2);
-        }
+        for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
+        if (tid == 0) A1_TRACE(18, k, j);
         // GEMM1 of this block completing implies GEMM2 of the previous block completed (it
         // waited for the chunks that GEMM2 released), so P and O^T are free to touch.
         uint8_t* prow = s.p + slot * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (slot & 7)) << 4)) =
-              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-        if (rescale) {
+        for (int c = 0; c < 4; ++c) {                  // 8 heads -> one 16-byte P store
+          uint32_t pk[4];
 #pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int h = 8 * c + 4 * v;
+            const float4 mo = *reinterpret_cast<const float4*>(&s.moff[hb + h]);
+            const float4 fa = *reinterpret_cast<const float4*>(&s.fac[hb + h]);
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(exp2f(z[h] - mo.x), exp2f(z[h + 1] - mo.y));
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(exp2f(z[h + 2] - mo.z), exp2f(z[h + 3] - mo.w));
+            // the denominator sums the same bf16-rounded weights the PV product uses
+            const float2 r0 = __bfloat1622float2(b0), r1 = __bfloat1622float2(b1);
+            lsum[h] = fmaf(lsum[h], fa.x, r0.x);
+            lsum[h + 1] = fmaf(lsum[h + 1], fa.y, r0.y);
+            lsum[h + 2] = fmaf(lsum[h + 2], fa.z, r1.x);
+            lsum[h + 3] = fmaf(lsum[h + 3], fa.w, r1.y);
+            pk[2 * v] = *reinterpret_cast<uint32_t*>(&b0);
+            pk[2 * v + 1] = *reinterpret_cast<uint32_t*>(&b1);
+          }
+          *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (slot & 7)) << 4)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        if (rescale) {                                 // rare: a head's max grew by > 2^TAU
+#pragma unroll 1
           for (int q = 0; q < 4; ++q) {
-            float o[32];
+            asm volatile("" ::: "memory");             // re-read the factors: keeps them out
+            float o[32];                               // of registers across iterations
             const uint32_t addr = tmem + lane_base + TM_O + 64 * q + hb;
             tc::tmem_ld32(addr, o);
-            tc::tmem_wait_ld();
+            tc::tmem_wait_ld_dep(o);
 #pragma unroll
-            for (int u = 0; u < 32; ++u) o[u] *= s.fac[hb + u];
+            for (int u = 0; u < 32; u += 4) {
+              const float4 fa = *reinterpret_cast<const float4*>(&s.fac[hb + u]);
+              o[u] *= fa.x;
+              o[u + 1] *= fa.y;
+              o[u + 2] *= fa.z;
+              o[u + 3] *= fa.w;
+            }
             tc::tmem_st32(addr, o);
           }
           tc::tmem_wait_st();
@@ -477,6 +557,14 @@ __global__ void __maxnreg__(168)
       }
       if (!ok) break;
       // ---------------------------------------------------------------- epilogue
+      const int nitem = item + gridDim.x;
+      ItemInfo nx = it;
+      float nsink = 0.f;
+      if (nitem < items) {
+        nx = item_info(a, nitem, head_groups);
+        nsink = (quad == 0 && a.sink) ? __ldg(a.sink + nx.hg * AT_H + hb + lane) : 0.f;
+        vnext = slot_row(a, nx.cs, nx.nc4, slot).valid;
+      }
       // GEMM2 of the last block is complete (GEMM1 of that block completing already implies
       // GEMM2 of the block before it, so the phase waited here is unambiguous).
       ok = tc::mbar_wait(&s.o_done, (G - 1) & 1, spin, abort);
@@ -534,11 +622,13 @@ __global__ void __maxnreg__(168)
       }
       tc::tc_fence_before();
       if (tid == 0) A1_TRACE(23, k, 0);
+      it = nx;
+      sink_h = nsink;
     }
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 11) {
+  if (warp == 13) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, TM_COLS);
   }
