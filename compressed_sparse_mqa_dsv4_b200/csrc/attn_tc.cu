@@ -222,7 +222,8 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int item, int h
 
 __global__ void __maxnreg__(128)
     attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q,
-                   const __grid_constant__ CUtensorMap map_local, int head_groups,
+                   const __grid_constant__ CUtensorMap map_local,
+                   const __grid_constant__ CUtensorMap map_o, int head_groups,
                    int items, float scale_log2, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& s = *reinterpret_cast<AttnSmem*>(
@@ -595,36 +596,61 @@ __global__ void __maxnreg__(128)
       }
       tc::named_barrier(1, AT_SOFT);
       if (tid == 0) A1_TRACE(22, k, 0);
-      // O^T tiles: each lane holds one channel for 32 heads; an 8x8 shuffle transpose within
-      // groups of 8 lanes gives each lane 8 consecutive channels of one head -> 16-byte stores
-      // (no shared-memory staging, no barrier).
-      __nv_bfloat16* O = reinterpret_cast<__nv_bfloat16*>(a.O) + ((long long)it.qi * a.H + h0 + hb) * AT_C;
+      // O^T tiles of 128 channels: each lane holds one channel for 32 heads; an 8x8 shuffle
+      // transpose within groups of 8 lanes gives each lane 8 consecutive channels of one head,
+      // which go as one 16-byte store into the P buffer (free now) laid out as two [64 heads x
+      // 64 channels] 128-byte-swizzle boxes; TMA stores the boxes, so the output never goes
+      // through the load/store pipeline the producers' gather is using.
       const int r8 = lane & 7, g8 = lane >> 3;
+      const int box = quad >> 1;
+      const int unit = 4 * (quad & 1) + g8;            // 16-byte unit within the box row
       for (int q = 0; q < 4; ++q) {
         float o[32];
         tc::tmem_ld32(tmem + lane_base + TM_O + 64 * q + hb, o);
-        tc::tmem_wait_ld();
+        tc::tmem_wait_ld_dep(o);
+        if (tid == 0 && q == 1) A1_TRACE(2, k, 0);
+        uint4 pk[4];
 #pragma unroll
         for (int hblk = 0; hblk < 4; ++hblk) {
-          float v[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = o[8 * hblk + i] * s.inv[hb + 8 * hblk + i];
+          const float4 i0 = *reinterpret_cast<const float4*>(&s.inv[hb + 8 * hblk]);
+          const float4 i1 = *reinterpret_cast<const float4*>(&s.inv[hb + 8 * hblk + 4]);
+          float v[8] = {o[8 * hblk] * i0.x,     o[8 * hblk + 1] * i0.y, o[8 * hblk + 2] * i0.z,
+                        o[8 * hblk + 3] * i0.w, o[8 * hblk + 4] * i1.x, o[8 * hblk + 5] * i1.y,
+                        o[8 * hblk + 6] * i1.z, o[8 * hblk + 7] * i1.w};
           transpose8x8(v, r8);
           // lane (g8, r8) now holds head hb + 8*hblk + r8, channels 32*quad + 8*g8 .. +7
-          uint4 pk;
-          pk.x = pack_bf16(v[0], v[1]);
-          pk.y = pack_bf16(v[2], v[3]);
-          pk.z = pack_bf16(v[4], v[5]);
-          pk.w = pack_bf16(v[6], v[7]);
-          *reinterpret_cast<uint4*>(O + (long long)(8 * hblk + r8) * AT_C + 128 * q + 32 * quad + 8 * g8) = pk;
+          pk[hblk] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
+                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
         }
-        if (tid == 0) A1_TRACE(24 + q, k, 0);
+        if (tid == 0 && q == 1) A1_TRACE(16, k, 0);
+        if (q > 0) {                                   // the previous tile's stores read P
+          if (tid == 0) tc::bulk_wait_read();
+          tc::named_barrier(1, AT_SOFT);
+        }
+        if (tid == 0 && q == 1) A1_TRACE(19, k, 0);
+#pragma unroll
+        for (int hblk = 0; hblk < 4; ++hblk) {
+          const int h = hb + 8 * hblk + r8;
+          *reinterpret_cast<uint4*>(s.p + box * (AT_H * 128) + h * 128 + ((unit ^ r8) << 4)) = pk[hblk];
+        }
+        tc::fence_proxy_async_smem();
+        tc::named_barrier(1, AT_SOFT);
+        if (tid == 0) {
+          const int orow = it.qi * a.H + h0;
+          tc::tma_store_2d(&map_o, s.p, 128 * q, orow);
+          tc::tma_store_2d(&map_o, s.p + AT_H * 128, 128 * q + 64, orow);
+          tc::bulk_commit();
+          A1_TRACE(24 + q, k, 0);
+        }
       }
+      // the next item's softmax writes P only after a barrier this thread reaches after here
+      if (tid == 0) tc::bulk_wait_read();
       tc::tc_fence_before();
       if (tid == 0) A1_TRACE(23, k, 0);
       it = nx;
       sink_h = nsink;
     }
+    if (tid == 0) tc::bulk_wait_all();                 // output stores complete before exit
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -657,15 +683,18 @@ int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used) {
   }
   const long long nrows_local = (long long)a.B * a.R;
   if (nrows_local >= (1ll << 31) || !aligned16(a.O)) return DSV4_OK;
-  CUtensorMap mq, mlocal;
+  CUtensorMap mq, mlocal, mo;
   int s = encode_tensor_map_2d(&mq, a.Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_q, 64,
                                AT_H, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (s != DSV4_OK) return s;
+  s = encode_tensor_map_2d(&mo, a.O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_q, 64, AT_H,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
   s = encode_tensor_map_2d(&mlocal, a.local, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_local,
                            64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
   const long long grid = items < sms ? items : sms;
-  attn_tc_kernel<<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(a, mq, mlocal, a.H / AT_H,
+  attn_tc_kernel<<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(a, mq, mlocal, mo, a.H / AT_H,
                                                              (int)items, a.scale * LOG2E,
                                                              spin_limit());
   *used = true;
