@@ -142,27 +142,6 @@ __device__ __forceinline__ float xpose_reduce32(float (&v)[32]) {
   return v[0];
 }
 
-// 8x8 transpose across the 8 lanes of a lane group (r = lane & 7): on entry v[i] is element
-// (row r, column i); on exit v[i] is element (row i, column r). Three exchange stages swap
-// the off-diagonal blocks of size 4, 2 and 1.
-__device__ __forceinline__ void transpose8x8(float (&v)[8], int r) {
-#pragma unroll
-  for (int m = 4; m >= 1; m >>= 1) {
-    const bool hi = (r & m) != 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if ((i & m) == 0) {
-        const float send = hi ? v[i] : v[i + m];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, m);
-        if (hi)
-          v[i] = recv;
-        else
-          v[i + m] = recv;
-      }
-    }
-  }
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
@@ -596,43 +575,46 @@ __global__ void __maxnreg__(128)
       }
       tc::named_barrier(1, AT_SOFT);
       if (tid == 0) A1_TRACE(22, k, 0);
-      // O^T tiles of 128 channels: each lane holds one channel for 32 heads; an 8x8 shuffle
-      // transpose within groups of 8 lanes gives each lane 8 consecutive channels of one head,
-      // which go as one 16-byte store into the P buffer (free now) laid out as two [64 heads x
-      // 64 channels] 128-byte-swizzle boxes; TMA stores the boxes, so the output never goes
-      // through the load/store pipeline the producers' gather is using.
-      const int r8 = lane & 7, g8 = lane >> 3;
-      const int box = quad >> 1;
-      const int unit = 4 * (quad & 1) + g8;            // 16-byte unit within the box row
-      for (int q = 0; q < 4; ++q) {
-        float o[32];
-        tc::tmem_ld32(tmem + lane_base + TM_O + 64 * q + hb, o);
-        tc::tmem_wait_ld_dep(o);
-        if (tid == 0 && q == 1) A1_TRACE(2, k, 0);
-        uint4 pk[4];
+      // O^T tiles of 128 channels. Each warp reads its 32 channels x 32 heads as two 16-lane
+      // loads in the m8n8 fragment layout (thread t: channels c0 + t/4 and c0 + 8 + t/4, head
+      // pairs 2(t%4) + 8k), scales and packs them to bf16 and writes them with transposing
+      // 8x8 matrix stores, so each stored 16-byte row is 8 consecutive channels of one head.
+      // The rows land in the P buffer (free now) as two [64 heads x 64 channels] 128-byte
+      // swizzle boxes, which TMA stores to O.
+      const int tq = lane & 3, mrow = lane & 7, mat = lane >> 3;
+      float2 inv2[4];                                  // 1/denominator of this thread's heads
 #pragma unroll
-        for (int hblk = 0; hblk < 4; ++hblk) {
-          const float4 i0 = *reinterpret_cast<const float4*>(&s.inv[hb + 8 * hblk]);
-          const float4 i1 = *reinterpret_cast<const float4*>(&s.inv[hb + 8 * hblk + 4]);
-          float v[8] = {o[8 * hblk] * i0.x,     o[8 * hblk + 1] * i0.y, o[8 * hblk + 2] * i0.z,
-                        o[8 * hblk + 3] * i0.w, o[8 * hblk + 4] * i1.x, o[8 * hblk + 5] * i1.y,
-                        o[8 * hblk + 6] * i1.z, o[8 * hblk + 7] * i1.w};
-          transpose8x8(v, r8);
-          // lane (g8, r8) now holds head hb + 8*hblk + r8, channels 32*quad + 8*g8 .. +7
-          pk[hblk] = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+      for (int kk = 0; kk < 4; ++kk) inv2[kk] = *reinterpret_cast<const float2*>(&s.inv[hb + 8 * kk + 2 * tq]);
+      const uint32_t p0 = tc::smem_u32(s.p) + (uint32_t)((quad >> 1) * (AT_H * 128));
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pk[2][8];                             // [channel half][matrix slot]
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          float v[16];
+          tc::tmem_ld16x256b_x4(tmem + ((uint32_t)(32 * quad + 16 * hh) << 16) + TM_O + 64 * q + hb, v);
+          tc::tmem_wait_ld_dep16(v);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            pk[hh][2 * kk] = pack_bf16(v[4 * kk] * inv2[kk].x, v[4 * kk + 1] * inv2[kk].y);
+            pk[hh][2 * kk + 1] = pack_bf16(v[4 * kk + 2] * inv2[kk].x, v[4 * kk + 3] * inv2[kk].y);
+          }
         }
-        if (tid == 0 && q == 1) A1_TRACE(16, k, 0);
         if (q > 0) {                                   // the previous tile's stores read P
           if (tid == 0) tc::bulk_wait_read();
           tc::named_barrier(1, AT_SOFT);
         }
-        if (tid == 0 && q == 1) A1_TRACE(19, k, 0);
 #pragma unroll
-        for (int hblk = 0; hblk < 4; ++hblk) {
-          const int h = hb + 8 * hblk + r8;
-          *reinterpret_cast<uint4*>(s.p + box * (AT_H * 128) + h * 128 + ((unit ^ r8) << 4)) = pk[hblk];
-        }
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int jx = 0; jx < 2; ++jx) {
+            // matrices {A_k, B_k, A_k+1, B_k+1}, k = 2 jx: A = channels c0..c0+7, B = c0+8..
+            const int kk = 2 * jx + (mat >> 1);
+            const int h = hb + 8 * kk + mrow;          // stored row: one head
+            const int unit = 4 * (quad & 1) + 2 * hh + (mat & 1);
+            const uint32_t addr = p0 + (uint32_t)(h * 128 + ((unit ^ mrow) << 4));
+            tc::stmatrix_x4_trans(addr, pk[hh][4 * jx], pk[hh][4 * jx + 1], pk[hh][4 * jx + 2],
+                                  pk[hh][4 * jx + 3]);
+          }
         tc::fence_proxy_async_smem();
         tc::named_barrier(1, AT_SOFT);
         if (tid == 0) {

@@ -220,12 +220,43 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 16 lanes x 256 bits, four 8-column chunks: thread t, register 4k+i holds lane
+// (base + t/4 + 8*(i>>1)), column (8k + 2*(t%4) + (i&1)) -- the m8n8 fragment layout.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32"
+      " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Four 8x8 b16 matrices, each stored transposed: register j of thread t holds elements
+// (t/4, 2(t%4)) and (t/4, 2(t%4)+1) of matrix j; threads 8j..8j+7 give the addresses of
+// the stored rows 0..7 of matrix j (stored row r = column r of the matrix).
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1,
+                                                  uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 // Wait for this thread's tcgen05.ld and tie the loaded registers to the wait, so the
 // compiler cannot move their first use above it.
 __device__ __forceinline__ void tmem_wait_ld_dep(float (&v)[32]) {
   tmem_wait_ld();
 #pragma unroll
   for (int i = 0; i < 32; ++i) asm volatile("" : "+f"(v[i]));
+}
+
+__device__ __forceinline__ void tmem_wait_ld_dep16(float (&v)[16]) {
+  tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) asm volatile("" : "+f"(v[i]));
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
