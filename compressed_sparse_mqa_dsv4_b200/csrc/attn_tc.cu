@@ -457,58 +457,94 @@ __global__ void __maxnreg__(128)
         tc::tmem_wait_ld_dep(z);
 #pragma unroll
         for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
-        // the butterfly consumes z; the scores are read from TMEM again (S^T is not
-        // overwritten before this block's P is published) while the block max is combined
-        s.red[quad][hb + lane] = xpose_reduce32<true>(z);
-        tc::tmem_ld32(tmem + lane_base + TM_S + hb, z);
-        tc::named_barrier(1, AT_SOFT);
-        bool grow = false;
-        if (quad == 0) {                               // warps 0 and 4 own heads hb + lane
-          const int h = hb + lane;
-          const float bm = fmaxf(fmaxf(s.red[0][h], s.red[1][h]), fmaxf(s.red[2][h], s.red[3][h]));
-          const float mo = s.mcur[h];
-          float mn = mo, f = 1.f;
-          if (mo == -INFINITY) {
-            mn = bm;
-            f = 0.f;
-          } else if (bm > mo + TAU) {
-            mn = bm;
-            f = exp2f(mo - mn);
-            grow = true;
-          }
-          s.mcur[h] = mn;
-          s.moff[h] = mn == -INFINITY ? 0.f : mn;
-          s.fac[h] = f;
-        }
-        const bool rescale = bar_red_or(2, AT_SOFT, grow) && j > 0;
-        tc::tmem_wait_ld_dep(z);
-#pragma unroll
-        for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
-        if (tid == 0) A1_TRACE(18, k, j);
         // GEMM1 of this block completing implies GEMM2 of the previous block completed (it
         // waited for the chunks that GEMM2 released), so P and O^T are free to touch.
         uint8_t* prow = s.p + slot * 128;
+        bool rescale = false;
+        // After an item's first block every head has a finite running max m. Weights taken
+        // against m are exact whatever m is (m cancels in the normalisation); they only have
+        // to stay bounded, so the block maxima are needed just when some score exceeds its
+        // running max by more than TAU -- then the exact path below recomputes this block.
+        bool exact = j == 0;
+        if (!exact) {
+          uint32_t pk[16];
+          bool over = false;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {                  // 8 heads -> one 16-byte P store
-          uint32_t pk[4];
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const int h = 8 * c + 4 * v;
-            const float4 mo = *reinterpret_cast<const float4*>(&s.moff[hb + h]);
-            const float4 fa = *reinterpret_cast<const float4*>(&s.fac[hb + h]);
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(exp2f(z[h] - mo.x), exp2f(z[h + 1] - mo.y));
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(exp2f(z[h + 2] - mo.z), exp2f(z[h + 3] - mo.w));
-            // the denominator sums the same bf16-rounded weights the PV product uses
-            const float2 r0 = __bfloat1622float2(b0), r1 = __bfloat1622float2(b1);
-            lsum[h] = fmaf(lsum[h], fa.x, r0.x);
-            lsum[h + 1] = fmaf(lsum[h + 1], fa.y, r0.y);
-            lsum[h + 2] = fmaf(lsum[h + 2], fa.z, r1.x);
-            lsum[h + 3] = fmaf(lsum[h + 3], fa.w, r1.y);
-            pk[2 * v] = *reinterpret_cast<uint32_t*>(&b0);
-            pk[2 * v + 1] = *reinterpret_cast<uint32_t*>(&b1);
+          for (int h = 0; h < 32; h += 4) {
+            const float4 m4 = *reinterpret_cast<const float4*>(&s.mcur[hb + h]);
+            over |= !(z[h] <= m4.x + TAU) | !(z[h + 1] <= m4.y + TAU) |
+                    !(z[h + 2] <= m4.z + TAU) | !(z[h + 3] <= m4.w + TAU);
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(exp2f(z[h] - m4.x), exp2f(z[h + 1] - m4.y));
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(exp2f(z[h + 2] - m4.z), exp2f(z[h + 3] - m4.w));
+            pk[h / 2] = *reinterpret_cast<uint32_t*>(&b0);
+            pk[h / 2 + 1] = *reinterpret_cast<uint32_t*>(&b1);
           }
-          *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (slot & 7)) << 4)) =
-              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          exact = bar_red_or(2, AT_SOFT, over);
+          if (!exact) {
+#pragma unroll
+            for (int h = 0; h < 32; h += 2) {
+              // the denominator sums the same bf16-rounded weights the PV product uses
+              const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[h / 2]));
+              lsum[h] += r.x;
+              lsum[h + 1] += r.y;
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (slot & 7)) << 4)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
+        }
+        if (exact) {
+          // the butterfly consumes z; the scores are read from TMEM again (S^T is not
+          // overwritten before this block's P is published) while the block max is combined
+          s.red[quad][hb + lane] = xpose_reduce32<true>(z);
+          tc::tmem_ld32(tmem + lane_base + TM_S + hb, z);
+          tc::named_barrier(1, AT_SOFT);
+          bool grow = false;
+          if (quad == 0) {                             // warps 0 and 4 own heads hb + lane
+            const int h = hb + lane;
+            const float bm = fmaxf(fmaxf(s.red[0][h], s.red[1][h]), fmaxf(s.red[2][h], s.red[3][h]));
+            const float mo = s.mcur[h];
+            float mn = mo, f = 1.f;
+            if (mo == -INFINITY) {
+              mn = bm;
+              f = 0.f;
+            } else if (bm > mo + TAU) {
+              mn = bm;
+              f = exp2f(mo - mn);
+              grow = true;
+            }
+            s.mcur[h] = mn;
+            s.moff[h] = mn == -INFINITY ? 0.f : mn;
+            s.fac[h] = f;
+          }
+          rescale = bar_red_or(2, AT_SOFT, grow) && j > 0;
+          tc::tmem_wait_ld_dep(z);
+#pragma unroll
+          for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
+          if (tid == 0) A1_TRACE(18, k, j);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {                // 8 heads -> one 16-byte P store
+            uint32_t pk[4];
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const int h = 8 * c + 4 * v;
+              const float4 mo = *reinterpret_cast<const float4*>(&s.moff[hb + h]);
+              const float4 fa = *reinterpret_cast<const float4*>(&s.fac[hb + h]);
+              __nv_bfloat162 b0 = __floats2bfloat162_rn(exp2f(z[h] - mo.x), exp2f(z[h + 1] - mo.y));
+              __nv_bfloat162 b1 = __floats2bfloat162_rn(exp2f(z[h + 2] - mo.z), exp2f(z[h + 3] - mo.w));
+              // the denominator sums the same bf16-rounded weights the PV product uses
+              const float2 r0 = __bfloat1622float2(b0), r1 = __bfloat1622float2(b1);
+              lsum[h] = fmaf(lsum[h], fa.x, r0.x);
+              lsum[h + 1] = fmaf(lsum[h + 1], fa.y, r0.y);
+              lsum[h + 2] = fmaf(lsum[h + 2], fa.z, r1.x);
+              lsum[h + 3] = fmaf(lsum[h + 3], fa.w, r1.y);
+              pk[2 * v] = *reinterpret_cast<uint32_t*>(&b0);
+              pk[2 * v + 1] = *reinterpret_cast<uint32_t*>(&b1);
+            }
+            *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (slot & 7)) << 4)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
         }
         if (rescale) {                                 // rare: a head's max grew by > 2^TAU
 #pragma unroll 1
