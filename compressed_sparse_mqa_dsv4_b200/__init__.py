@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "DSV4Error", "lib", "LIB_PATH", "F32", "BF16", "FP4",
     "dsv4_compress", "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
-    "dsv4_hybrid_sparse_attn", "dsv4_check_errors",
+    "dsv4_hybrid_sparse_attn", "dsv4_hybrid_sparse_attn_workspace_size", "dsv4_check_errors",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsv4.so")
@@ -28,7 +28,7 @@ F32, BF16, FP4 = 0, 1, 2
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"libdsv4.so not found at {LIB_PATH}: build it with "
-        "`python -m compressed_sparse_mqa_dsv4_b200.build` (nvcc, sm_100a)")
+        "`python compressed_sparse_mqa_dsv4_b200/build.py` (nvcc, sm_100a)")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -50,7 +50,9 @@ lib.dsv4_index_topk.argtypes = [_I, _P, _P, _P, _P, _P, _L, _P, _P, _I, _I, _I, 
                                 _P, _P, _P, _L, _P, _S, _P]
 lib.dsv4_hybrid_sparse_attn.restype = _I
 lib.dsv4_hybrid_sparse_attn.argtypes = [_I, _P, _P, _L, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
-                                        _I, _I, _I, _P, _F, _P, _P, _P]
+                                        _I, _I, _I, _P, _F, _P, _P, _P, _S, _P]
+lib.dsv4_hybrid_sparse_attn_workspace_size.restype = _S
+lib.dsv4_hybrid_sparse_attn_workspace_size.argtypes = [_I, _I, _I, _I]
 
 
 class DSV4Error(RuntimeError):
@@ -177,11 +179,14 @@ def dsv4_hybrid_sparse_attn(Q: torch.Tensor, pool: torch.Tensor, kv_row_off: tor
                             local: torch.Tensor, q_pos0: torch.Tensor, m: int, w: int,
                             sink: Optional[torch.Tensor] = None, scale: Optional[float] = None,
                             O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                            want_lse: bool = True, stream=None):
+                            want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
+                            stream=None):
     """Hybrid shared-KV MQA. Q [B, nq, H, c]; pool [rows, c]; local [B, R, c].
 
     idx/counts: int32 [B, nq, k] / [B, nq] (CSA) or None (HCA dense read with ratio m).
     Returns (O [B, nq, H, c], lse fp32 [B, nq, H] or None).
+    workspace: uint8 device scratch for split candidate lists (decode); allocated here when
+    the request would use it and none is given.
     """
     _dev(Q, "Q"), _dev(pool, "pool", Q.dtype), _dev(local, "local", Q.dtype)
     _dev(kv_row_off, "kv_row_off", torch.int64), _dev(q_pos0, "q_pos0", torch.int32)
@@ -203,12 +208,21 @@ def dsv4_hybrid_sparse_attn(Q: torch.Tensor, pool: torch.Tensor, kv_row_off: tor
         O = torch.empty_like(Q)
     if lse is None and want_lse:
         lse = torch.empty(B, nq, H, dtype=torch.float32, device=Q.device)
+    ws_bytes = dsv4_hybrid_sparse_attn_workspace_size(B, nq, H, c)
+    if ws_bytes and (workspace is None or workspace.numel() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
+    ws_bytes = workspace.numel() if workspace is not None else 0
     _check(lib.dsv4_hybrid_sparse_attn(_code(Q.dtype), _ptr(Q), _ptr(pool), pool.shape[0],
                                        _ptr(kv_row_off), idx_p, _ptr(counts), k, _ptr(local),
                                        R, _ptr(q_pos0), B, nq, H, c, m, w, _ptr(sink),
-                                       float(scale), _ptr(O), _ptr(lse), _stream(stream)),
+                                       float(scale), _ptr(O), _ptr(lse), _ptr(workspace),
+                                       ws_bytes, _stream(stream)),
            "dsv4_hybrid_sparse_attn")
     return O, lse
+
+
+def dsv4_hybrid_sparse_attn_workspace_size(B: int, nq: int, H: int, c: int) -> int:
+    return int(lib.dsv4_hybrid_sparse_attn_workspace_size(B, nq, H, c))
 
 
 def dsv4_check_errors(stream=None):

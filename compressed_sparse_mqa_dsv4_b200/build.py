@@ -1,6 +1,6 @@
 """Build libdsv4.so in-tree: every csrc/*.cu compiled for sm_100a with nvcc, then linked.
 
-Usage: python -m compressed_sparse_mqa_dsv4_b200.build [--force] [-j N]
+Usage: python compressed_sparse_mqa_dsv4_b200/build.py [--force] [-j N]
 Objects go to <repo>/_build/ (not committed); the library lands next to this file.
 """
 from __future__ import annotations

@@ -20,6 +20,11 @@ struct AttnArgs {
   float scale;
   void* O;
   float* lse;
+  // split candidate lists (tensor-core path): nsplit partials per (query, head group) in
+  // part_o [items * nsplit][64 heads][c] fp32 and part_ml [items * nsplit][64] (m, L)
+  int nsplit;
+  float* part_o;
+  float2* part_ml;
 };
 
 // Candidate j of query (b, t): compressed part first, then the local window
@@ -78,6 +83,10 @@ __device__ __forceinline__ long long candidate_row(const AttnArgs& a, const Cand
 
 int launch_attn_simt(const AttnArgs& a, int dtype, cudaStream_t st);
 int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used);
+// Split partials: at most this many splits per (query, head group); bytes per split of one
+// (query, 64-head group) item.
+constexpr int ATTN_MAX_SPLIT = 8;
+long long attn_split_bytes_per_item(int c);
 int launch_attn_tc2(const AttnArgs& a, cudaStream_t st, bool* used);
 
 }  // namespace dsv4

@@ -182,23 +182,32 @@ __device__ __forceinline__ SlotRow slot_row(const AttnArgs& a, const CandidateSe
   return r;
 }
 
+// Work item = (query, group of 64 heads, split). With nsplit > 1 the candidate blocks of a
+// query are divided evenly among its splits (a split may own none) and each split leaves
+// an unnormalised partial for the combine kernel.
 struct ItemInfo {
-  int qi, hg, nc4, nb;
+  int qi, hg, nc4, nb, jb, je, base;
   CandidateSet cs;
 };
 
+template <bool kSplit>
 __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int item, int head_groups) {
   ItemInfo it;
-  it.qi = item / head_groups;
-  it.hg = item % head_groups;
+  const int split = kSplit ? item % a.nsplit : 0;
+  it.base = kSplit ? item / a.nsplit : item;
+  it.qi = it.base / head_groups;
+  it.hg = it.base % head_groups;
   const int b = it.qi / a.nq, i = it.qi % a.nq;
   it.cs = make_candidates(a, b, i);
   it.nc4 = (it.cs.n_comp + 3) & ~3;
   const int nl4 = (it.cs.n_local + 3) & ~3;
   it.nb = (it.nc4 + nl4 + AT_BLK - 1) / AT_BLK;
+  it.jb = kSplit ? (int)((long long)split * it.nb / a.nsplit) : 0;
+  it.je = kSplit ? (int)((long long)(split + 1) * it.nb / a.nsplit) : it.nb;
   return it;
 }
 
+template <bool kSplit>
 __global__ void __maxnreg__(128)
     attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q,
                    const __grid_constant__ CUtensorMap map_local,
@@ -241,8 +250,9 @@ __global__ void __maxnreg__(128)
     int k = 0;
     bool ok = true;
     if (pt == 0) tc::prefetch_tensormap(&map_q);
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
-      const ItemInfo it = item_info(a, item, head_groups);
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+      const ItemInfo it = item_info<kSplit>(a, item, head_groups);
+      if (kSplit && it.je <= it.jb) continue;          // a split without blocks: no work
       ok = !gate(GATE_ITEM, false);                    // the Q buffer is free (or abort)
       if (!ok) break;
       if (pt == 0) {
@@ -250,7 +260,7 @@ __global__ void __maxnreg__(128)
         const int qrow = it.qi * a.H + it.hg * AT_H;
         for (int c = 0; c < AT_CHUNKS; ++c) tc::tma_load_2d(s.q[c], &map_q, &s.q_full, 64 * c, qrow);
       }
-      for (int j = 0; j < it.nb && ok; ++j, ++G) {
+      for (int j = it.jb; j < it.je && ok; ++j, ++G) {
         // Local-window slots of this block whose rows are contiguous (no ring wrap) and start
         // on a 32-slot boundary come in by 2D TMA boxes of 32 rows; the rest by cp.async.
         const int bs = j * AT_BLK;
@@ -320,6 +330,7 @@ __global__ void __maxnreg__(128)
         if (pt == 0) A1_TRACE(1, k, j);
         tc::named_barrier(5, AT_PROD);                 // rowaddr[] is rewritten next block
       }
+      ++k;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (pt == 0 && *abort) {
@@ -345,11 +356,13 @@ __global__ void __maxnreg__(128)
     uint32_t G = 0;
     int k = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
-      const ItemInfo it = item_info(a, item, head_groups);
+    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+      const ItemInfo it = item_info<kSplit>(a, item, head_groups);
+      if (kSplit && it.je <= it.jb) continue;
       if (k > 0) ok = wwait(&s.q_empty, (uint32_t)((k - 1) & 1));
       ok = !gate(GATE_ITEM, !ok || *abort != 0);
-      for (int j = 0; j < it.nb && ok; ++j, ++G) {
+      ++k;
+      for (int j = it.jb; j < it.je && ok; ++j, ++G) {
         if (G == 0) continue;
         for (int q = 0; q < 4; ++q) {
           if (wwait(&s.ch_empty[q], (G - 1) & 1))
@@ -377,10 +390,12 @@ __global__ void __maxnreg__(128)
       uint32_t G = 0;
       int k = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < items && ok; item += gridDim.x, ++k) {
-        const ItemInfo it = item_info(a, item, head_groups);
+      for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+        const ItemInfo it = item_info<kSplit>(a, item, head_groups);
+        if (kSplit && it.je <= it.jb) continue;
         ok = wwait(&s.q_full, (uint32_t)(k & 1));
-        for (int j = 0; j < it.nb && ok; ++j, ++G) {
+        ++k;
+        for (int j = it.jb; j < it.je && ok; ++j, ++G) {
 #pragma unroll
           for (int c = 0; c < AT_CHUNKS; ++c) {
             ok = wwait(&s.ch_full[c], G & 1);
@@ -397,12 +412,12 @@ __global__ void __maxnreg__(128)
           if (!ok) break;
           tc::mma_commit_warp(&s.s_full);
           if (lane == 0) A1_TRACE(3, k, j);
-          if (j + 1 == it.nb) tc::mma_commit_warp(&s.q_empty);
+          if (j + 1 == it.je) tc::mma_commit_warp(&s.q_empty);
           ok = wwait(&s.p_full, G & 1);
           if (!ok) break;
           if (lane == 0) A1_TRACE(4, k, j);
           tc::tc_fence_after();
-          const uint32_t acc0 = j > 0 ? 1u : 0u;
+          const uint32_t acc0 = j > it.jb ? 1u : 0u;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
 #pragma unroll
@@ -436,16 +451,26 @@ __global__ void __maxnreg__(128)
     // next block are loaded one step ahead (global loads queue behind the producers' gather
     // traffic, so their latency is long).
     int item = blockIdx.x;
-    ItemInfo it = item_info(a, item < items ? item : 0, head_groups);
+    ItemInfo it = item_info<kSplit>(a, item < items ? item : 0, head_groups);
     float sink_h = (quad == 0 && a.sink) ? __ldg(a.sink + it.hg * AT_H + hb + lane) : 0.f;
-    bool vnext = item < items && slot_row(a, it.cs, it.nc4, slot).valid;
-    for (; item < items && ok; item += gridDim.x, ++k) {
+    bool vnext = item < items && it.je > it.jb && slot_row(a, it.cs, it.nc4, it.jb * AT_BLK + slot).valid;
+    for (; item < items && ok; item += gridDim.x) {
+      if (kSplit && it.je <= it.jb) {                  // a split without blocks: empty partial
+        if (quad == 0) a.part_ml[((long long)item * AT_H + hb + lane)] = make_float2(-INFINITY, 0.f);
+        const int nitem = item + gridDim.x;
+        if (nitem < items) {
+          it = item_info<kSplit>(a, nitem, head_groups);
+          sink_h = (quad == 0 && a.sink) ? __ldg(a.sink + it.hg * AT_H + hb + lane) : 0.f;
+          vnext = it.je > it.jb && slot_row(a, it.cs, it.nc4, it.jb * AT_BLK + slot).valid;
+        }
+        continue;
+      }
       float lsum[32];                                  // sums of the bf16-rounded weights
 #pragma unroll
       for (int h = 0; h < 32; ++h) lsum[h] = 0.f;
-      for (int j = 0; j < it.nb; ++j, ++G) {
+      for (int j = it.jb; j < it.je; ++j, ++G) {
         const bool valid = vnext;
-        if (j + 1 < it.nb) vnext = slot_row(a, it.cs, it.nc4, (j + 1) * AT_BLK + slot).valid;
+        if (j + 1 < it.je) vnext = slot_row(a, it.cs, it.nc4, (j + 1) * AT_BLK + slot).valid;
         if (tid == 0) A1_TRACE(6, k, j);
         ok = tc::mbar_wait(&s.s_full, G & 1, spin, abort);
         ok = !bar_red_or(3, AT_SOFT, !ok);             // all 256 threads take the same branch
@@ -465,7 +490,7 @@ __global__ void __maxnreg__(128)
         // against m are exact whatever m is (m cancels in the normalisation); they only have
         // to stay bounded, so the block maxima are needed just when some score exceeds its
         // running max by more than TAU -- then the exact path below recomputes this block.
-        bool exact = j == 0;
+        bool exact = j == it.jb;
         if (!exact) {
           uint32_t pk[16];
           bool over = false;
@@ -518,7 +543,7 @@ __global__ void __maxnreg__(128)
             s.moff[h] = mn == -INFINITY ? 0.f : mn;
             s.fac[h] = f;
           }
-          rescale = bar_red_or(2, AT_SOFT, grow) && j > 0;
+          rescale = bar_red_or(2, AT_SOFT, grow) && j > it.jb;
           tc::tmem_wait_ld_dep(z);
 #pragma unroll
           for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
@@ -577,9 +602,9 @@ __global__ void __maxnreg__(128)
       ItemInfo nx = it;
       float nsink = 0.f;
       if (nitem < items) {
-        nx = item_info(a, nitem, head_groups);
+        nx = item_info<kSplit>(a, nitem, head_groups);
         nsink = (quad == 0 && a.sink) ? __ldg(a.sink + nx.hg * AT_H + hb + lane) : 0.f;
-        vnext = slot_row(a, nx.cs, nx.nc4, slot).valid;
+        vnext = nx.je > nx.jb && slot_row(a, nx.cs, nx.nc4, nx.jb * AT_BLK + slot).valid;
       }
       // GEMM2 of the last block is complete (GEMM1 of that block completing already implies
       // GEMM2 of the block before it, so the phase waited here is unambiguous).
@@ -592,6 +617,29 @@ __global__ void __maxnreg__(128)
       tc::named_barrier(1, AT_SOFT);
       if (tid == 0) A1_TRACE(21, k, 0);
       const int h0 = it.hg * AT_H;
+      if (kSplit) {
+        // partial of this split: running max m (log2 units), denominator L relative to m and
+        // the unnormalised O^T, all fp32; the combine kernel applies the sink and normalises
+        if (quad == 0) {
+          const int h = hb + lane;
+          const float L = (s.red[0][h] + s.red[1][h]) + (s.red[2][h] + s.red[3][h]);
+          a.part_ml[(long long)item * AT_H + h] = make_float2(s.mcur[h], L);
+          s.mcur[h] = -INFINITY;
+        }
+        float* po = a.part_o + ((long long)item * AT_H + hb) * AT_C + 32 * quad + lane;
+        for (int q = 0; q < 4; ++q) {
+          float o[32];
+          tc::tmem_ld32(tmem + lane_base + TM_O + 64 * q + hb, o);
+          tc::tmem_wait_ld_dep(o);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) po[(long long)u * AT_C + 128 * q] = o[u];
+        }
+        tc::tc_fence_before();
+        ++k;
+        it = nx;
+        sink_h = nsink;
+        continue;
+      }
       if (quad == 0) {
         const int h = hb + lane;
         const float L = (s.red[0][h] + s.red[1][h]) + (s.red[2][h] + s.red[3][h]);
@@ -665,6 +713,7 @@ __global__ void __maxnreg__(128)
       if (tid == 0) tc::bulk_wait_read();
       tc::tc_fence_before();
       if (tid == 0) A1_TRACE(23, k, 0);
+      ++k;
       it = nx;
       sink_h = nsink;
     }
@@ -678,9 +727,65 @@ __global__ void __maxnreg__(128)
   }
 }
 
+// Merges the nsplit partials of every (query, head group): one warp per head, the combined
+// max M over the splits and the sink, weights 2^(m_s - M), one normalisation, bf16 output,
+// LSE. Splits without candidates carry m = -inf and are not read.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const AttnArgs a, int head_groups) {
+  const int base = blockIdx.x;
+  const int qi = base / head_groups, hg = base % head_groups;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.nsplit;
+  for (int r = 0; r < AT_H / 8; ++r) {
+    const int hl = 8 * warp + r;                       // head within the group
+    const int h = hg * AT_H + hl;
+    const float2 ml = lane < S ? a.part_ml[((long long)base * S + lane) * AT_H + hl]
+                               : make_float2(-INFINITY, 0.f);
+    float M = ml.x;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float s2 = a.sink ? __ldg(a.sink + h) * LOG2E : -INFINITY;
+    M = fmaxf(M, s2);
+    const float e = (ml.x == -INFINITY || M == -INFINITY) ? 0.f : exp2f(ml.x - M);
+    float den = e * ml.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    if (a.sink && M != -INFINITY) den += exp2f(s2 - M);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    float acc[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) acc[u] = 0.f;
+    for (int sp = 0; sp < S; ++sp) {
+      const float es = __shfl_sync(0xffffffffu, e, sp);
+      if (es == 0.f) continue;
+      const float4* src = reinterpret_cast<const float4*>(
+          a.part_o + (((long long)base * S + sp) * AT_H + hl) * AT_C + 16 * lane);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const float4 x = src[v];
+        acc[4 * v] = fmaf(es, x.x, acc[4 * v]);
+        acc[4 * v + 1] = fmaf(es, x.y, acc[4 * v + 1]);
+        acc[4 * v + 2] = fmaf(es, x.z, acc[4 * v + 2]);
+        acc[4 * v + 3] = fmaf(es, x.w, acc[4 * v + 3]);
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.O) +
+                                          ((long long)qi * a.H + h) * AT_C + 16 * lane);
+    dst[0] = make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
+                        pack_bf16(acc[4] * inv, acc[5] * inv), pack_bf16(acc[6] * inv, acc[7] * inv));
+    dst[1] = make_uint4(pack_bf16(acc[8] * inv, acc[9] * inv), pack_bf16(acc[10] * inv, acc[11] * inv),
+                        pack_bf16(acc[12] * inv, acc[13] * inv), pack_bf16(acc[14] * inv, acc[15] * inv));
+    if (lane == 0 && a.lse)
+      a.lse[(long long)qi * a.H + h] = (den > 0.f && M != -INFINITY) ? (M + log2f(den)) * LN2 : -INFINITY;
+  }
+}
+
 }  // namespace
 
-int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used) {
+// Bytes of split partials per (query, head group) and split.
+long long attn_split_bytes_per_item(int c) { return (long long)AT_H * ((long long)c * 4 + 8); }
+
+int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
+  AttnArgs a = a_in;
   *used = false;
   const char* force = std::getenv("DSV4_FORCE_SIMT");
   if (force && force[0] == '1') return DSV4_OK;
@@ -695,8 +800,11 @@ int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (sms <= 0) sms = 148;
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)AT_SMEM);
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)AT_SMEM);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(attn_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)AT_SMEM);
     if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "attn_tc: %s", cudaGetErrorString(e));
   }
   const long long nrows_local = (long long)a.B * a.R;
@@ -711,12 +819,35 @@ int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used) {
   s = encode_tensor_map_2d(&mlocal, a.local, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_local,
                            64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
-  const long long grid = items < sms ? items : sms;
-  attn_tc_kernel<<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(a, mq, mlocal, mo, a.H / AT_H,
-                                                             (int)items, a.scale * LOG2E,
-                                                             spin_limit());
+  // Few (query, head group) items: split each candidate list so that about two work items
+  // per SM exist, as far as the caller's workspace (a.nsplit = its capacity) allows.
+  // A selected list has at most round4(k) + round4(w) candidates; a split must keep at least
+  // 4 blocks to pay for its own Q load, setup and partial write.
+  int nsplit = 1;
+  if (a.part_o && a.nsplit > 1 && items < sms) {
+    nsplit = (int)((2 * sms + items - 1) / items);
+    if (nsplit > a.nsplit) nsplit = a.nsplit;
+    if (a.idx) {
+      const int nb_max = (((a.k + 3) & ~3) + ((a.w + 3) & ~3) + AT_BLK - 1) / AT_BLK;
+      if (nsplit > nb_max / 4) nsplit = nb_max / 4 > 1 ? nb_max / 4 : 1;
+    }
+  }
+  a.nsplit = nsplit;
+  if (nsplit > 1)
+    a.part_ml = reinterpret_cast<float2*>(a.part_o + items * nsplit * AT_H * (long long)AT_C);
+  const long long work = items * nsplit;
+  const long long grid = work < sms ? work : sms;
+  if (nsplit > 1)
+    attn_tc_kernel<true><<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(
+        a, mq, mlocal, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
+  else
+    attn_tc_kernel<false><<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(
+        a, mq, mlocal, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
   *used = true;
-  return launch_status("hybrid attention (tensor cores)");
+  int s2 = launch_status("hybrid attention (tensor cores)");
+  if (s2 != DSV4_OK || nsplit == 1) return s2;
+  attn_combine_kernel<<<(unsigned)items, 256, 0, st>>>(a, a.H / AT_H);
+  return launch_status("hybrid attention split combine");
 }
 
 }  // namespace dsv4

@@ -84,15 +84,27 @@ static long long scores_ld_for(int max_entries) { return round_up(max_entries > 
 
 static const long long kScoreChunkBytes = 256ll << 20;
 
+// Workspace bytes per query row: its fp32 scores and, for long rows, the candidate blocks
+// of the two-stage top-k (k scores + k entry indices per segment).
+static long long candidate_bytes_per_row(int max_entries, int k) {
+  const int nseg = topk_segments(max_entries);
+  return nseg > 1 ? (long long)nseg * k * 8 : 0;
+}
+
+// Rows of the workspace layout [scores: rows x ld fp32][candidate scores][candidate indices]
+static long long workspace_bytes_for(long long rows, long long ld, long long cand_per_row) {
+  return round_up(rows * ld * 4, 256) + round_up(rows * cand_per_row, 256);
+}
+
 extern "C" size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k) {
-  (void)k;
   if (B <= 0 || nq <= 0 || max_entries <= 0) return 0;
   const long long ld = scores_ld_for(max_entries);
+  const long long cand = candidate_bytes_per_row(max_entries, k > 0 ? k : 0);
   const long long total = (long long)B * nq;
-  long long rows = kScoreChunkBytes / (ld * 4);
+  long long rows = kScoreChunkBytes / (ld * 4 + cand);
   if (rows < 1) rows = 1;
   if (rows > total) rows = total;
-  return (size_t)round_up(rows * ld * 4, 256);
+  return (size_t)workspace_bytes_for(rows, ld, cand);
 }
 
 extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_scales,
@@ -126,6 +138,9 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   a.B = B; a.nq = nq; a.H_I = H_I; a.c_I = c_I; a.m = m; a.k = k; a.max_e = max_entries;
   a.idx = idx;
   a.counts = counts;
+  a.nseg = 1;
+  a.cand_score = nullptr;
+  a.cand_idx = nullptr;
   cudaStream_t st = (cudaStream_t)stream;
   const int total = B * nq;
   int chunk;
@@ -134,17 +149,28 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
       return fail(DSV4_ERR_INVALID_ARG, "dsv4_index_topk: scores_ld %lld < max_entries %d",
                   (long long)scores_ld, max_entries);
     a.scores = scores_out; a.scores_ld = scores_ld > 0 ? scores_ld : 1;
-    chunk = total;
+    chunk = total;                                 // single-stage top-k (no candidate scratch)
   } else {
     const long long ld = scores_ld_for(max_entries);
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
       return fail(DSV4_ERR_WORKSPACE, "dsv4_index_topk: workspace missing or not 256-byte aligned");
-    const long long rows = (long long)workspace_bytes / (ld * 4);
+    const long long cand = candidate_bytes_per_row(max_entries, k);
+    long long rows = (long long)workspace_bytes / (ld * 4 + cand);
+    if (rows > total) rows = total;
+    while (rows > 1 && workspace_bytes_for(rows, ld, cand) > (long long)workspace_bytes) --rows;
+    if (rows >= 1 && cand > 0 && workspace_bytes_for(rows, ld, cand) <= (long long)workspace_bytes) {
+      a.nseg = topk_segments(max_entries);
+      a.cand_score = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(rows * ld * 4, 256));
+      a.cand_idx = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(a.cand_score) + rows * a.nseg * k * 4);
+    } else {                                       // no room for candidates: single stage
+      rows = (long long)workspace_bytes / (ld * 4);
+      if (rows > total) rows = total;
+    }
     if (rows < 1)
       return fail(DSV4_ERR_WORKSPACE, "dsv4_index_topk: workspace %zu bytes < one score row (%lld)",
                   workspace_bytes, ld * 4);
     a.scores = reinterpret_cast<float*>(workspace); a.scores_ld = ld;
-    chunk = (int)(rows < total ? rows : total);
+    chunk = (int)rows;
   }
   for (int q0 = 0; q0 < total; q0 += chunk) {
     const int qn = total - q0 < chunk ? total - q0 : chunk;
@@ -164,12 +190,32 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
 
 // ----------------------------------------------------------------------------- attention
 
+// Split partials pay off only when (query, 64-head group) items are fewer than the SMs.
+static int attn_sm_count() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+  }
+  return sms;
+}
+
+extern "C" size_t dsv4_hybrid_sparse_attn_workspace_size(int B, int nq, int H, int c) {
+  if (B <= 0 || nq <= 0 || H < 64 || H % 64 != 0 || c <= 0) return 0;
+  const long long items = (long long)B * nq * (H / 64);
+  if (items >= attn_sm_count()) return 0;
+  return (size_t)round_up(items * ATTN_MAX_SPLIT * attn_split_bytes_per_item(c), 256);
+}
+
 extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* pool,
                                        int64_t pool_rows, const int64_t* kv_row_off,
                                        const int32_t* idx, const int32_t* counts, int k,
                                        const void* local, int R, const int32_t* q_pos0, int B,
                                        int nq, int H, int c, int m, int w, const float* sink,
-                                       float scale, void* O, float* lse, void* stream) {
+                                       float scale, void* O, float* lse, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
   if (dtype != DSV4_F32 && dtype != DSV4_BF16)
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_hybrid_sparse_attn: dtype %d", dtype);
   if (B < 0 || nq < 0 || H < 1 || c < 1 || m < 1 || w < 1 || R < 1 || pool_rows < 0 ||
@@ -187,6 +233,20 @@ extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* poo
   a.counts = counts; a.k = idx ? k : 0; a.local = local; a.R = R; a.q_pos0 = q_pos0; a.B = B;
   a.nq = nq; a.H = H; a.c = c; a.m = m; a.w = w; a.sink = sink; a.scale = scale; a.O = O;
   a.lse = lse;
+  a.nsplit = 1;
+  a.part_o = nullptr;
+  a.part_ml = nullptr;
+  if (workspace && workspace_bytes > 0 && H % 64 == 0) {
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+      return fail(DSV4_ERR_WORKSPACE, "dsv4_hybrid_sparse_attn: workspace not 256-byte aligned");
+    const long long items = (long long)B * nq * (H / 64);
+    long long cap = (long long)workspace_bytes / (items * attn_split_bytes_per_item(c));
+    if (cap > ATTN_MAX_SPLIT) cap = ATTN_MAX_SPLIT;
+    if (cap > 1) {
+      a.nsplit = (int)cap;                           // capacity; the launcher picks the count
+      a.part_o = reinterpret_cast<float*>(workspace);
+    }
+  }
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == DSV4_BF16) {
     bool used = false;

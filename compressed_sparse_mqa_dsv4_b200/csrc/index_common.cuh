@@ -21,6 +21,10 @@ struct IndexArgs {
   float* scores;       // score rows of queries [score_q0, score_q0 + rows)
   long long scores_ld;
   int score_q0;        // global query id of score row 0
+  // two-stage top-k of long rows: nseg candidate blocks of k per score row (nseg = 1: off)
+  int nseg;
+  float* cand_score;
+  int32_t* cand_idx;
 };
 
 // Completed entries of query (b, i), clamped to the score-row capacity (flagged).
@@ -65,5 +69,7 @@ int launch_index_scores_simt(const IndexArgs& a, int q_begin, int q_count, int m
 int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max_e,
                            cudaStream_t st, bool* used);
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
+// Segments of the two-stage top-k for rows of up to max_entries entries (1: single stage).
+int topk_segments(int max_entries);
 
 }  // namespace dsv4

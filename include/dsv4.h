@@ -186,6 +186,12 @@ int dsv4_index_topk_noalloc(int qdtype, const void* qI, const uint8_t* qI_scales
  *   w          local window, >= 1 (so every candidate list is non-empty).
  *   sink       fp32 [H] or NULL.  scale: logit scale (1/sqrt(c) in the model).
  *   O          [B, nq, H, c] (dtype) output.  lse: fp32 [B, nq, H] output or NULL.
+ *   workspace  device scratch (256-byte aligned) of workspace_bytes, or NULL / 0. When the
+ *              request has fewer (query, 64-head group) items than the device has SMs
+ *              (decode), the tensor-core path splits each candidate list into up to 8
+ *              parts that run on separate SMs and are merged afterwards (exact up to fp32
+ *              rounding order); the parts live here. Without workspace nothing is split.
+ *              dsv4_hybrid_sparse_attn_workspace_size gives the size that allows all splits.
  *   Requires c % 8 == 0 for bf16 (c % 4 for fp32), R >= min(w, q_pos0+nq).
  *   Device-checked: every used idx value in [0, floor((t+1)/m_csa)) when `m` > 0, and
  *   every pool row < pool_rows; out-of-range candidates are skipped and flagged.
@@ -195,7 +201,11 @@ int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* pool, int64_t 
                             const int32_t* counts, int k, const void* local, int R,
                             const int32_t* q_pos0, int B, int nq, int H, int c, int m, int w,
                             const float* sink, float scale, void* O, float* lse,
-                            void* stream);
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes for dsv4_hybrid_sparse_attn to split every candidate list of a request of
+ * B x nq queries with H heads of dimension c (0 when no split would be used). */
+size_t dsv4_hybrid_sparse_attn_workspace_size(int B, int nq, int H, int c);
 
 #ifdef __cplusplus
 }

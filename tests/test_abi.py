@@ -54,7 +54,7 @@ def test_host_validation_rejects_bad_arguments(lib):
     assert lib.dsv4_quantize_fp4(P(16), P(16), P(16), ctypes.c_int64(4), 24, None) == 1
     # attention: w < 1 rejected
     args = [1, P(16), P(16), ctypes.c_int64(4), P(16), None, None, 0, P(16), 8, P(16), 1, 1, 64,
-            512, 4, 0, None, ctypes.c_float(1.0), P(16), None, None]
+            512, 4, 0, None, ctypes.c_float(1.0), P(16), None, None, ctypes.c_size_t(0), None]
     assert lib.dsv4_hybrid_sparse_attn(*args) == 1
     # index top-k: k above the supported maximum
     lib.dsv4_index_topk.restype = ctypes.c_int

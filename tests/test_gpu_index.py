@@ -113,6 +113,21 @@ def test_index_long_rows_radix_path(dsv4):
     _run_and_check(dsv4, qI, w, KI, [0], pos0, 4, 1000, [(0, 0), (0, 1)], what="radix ties")
 
 
+def test_index_decode_long_contexts(dsv4):
+    """Decode over long contexts: one query per sequence, rows of 17.5k-75k entries (the
+    workspace path selects per 16384-entry segment first, then among the candidates)."""
+    shape = preset("flash_csa_prefill", B=3)
+    lens = [300001, 131075, 70003]
+    rows = [L // 4 for L in lens]
+    offs = list(np.concatenate([[0], np.cumsum(rows)[:-1]]).astype(np.int64))
+    g = Generator(21)
+    qI, w = g.index_queries(shape, 1)
+    KI = g.index_keys(shape, int(sum(rows)) + 1)
+    pos0 = [L - 1 for L in lens]
+    _run_and_check(dsv4, qI, w, KI, offs, pos0, 4, 512, [(b, 0) for b in range(3)],
+                   what="decode long")
+
+
 def test_index_flash_full_sampled(dsv4, index_path):
     """V4-Flash shape: n=8192, H_I=64, c_I=128, k=512; every query run, a sample compared."""
     shape = preset("flash_csa_prefill")
