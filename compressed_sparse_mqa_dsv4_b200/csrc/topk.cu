@@ -71,7 +71,9 @@ struct TopkShared {
 
 // Selects the keff (< n) largest of sc[0, n) under (score descending, position ascending) and
 // calls emit(p, j) for the p-th selected position j, p ascending with j. All NT threads call.
-template <int NT, typename Emit>
+// kShort: rows of at most a few thousand entries -- scalar loads and plain shared atomics
+// for the histograms and per-thread contiguous ranges for the compaction cost less there.
+template <int NT, bool kShort, typename Emit>
 __device__ __forceinline__ void select_topk(const float* sc, int n, int keff, TopkShared& sh,
                                             Emit emit) {
   int* hist = sh.hist;
@@ -87,22 +89,38 @@ __device__ __forceinline__ void select_topk(const float* sc, int n, int keff, To
     __syncthreads();
     // whole warps iterate together (match/ballot need converged lanes); four keys per lane
     // per step from one 16-byte load when the row is aligned
-    for (int j0 = 4 * (threadIdx.x & ~31); j0 < Et; j0 += 4 * NT) {
-      const int j = j0 + 4 * (threadIdx.x & 31);
-      float4 f = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (vec && j + 3 < Et) {
-        f = __ldg(reinterpret_cast<const float4*>(sc + j));
-      } else {
-        if (j < Et) f.x = __ldg(sc + j);
-        if (j + 1 < Et) f.y = __ldg(sc + j + 1);
-        if (j + 2 < Et) f.z = __ldg(sc + j + 2);
-        if (j + 3 < Et) f.w = __ldg(sc + j + 3);
+    if (kShort) {
+      for (int j = threadIdx.x; j < Et; j += NT) {
+        const uint32_t key = score_key(__ldg(sc + j));
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
       }
-      const float fv[4] = {f.x, f.y, f.z, f.w};
+    }
+    // (UNR independent loads in flight per thread: the scan is latency bound otherwise)
+    constexpr int UNR = 4;
+    for (int j0 = 4 * (threadIdx.x & ~31); !kShort && j0 < Et; j0 += 4 * NT * UNR) {
+      float4 f[UNR];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t key = score_key(fv[u]);
-        hist_add(hist, (key >> shift) & 255u, j + u < Et && (key & pmask) == prefix);
+      for (int r = 0; r < UNR; ++r) {
+        const int j = j0 + 4 * NT * r + 4 * (threadIdx.x & 31);
+        f[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (vec && j + 3 < Et) {
+          f[r] = __ldg(reinterpret_cast<const float4*>(sc + j));
+        } else {
+          if (j < Et) f[r].x = __ldg(sc + j);
+          if (j + 1 < Et) f[r].y = __ldg(sc + j + 1);
+          if (j + 2 < Et) f[r].z = __ldg(sc + j + 2);
+          if (j + 3 < Et) f[r].w = __ldg(sc + j + 3);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < UNR; ++r) {
+        const int j = j0 + 4 * NT * r + 4 * (threadIdx.x & 31);
+        const float fv[4] = {f[r].x, f[r].y, f[r].z, f[r].w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t key = score_key(fv[u]);
+          hist_add(hist, (key >> shift) & 255u, j + u < Et && (key & pmask) == prefix);
+        }
       }
     }
     __syncthreads();
@@ -125,6 +143,29 @@ __device__ __forceinline__ void select_topk(const float* sc, int n, int keff, To
   const uint32_t T = prefix;
   const int need_eq = remaining;                  // keys equal to T to take (lowest index first)
 
+  if (kShort) {
+    // ---- order-preserving compaction over contiguous per-thread ranges
+    const int per = (Et + NT - 1) / NT;
+    const int lo = threadIdx.x * per, hi = min(Et, lo + per);
+    int n_gt = 0, n_eq = 0;
+    for (int j = lo; j < hi; ++j) {
+      const uint32_t key = score_key(__ldg(sc + j));
+      n_gt += key > T;
+      n_eq += key == T;
+    }
+    int tot;
+    const int eq_before = block_exclusive_scan<NT>(n_eq, warp_tot, tot);
+    const int take_eq = max(0, min(n_eq, need_eq - eq_before));
+    int pos = block_exclusive_scan<NT>(n_gt + take_eq, warp_tot, tot), eq_seen = 0;
+    for (int j = lo; j < hi; ++j) {
+      const uint32_t key = score_key(__ldg(sc + j));
+      if (key > T || (key == T && eq_seen++ < take_eq)) {
+        if (pos < keff) emit(pos, j);
+        ++pos;
+      }
+    }
+    return;
+  }
   // ---- order-preserving compaction: each warp owns a contiguous range of entries, read
   // 32 at a time (coalesced); ballots give in-warp ranks, block scans give warp offsets.
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -132,11 +173,20 @@ __device__ __forceinline__ void select_topk(const float* sc, int n, int keff, To
   const int per_w = ((Et + NT / 32 - 1) / (NT / 32) + 31) & ~31;
   const int lo = wid * per_w, hi = min(Et, lo + per_w);
   int n_gt = 0, n_eq = 0;
-  for (int j0 = lo; j0 < hi; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < hi ? score_key(__ldg(sc + j)) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, j < hi && key > T));
-    n_eq += __popc(__ballot_sync(0xffffffffu, j < hi && key == T));
+  for (int j0 = lo; j0 < hi; j0 += 128) {
+    float v[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = j0 + 32 * r + lane;
+      v[r] = j < hi ? __ldg(sc + j) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = j0 + 32 * r + lane;
+      const uint32_t key = score_key(v[r]);
+      n_gt += __popc(__ballot_sync(0xffffffffu, j < hi && key > T));
+      n_eq += __popc(__ballot_sync(0xffffffffu, j < hi && key == T));
+    }
   }
   // warp totals are uniform across the warp: lane 0 contributes them to the block scans
   int tot;
@@ -145,17 +195,26 @@ __device__ __forceinline__ void select_topk(const float* sc, int n, int keff, To
   const int take_eq = max(0, min(n_eq, need_eq - eq_b));
   const int pos_b = block_exclusive_scan<NT>(lane == 0 ? n_gt + take_eq : 0, warp_tot, tot);
   int pos = __shfl_sync(0xffffffffu, pos_b, 0), eq_seen = 0;
-  for (int j0 = lo; j0 < hi; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < hi ? score_key(__ldg(sc + j)) : 0u;
-    const bool gt = j < hi && key > T, eq = j < hi && key == T;
-    const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-    const bool sel = gt || (eq && eq_seen + __popc(eqb & lt) < take_eq);
-    const uint32_t selb = __ballot_sync(0xffffffffu, sel);
-    const int p = pos + __popc(selb & lt);
-    if (sel && p < keff) emit(p, j);
-    pos += __popc(selb);
-    eq_seen += __popc(eqb);
+  for (int j0 = lo; j0 < hi; j0 += 128) {
+    float v[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = j0 + 32 * r + lane;
+      v[r] = j < hi ? __ldg(sc + j) : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = j0 + 32 * r + lane;
+      const uint32_t key = score_key(v[r]);
+      const bool gt = j < hi && key > T, eq = j < hi && key == T;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+      const bool sel = gt || (eq && eq_seen + __popc(eqb & lt) < take_eq);
+      const uint32_t selb = __ballot_sync(0xffffffffu, sel);
+      const int p = pos + __popc(selb & lt);
+      if (sel && p < keff) emit(p, j);
+      pos += __popc(selb);
+      eq_seen += __popc(eqb);
+    }
   }
 }
 
@@ -177,7 +236,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(IndexArgs a, int q_begin) {
     return;
   }
   const float* sc = a.scores + (long long)(qg - a.score_q0) * a.scores_ld;
-  select_topk<NT>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; });
+  select_topk<NT, NT == 256>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; });
 }
 
 // Stage 1 of the long-row path: grid (segment, query). Writes the segment's top
@@ -208,7 +267,7 @@ __global__ void __launch_bounds__(NT) topk_seg_kernel(IndexArgs a, int q_begin) 
     }
     return;
   }
-  select_topk<NT>(sc, len, kseg, sh, [&](int p, int j) {
+  select_topk<NT, false>(sc, len, kseg, sh, [&](int p, int j) {
     cs[p] = sc[j];
     ci[p] = lo + j;
   });
@@ -234,14 +293,14 @@ __global__ void __launch_bounds__(NT) topk_merge_kernel(IndexArgs a, int q_begin
   const long long row = qg - a.score_q0;
   const float* cs = a.cand_score + row * a.nseg * k;
   const int32_t* ci = a.cand_idx + row * a.nseg * k;
-  select_topk<NT>(cs, a.nseg * k, keff, sh, [&](int p, int j) { out[p] = ci[j]; });
+  select_topk<NT, false>(cs, a.nseg * k, keff, sh, [&](int p, int j) { out[p] = ci[j]; });
 }
 
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
   if (q_count <= 0) return DSV4_OK;
   if (a.nseg > 1) {
     topk_seg_kernel<256><<<dim3(a.nseg, q_count), 256, 0, st>>>(a, q_begin);
-    if ((long long)a.nseg * a.k > 4 * TOPK_SEG)
+    if ((long long)a.nseg * a.k >= 4096)
       topk_merge_kernel<1024><<<q_count, 1024, 0, st>>>(a, q_begin);
     else
       topk_merge_kernel<256><<<q_count, 256, 0, st>>>(a, q_begin);
