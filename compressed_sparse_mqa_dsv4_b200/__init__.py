@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "DSV4Error", "lib", "LIB_PATH", "F32", "BF16", "FP4",
     "dsv4_compress", "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
+    "dsv4_index_topk_workspace_size_ex",
     "dsv4_hybrid_sparse_attn", "dsv4_hybrid_sparse_attn_workspace_size", "dsv4_check_errors",
 ]
 
@@ -45,6 +46,8 @@ lib.dsv4_quantize_fp4.restype = _I
 lib.dsv4_quantize_fp4.argtypes = [_P, _P, _P, _L, _I, _P]
 lib.dsv4_index_topk_workspace_size.restype = _S
 lib.dsv4_index_topk_workspace_size.argtypes = [_I, _I, _I, _I]
+lib.dsv4_index_topk_workspace_size_ex.restype = _S
+lib.dsv4_index_topk_workspace_size_ex.argtypes = [_I, _I, _I, _I, _I, _I, _I, _L]
 lib.dsv4_index_topk.restype = _I
 lib.dsv4_index_topk.argtypes = [_I, _P, _P, _P, _P, _P, _L, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                 _P, _P, _P, _L, _P, _S, _P]
@@ -129,6 +132,12 @@ def dsv4_index_topk_workspace_size(B: int, nq: int, max_entries: int, k: int) ->
     return int(lib.dsv4_index_topk_workspace_size(B, nq, max_entries, k))
 
 
+def dsv4_index_topk_workspace_size_ex(qdtype: int, B: int, nq: int, H_I: int, c_I: int,
+                                      max_entries: int, k: int, ki_rows: int) -> int:
+    return int(lib.dsv4_index_topk_workspace_size_ex(qdtype, B, nq, H_I, c_I, max_entries, k,
+                                                     ki_rows))
+
+
 def dsv4_index_topk(qI: torch.Tensor, w: torch.Tensor, KI: torch.Tensor,
                     kv_row_off: torch.Tensor, q_pos0: torch.Tensor, m: int, k: int,
                     max_entries: int, qI_scales: Optional[torch.Tensor] = None,
@@ -156,21 +165,23 @@ def dsv4_index_topk(qI: torch.Tensor, w: torch.Tensor, KI: torch.Tensor,
         idx = torch.empty(B, nq, k, dtype=torch.int32, device=qI.device)
     if counts is None:
         counts = torch.empty(B, nq, dtype=torch.int32, device=qI.device)
-    ws_bytes = 0
     scores_ld = 0
     if scores_out is not None:
         _dev(scores_out, "scores_out", torch.float32)
         scores_ld = scores_out.shape[-1]
-    else:
-        ws_bytes = dsv4_index_topk_workspace_size(B, nq, max_entries, k)
-        if workspace is None or workspace.numel() < ws_bytes:
-            workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=qI.device)
-        ws_bytes = workspace.numel()
+    ws_bytes = dsv4_index_topk_workspace_size_ex(qd, B, nq, H_I, c_I, max_entries, k, ki_rows)
+    if scores_out is not None and fp4:
+        # room for the bf16 expansion of K^I and of every query's q^I (one chunk)
+        ws_bytes = ki_rows * c_I * 2 + B * nq * H_I * c_I * 2 + 1024
+    elif scores_out is not None:
+        ws_bytes = 0
+    if ws_bytes and (workspace is None or workspace.numel() < ws_bytes):
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=qI.device)
+    ws_bytes = workspace.numel() if workspace is not None else 0
     _check(lib.dsv4_index_topk(qd, _ptr(qI), _ptr(qI_scales), _ptr(w), _ptr(KI), _ptr(KI_scales),
                                ki_rows, _ptr(kv_row_off), _ptr(q_pos0), B, nq, H_I, c_I, m, k,
                                max_entries, _ptr(idx), _ptr(counts), _ptr(scores_out), scores_ld,
-                               _ptr(workspace) if scores_out is None else None, ws_bytes,
-                               _stream(stream)), "dsv4_index_topk")
+                               _ptr(workspace), ws_bytes, _stream(stream)), "dsv4_index_topk")
     return idx, counts
 
 

@@ -91,20 +91,50 @@ static long long candidate_bytes_per_row(int max_entries, int k) {
   return nseg > 1 ? (long long)nseg * k * 8 : 0;
 }
 
-// Rows of the workspace layout [scores: rows x ld fp32][candidate scores][candidate indices]
-static long long workspace_bytes_for(long long rows, long long ld, long long cand_per_row) {
-  return round_up(rows * ld * 4, 256) + round_up(rows * cand_per_row, 256);
+// Workspace layout for a chunk of `rows` queries:
+//   [bf16 expansion of K^I (FP4 tensor-core path)]
+//   [scores: rows x ld fp32 (absent when the caller supplies score rows)]
+//   [candidate scores and indices of the two-stage top-k]
+//   [bf16 expansion of the chunk's q^I rows (FP4 tensor-core path)]
+struct IxLayout {
+  long long scores, cand, qx, total;
+};
+static IxLayout ix_layout(long long rows, long long ld, long long cand_per_row, long long kx_bytes,
+                          long long qx_per_row, bool with_scores) {
+  IxLayout L;
+  long long off = round_up(kx_bytes, 256);
+  L.scores = off;
+  off += with_scores ? round_up(rows * ld * 4, 256) : 0;
+  L.cand = off;
+  off += round_up(rows * cand_per_row, 256);
+  L.qx = off;
+  off += round_up(rows * qx_per_row, 256);
+  L.total = off;
+  return L;
+}
+
+static bool fp4_tensor_path(int qdtype, int H_I, int c_I) {
+  const char* force = std::getenv("DSV4_FORCE_SIMT");
+  return qdtype == DSV4_FP4 && H_I == 64 && c_I == 128 && !(force && force[0] == '1');
+}
+
+extern "C" size_t dsv4_index_topk_workspace_size_ex(int qdtype, int B, int nq, int H_I, int c_I,
+                                                    int max_entries, int k, int64_t ki_rows) {
+  if (B <= 0 || nq <= 0 || max_entries <= 0) return 0;
+  const bool fp4 = fp4_tensor_path(qdtype, H_I, c_I);
+  const long long ld = scores_ld_for(max_entries);
+  const long long cand = candidate_bytes_per_row(max_entries, k > 0 ? k : 0);
+  const long long qx = fp4 ? (long long)H_I * c_I * 2 : 0;
+  const long long kx = fp4 ? (ki_rows > 0 ? ki_rows : 0) * c_I * 2 : 0;
+  const long long total = (long long)B * nq;
+  long long rows = kScoreChunkBytes / (ld * 4 + cand + qx);
+  if (rows < 1) rows = 1;
+  if (rows > total) rows = total;
+  return (size_t)ix_layout(rows, ld, cand, kx, qx, true).total;
 }
 
 extern "C" size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k) {
-  if (B <= 0 || nq <= 0 || max_entries <= 0) return 0;
-  const long long ld = scores_ld_for(max_entries);
-  const long long cand = candidate_bytes_per_row(max_entries, k > 0 ? k : 0);
-  const long long total = (long long)B * nq;
-  long long rows = kScoreChunkBytes / (ld * 4 + cand);
-  if (rows < 1) rows = 1;
-  if (rows > total) rows = total;
-  return (size_t)workspace_bytes_for(rows, ld, cand);
+  return dsv4_index_topk_workspace_size_ex(DSV4_BF16, B, nq, 64, 128, max_entries, k, 0);
 }
 
 extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_scales,
@@ -141,43 +171,97 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   a.nseg = 1;
   a.cand_score = nullptr;
   a.cand_idx = nullptr;
+  a.q_map_q0 = 0;
+  a.q_map_rows = 0;
   cudaStream_t st = (cudaStream_t)stream;
   const int total = B * nq;
-  int chunk;
+  const bool ws_ok = workspace && !(reinterpret_cast<uintptr_t>(workspace) & 255u);
+  if (!scores_out && !ws_ok)
+    return fail(DSV4_ERR_WORKSPACE, "dsv4_index_topk: workspace missing or not 256-byte aligned");
+  if (scores_out && scores_ld < max_entries)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_index_topk: scores_ld %lld < max_entries %d",
+                (long long)scores_ld, max_entries);
+  // FP4 operands take the tensor-core kernel through an exact bf16 expansion in the workspace
+  // (K^I once, q^I per chunk) when the workspace has room for it; else the CUDA-core kernel.
+  const long long ld = scores_ld_for(max_entries);
+  const long long cand = candidate_bytes_per_row(max_entries, k);
+  const long long wsb = ws_ok ? (long long)workspace_bytes : 0;
+  bool fp4x = ws_ok && fp4_tensor_path(qdtype, H_I, c_I) && ki_rows > 0 &&
+              !(reinterpret_cast<uintptr_t>(KI) & 7u) && !(reinterpret_cast<uintptr_t>(qI) & 7u);
+  const long long kx = fp4x ? ki_rows * c_I * 2 : 0;
+  const long long qx = fp4x ? (long long)H_I * c_I * 2 : 0;
+  long long rows;
   if (scores_out) {
-    if (scores_ld < max_entries)
-      return fail(DSV4_ERR_INVALID_ARG, "dsv4_index_topk: scores_ld %lld < max_entries %d",
-                  (long long)scores_ld, max_entries);
-    a.scores = scores_out; a.scores_ld = scores_ld > 0 ? scores_ld : 1;
-    chunk = total;                                 // single-stage top-k (no candidate scratch)
+    rows = total;                                  // one chunk; single-stage top-k
+    if (fp4x && ix_layout(rows, ld, 0, kx, qx, false).total > wsb) fp4x = false;
   } else {
-    const long long ld = scores_ld_for(max_entries);
-    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
-      return fail(DSV4_ERR_WORKSPACE, "dsv4_index_topk: workspace missing or not 256-byte aligned");
-    const long long cand = candidate_bytes_per_row(max_entries, k);
-    long long rows = (long long)workspace_bytes / (ld * 4 + cand);
-    if (rows > total) rows = total;
-    while (rows > 1 && workspace_bytes_for(rows, ld, cand) > (long long)workspace_bytes) --rows;
-    if (rows >= 1 && cand > 0 && workspace_bytes_for(rows, ld, cand) <= (long long)workspace_bytes) {
-      a.nseg = topk_segments(max_entries);
-      a.cand_score = reinterpret_cast<float*>(static_cast<char*>(workspace) + round_up(rows * ld * 4, 256));
-      a.cand_idx = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(a.cand_score) + rows * a.nseg * k * 4);
-    } else {                                       // no room for candidates: single stage
-      rows = (long long)workspace_bytes / (ld * 4);
-      if (rows > total) rows = total;
-    }
+    // largest chunk that fits, preferring the two-stage top-k, then the FP4 expansion
+    auto fit = [&](long long c_row, long long kx_b, long long qx_row) {
+      const long long per = ld * 4 + c_row + qx_row;
+      long long r = (wsb - round_up(kx_b, 256)) / per;
+      if (r > total) r = total;
+      while (r > 1 && ix_layout(r, ld, c_row, kx_b, qx_row, true).total > wsb) --r;
+      return (r >= 1 && ix_layout(r, ld, c_row, kx_b, qx_row, true).total <= wsb) ? r : 0ll;
+    };
+    long long c_use = cand;
+    rows = fit(c_use, kx, qx);
+    if (rows < 1 && cand > 0) { c_use = 0; rows = fit(c_use, kx, qx); }
+    if (rows < 1 && fp4x) { fp4x = false; c_use = cand; rows = fit(c_use, 0, 0); }
+    if (rows < 1 && cand > 0) { c_use = 0; rows = fit(c_use, 0, 0); }
     if (rows < 1)
       return fail(DSV4_ERR_WORKSPACE, "dsv4_index_topk: workspace %zu bytes < one score row (%lld)",
                   workspace_bytes, ld * 4);
-    a.scores = reinterpret_cast<float*>(workspace); a.scores_ld = ld;
-    chunk = (int)rows;
+    const IxLayout L = ix_layout(rows, ld, c_use, fp4x ? kx : 0, fp4x ? qx : 0, true);
+    char* base = static_cast<char*>(workspace);
+    a.scores = reinterpret_cast<float*>(base + L.scores);
+    a.scores_ld = ld;
+    if (c_use > 0) {
+      a.nseg = topk_segments(max_entries);
+      a.cand_score = reinterpret_cast<float*>(base + L.cand);
+      a.cand_idx = reinterpret_cast<int32_t*>(base + L.cand + rows * a.nseg * k * 4);
+    }
   }
+  if (scores_out) {
+    a.scores = scores_out;
+    a.scores_ld = scores_ld > 0 ? scores_ld : 1;
+  }
+  IndexArgs ax = a;                                // the bf16 view of FP4 operands
+  if (fp4x) {
+    const IxLayout L = ix_layout(rows, ld, scores_out ? 0 : (a.nseg > 1 ? cand : 0), kx, qx,
+                                 !scores_out);
+    char* base = static_cast<char*>(workspace);
+    __nv_bfloat16* kbuf = reinterpret_cast<__nv_bfloat16*>(base);
+    int s = launch_fp4_expand(static_cast<const uint8_t*>(KI), KI_scales, ki_rows, c_I, kbuf, st);
+    if (s != DSV4_OK) return s;
+    ax.qdtype = DSV4_BF16;
+    ax.KI = kbuf;
+    ax.KI_scales = nullptr;
+    ax.qI = base + L.qx;
+    ax.qI_scales = nullptr;
+  }
+  const int chunk = (int)rows;
   for (int q0 = 0; q0 < total; q0 += chunk) {
     const int qn = total - q0 < chunk ? total - q0 : chunk;
     a.score_q0 = scores_out ? 0 : q0;
+    ax.score_q0 = a.score_q0;
     bool used = false;
-    int s = launch_index_scores_tc(a, q0, qn, max_entries, st, &used);
+    int s = DSV4_OK;
+    if (fp4x) {
+      const long long qrow0 = (long long)q0 * H_I;
+      s = launch_fp4_expand(static_cast<const uint8_t*>(qI) + qrow0 * (c_I / 2),
+                            qI_scales + qrow0 * (c_I / 16), (long long)qn * H_I, c_I,
+                            static_cast<__nv_bfloat16*>(const_cast<void*>(ax.qI)), st);
+      if (s != DSV4_OK) return s;
+      ax.q_map_q0 = q0;
+      ax.q_map_rows = (long long)qn * H_I;
+      s = launch_index_scores_tc(ax, q0, qn, max_entries, st, &used);
+    } else {
+      s = launch_index_scores_tc(a, q0, qn, max_entries, st, &used);
+    }
     if (s != DSV4_OK) return s;
+    if (q0 == 0)
+      trace_path(used ? (fp4x ? "index scores: tcgen05 (FP4 expanded to bf16)" : "index scores: tcgen05")
+                      : "index scores: CUDA cores");
     if (!used) {
       s = launch_index_scores_simt(a, q0, qn, max_entries, st);
       if (s != DSV4_OK) return s;

@@ -21,6 +21,10 @@ struct IndexArgs {
   float* scores;       // score rows of queries [score_q0, score_q0 + rows)
   long long scores_ld;
   int score_q0;        // global query id of score row 0
+  // Q rows the tensor-core kernel reads start at query q_map_q0 and number q_map_rows
+  // (0: the whole request; the FP4 path reads a per-chunk bf16 expansion)
+  int q_map_q0;
+  long long q_map_rows;
   // two-stage top-k of long rows: nseg candidate blocks of k per score row (nseg = 1: off)
   int nseg;
   float* cand_score;
@@ -71,5 +75,8 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
 // Segments of the two-stage top-k for rows of up to max_entries entries (1: single stage).
 int topk_segments(int max_entries);
+// FP4 codes [rows, cols/2] + E4M3 scales [rows, cols/16] -> bf16 [rows, cols] (exact).
+int launch_fp4_expand(const uint8_t* codes, const uint8_t* scales, long long rows, int cols,
+                      __nv_bfloat16* out, cudaStream_t st);
 
 }  // namespace dsv4

@@ -107,7 +107,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       tc::prefetch_tensormap(&map_q);
       tc::prefetch_tensormap(&map_k);
       tc::mbar_arrive_expect_tx(&s.q_full, 2 * IX_QT * IX_HI * 128);
-      const int qrow = qlo * IX_HI;
+      const int qrow = (qlo - a.q_map_q0) * IX_HI;
       tc::tma_load_2d(s.q[0], &map_q, &s.q_full, 0, qrow);
       tc::tma_load_2d(s.q[1], &map_q, &s.q_full, 64, qrow);
       for (int blk = 0; blk < nblk; ++blk) {
@@ -225,7 +225,7 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
     *used = true;
     return DSV4_OK;
   }
-  const long long q_rows = (long long)a.B * a.nq * IX_HI;
+  const long long q_rows = a.q_map_rows > 0 ? a.q_map_rows : (long long)a.B * a.nq * IX_HI;
   if (q_rows >= (1ll << 31) || a.ki_rows >= (1ll << 31) || a.ki_rows <= 0) return DSV4_OK;
   CUtensorMap mq, mk;
   int s = encode_tensor_map_2d(&mq, a.qI, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, IX_CI, q_rows, 64,

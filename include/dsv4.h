@@ -100,10 +100,18 @@ int dsv4_compress(int dtype, const void* C, const void* Z, const float* bias, vo
 int dsv4_quantize_fp4(const void* x, uint8_t* codes, uint8_t* scales, int64_t rows, int cols,
                       void* stream);
 
-/* Bytes of workspace dsv4_index_topk needs for this request (0 when scores_out is
- * given, which then serves as the score buffer). max_entries = the largest number of
- * completed entries any query of the request can see. */
+/* Bytes of workspace dsv4_index_topk needs for a bf16 / fp32 request: per chunk of queries
+ * the fp32 score rows and, for rows longer than 16384 entries, the candidates of the
+ * two-stage top-k (a smaller workspace makes smaller chunks; a larger one is not used).
+ * max_entries = the largest number of completed entries any query of the request can see. */
 size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k);
+
+/* The same for any operand type. FP4 operands at H_I = 64, c_I = 128 are scored on the
+ * tensor cores after an exact expansion to bf16 in the workspace (K^I: ki_rows x c_I, the
+ * chunk's q^I rows); this size includes that room. With less room (or with scores_out and a
+ * workspace too small for the expansion of every query) FP4 is scored on CUDA cores. */
+size_t dsv4_index_topk_workspace_size_ex(int qdtype, int B, int nq, int H_I, int c_I,
+                                         int max_entries, int k, int64_t ki_rows);
 
 /*
  * dsv4_index_topk -- lightning-indexer score and per-query TopK, [CSA-DEF] s3.1:

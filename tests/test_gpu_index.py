@@ -136,8 +136,9 @@ def test_index_flash_full_sampled(dsv4, index_path):
     _run_and_check(dsv4, qI, w, KI, [0], [0], 4, 512, pos, what="flash")
 
 
-def test_index_fp4(dsv4):
-    """FP4 operands (e2m1 + E4M3 per 16): the oracle scores the same dequantised values."""
+def test_index_fp4(dsv4, index_path):
+    """FP4 operands (e2m1 + E4M3 per 16): the oracle scores the same dequantised values. The
+    tensor-core path scores an exact bf16 expansion; the CUDA-core path decodes per element."""
     shape = preset("pro_csa_prefill", n=4 * 700 + 1)
     n, E = shape.n, shape.n // 4
     qI, w, KI = _inputs(shape, n, E, 2)
@@ -149,7 +150,7 @@ def test_index_fp4(dsv4):
     pos = [(0, t) for t in sample_positions(n, 4, extra=[1023, 1024, 2799])]
     _run_and_check(dsv4, qc_t, w, torch.from_numpy(kc), [0], [0], 4, 256, pos,
                    qI_sc=torch.from_numpy(qs), KI_sc=torch.from_numpy(ks), qI64=qI64,
-                   KI64=KI64, c_I=128, what="fp4")
+                   KI64=KI64, c_I=128, what=f"fp4 {index_path}")
 
 
 def test_index_k_zero_and_short(dsv4):
