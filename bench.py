@@ -64,6 +64,14 @@ def attention_flops(n: int, m: int, k: int, w: int, H: int, c: int) -> float:
     return 4.0 * H * c * tot
 
 
+def hca_attention_flops(n: int, m: int, w: int, H: int, c: int) -> float:
+    """Dense read: 4*H*c*sum_t (floor((t+1)/m) + min(w, t+1))."""
+    tot = 0
+    for t in range(n):
+        tot += (t + 1) // m + min(w, t + 1)
+    return 4.0 * H * c * tot
+
+
 def index_flops(n: int, m: int, HI: int, cI: int) -> float:
     return 2.0 * HI * cI * sum((t + 1) // m for t in range(n))
 
@@ -283,6 +291,9 @@ def run_cuda(args, rank: int, world: int):
     }
     if not args.no_decode:
         res["decode"] = run_decode(args, dev, stream)
+    if args.layers:
+        res["other_layers"] = {nm: run_layer(args, dev, stream, nm)
+                               for nm in ("flash_hca_prefill", "pro_csa_prefill")}
     return res
 
 
@@ -376,6 +387,96 @@ def run_decode(args, dev, stream):
             "steps": steps, "l2": "flushed (256 MiB write) before every step"}
 
 
+# ----------------------------------------------------------------------------- other layers
+
+
+def run_layer(args, dev, stream, name):
+    """One full prefill layer of another configuration, inputs drawn on the device:
+    flash_hca_prefill (B=2, n=65536, HCA m'=128 dense read + window) or pro_csa_prefill
+    (n=131072, H=128, k=1024, indexer operands quantised to FP4 inside the step)."""
+    import torch
+    import compressed_sparse_mqa_dsv4_b200 as dsv4
+    from workloads import Generator, preset
+    s = preset(name)
+    g = Generator(args.seed + 3, device=dev.type)
+    E = s.n // s.m
+    C, Z, bias = g.compressor_inputs(s, "main")
+    Q = g.queries(s)
+    local = g.local_kv(s)
+    sink = g.sink(s)
+    off = torch.arange(s.B, dtype=torch.int64, device=dev) * E
+    pos0 = torch.zeros(s.B, dtype=torch.int32, device=dev)
+    pool = torch.empty(s.B, E, s.c, dtype=torch.bfloat16, device=dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty(s.B, s.n, s.H, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    extra = {}
+    if s.kind == "csa":
+        CI, ZI, biasI = g.compressor_inputs(s, "index")
+        qI, w = g.index_queries(s)
+        KI = torch.empty(s.B, E, s.c_I, dtype=torch.bfloat16, device=dev)
+        qc = torch.empty(s.B * s.n * s.H_I, s.c_I // 2, dtype=torch.uint8, device=dev)
+        qs = torch.empty(s.B * s.n * s.H_I, s.c_I // 16, dtype=torch.uint8, device=dev)
+        kc = torch.empty(s.B * E, s.c_I // 2, dtype=torch.uint8, device=dev)
+        ks = torch.empty(s.B * E, s.c_I // 16, dtype=torch.uint8, device=dev)
+        idx = torch.empty(s.B, s.n, s.k, dtype=torch.int32, device=dev)
+        cnt = torch.empty(s.B, s.n, dtype=torch.int32, device=dev)
+        ws = torch.empty(dsv4.dsv4_index_topk_workspace_size_ex(dsv4.FP4, s.B, s.n, s.H_I, s.c_I, E, s.k,
+                                                                s.B * E), dtype=torch.uint8, device=dev)
+
+    def step(rec):
+        rec[0].record(stream)
+        dsv4.dsv4_compress(C, Z, bias, s.m, s.kind == "csa", out=pool)
+        if s.kind == "csa":
+            dsv4.dsv4_compress(CI, ZI, biasI, s.m, True, out=KI)
+            dsv4.dsv4_quantize_fp4(qI.view(-1, s.c_I), qc, qs)
+            dsv4.dsv4_quantize_fp4(KI.view(-1, s.c_I), kc, ks)
+            rec[1].record(stream)
+            dsv4.dsv4_index_topk(qc.view(s.B, s.n, s.H_I, s.c_I // 2), w, kc, off, pos0, s.m, s.k, E,
+                                 qI_scales=qs, KI_scales=ks, c_I=s.c_I, idx=idx, counts=cnt,
+                                 workspace=ws)
+            rec[2].record(stream)
+            dsv4.dsv4_hybrid_sparse_attn(Q, pool.view(-1, s.c), off, idx, cnt, local, pos0, s.m, s.w,
+                                         sink, O=O, lse=lse)
+        else:
+            rec[1].record(stream)
+            rec[2].record(stream)
+            dsv4.dsv4_hybrid_sparse_attn(Q, pool.view(-1, s.c), off, None, None, local, pos0, s.m, s.w,
+                                         sink, O=O, lse=lse)
+        rec[3].record(stream)
+
+    for _ in range(2):
+        flush.zero_()
+        step([torch.cuda.Event(enable_timing=True) for _ in range(4)])
+    dsv4.dsv4_check_errors()
+    steps = 3
+    recs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        step(recs[i])
+    torch.cuda.synchronize()
+    dsv4.dsv4_check_errors()
+    ms = statistics.median([r[0].elapsed_time(r[3]) for r in recs])
+    t_pre = statistics.median([r[0].elapsed_time(r[1]) for r in recs])
+    t_idx = statistics.median([r[1].elapsed_time(r[2]) for r in recs])
+    t_att = statistics.median([r[2].elapsed_time(r[3]) for r in recs])
+    peaks, src = _peaks()
+    peak = float(peaks["bf16_tflops"])
+    attn_fl = s.B * attention_flops(s.n, s.m, s.k if s.kind == "csa" else 0, s.w, s.H, s.c) \
+        if s.kind == "csa" else s.B * hca_attention_flops(s.n, s.m, s.w, s.H, s.c)
+    rec = {"workload": f"{name}: B={s.B}, n={s.n}, H={s.H}, c={s.c}, m={s.m}, w={s.w}"
+                       + (f", k={s.k}, H_I={s.H_I}, c_I={s.c_I}, FP4 indexer" if s.kind == "csa" else ", dense"),
+           "tokens_per_s": round(s.B * s.n / (ms / 1e3), 1), "ms_per_step": round(ms, 3),
+           "breakdown_ms": {"compress_quantize": round(t_pre, 3), "index_topk": round(t_idx, 3),
+                            "attention": round(t_att, 3)},
+           "attention_tflops": round(attn_fl / (t_att / 1e3) / 1e12, 1),
+           "attention_frac": round(attn_fl / (t_att / 1e3) / 1e12 / peak, 4), "steps": steps}
+    if s.kind == "csa":
+        ifl = s.B * index_flops(s.n, s.m, s.H_I, s.c_I)
+        rec["index_tflops"] = round(ifl / (t_idx / 1e3) / 1e12, 1)
+    return rec
+
+
 # ----------------------------------------------------------------------------- oracle arm
 
 
@@ -464,6 +565,8 @@ def main():
     ap.add_argument("--oracle-queries", type=int, default=2048)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the batched-decode measurement")
+    ap.add_argument("--layers", action="store_true",
+                    help="also time the HCA-prefill and V4-Pro (FP4 indexer) layers at full size")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
