@@ -8,7 +8,7 @@
 // entry's dot products with every head of every query in the tile, and the weighted
 // ReLU head sum is a per-thread reduction in registers:
 //     D[128 entries x 64*nqt] = K^I_blk[128 x c_I] . qI_tile[64*nqt x c_I]^T
-// One CTA per (tile of <= 4 queries of one sequence, chunk of <= 4096 entries), 10 warps:
+// One CTA per (tile of <= 4 queries of one sequence, chunk of 4096-16384 entries), 10 warps:
 //   warps 0-7  epilogue: warp w reads TMEM lane quadrant w%4 for queries 2(w/4), 2(w/4)+1
 //   warp 8     producer: the query tile once, then 128-entry key blocks by 2D TMA into a
 //              4-stage ring
@@ -27,7 +27,7 @@ constexpr int IX_HI = 64;              // indexer heads per query
 constexpr int IX_QT = 4;               // queries per tile
 constexpr int IX_BLK = 128;            // entries per MMA tile
 constexpr int IX_STAGES = 4;
-constexpr int IX_CHUNK = 4096;         // entries per CTA (grid.y splits longer rows)
+constexpr int IX_CHUNK = 4096;         // smallest entry chunk per CTA (grid.y splits rows)
 constexpr int IX_THREADS = 320;
 constexpr uint32_t IX_TM_COLS = 512;
 
@@ -47,7 +47,7 @@ constexpr size_t IX_SMEM = sizeof(IndexSmem) + 1024;
 __global__ void __launch_bounds__(IX_THREADS, 1)
     index_tc_kernel(const IndexArgs a, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k, int q_begin, int q_count,
-                    int tile0, int tiles_per_seq, uint32_t spin) {
+                    int tile0, int tiles_per_seq, int chunk, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
   IndexSmem& s = *reinterpret_cast<IndexSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -62,8 +62,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   const int nqt = qhi - qlo;                       // queries in the tile (may be 0)
   int e_tile = 0;                                  // entries seen by the tile's last query
   if (nqt > 0) e_tile = visible_entries(a, b, qhi - 1 - b * a.nq);
-  const int e0 = blockIdx.y * IX_CHUNK;
-  const int e1 = min(e_tile, e0 + IX_CHUNK);
+  const int e0 = blockIdx.y * chunk;
+  const int e1 = min(e_tile, e0 + chunk);
   const long long base = nqt > 0 ? a.kv_row_off[b] : 0;
   const bool bounds_ok = base >= 0 && base + e_tile <= a.ki_rows;
   if (nqt <= 0 || e1 <= e0 || !bounds_ok) {
@@ -237,12 +237,17 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
   const int tps = (a.nq + IX_QT - 1) / IX_QT;
   auto tile_of = [&](int qg) { return (qg / a.nq) * tps + (qg % a.nq) / IX_QT; };
   const int t0 = tile_of(q_begin), t1 = tile_of(q_begin + q_count - 1);
-  dim3 grid(t1 - t0 + 1, (max_e + IX_CHUNK - 1) / IX_CHUNK);
+  // Long rows with few query tiles (decode): larger entry chunks per CTA amortise its setup
+  // (Q tile, TMEM, pipeline fill) while keeping at least 4 CTAs per SM of work.
+  int chunk = IX_CHUNK;
+  const long long tiles = t1 - t0 + 1;
+  while (chunk < 4 * IX_CHUNK && tiles * ((max_e + 2 * chunk - 1) / (2 * chunk)) >= 4 * 148) chunk *= 2;
+  dim3 grid((unsigned)tiles, (max_e + chunk - 1) / chunk);
   if (grid.y > 65535) return DSV4_OK;
   cudaError_t e = cudaFuncSetAttribute(index_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)IX_SMEM);
   if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "index_tc: %s", cudaGetErrorString(e));
-  index_tc_kernel<<<grid, IX_THREADS, IX_SMEM, st>>>(a, mq, mk, q_begin, q_count, t0, tps,
+  index_tc_kernel<<<grid, IX_THREADS, IX_SMEM, st>>>(a, mq, mk, q_begin, q_count, t0, tps, chunk,
                                                     spin_limit());
   *used = true;
   return launch_status("index scores (tensor cores)");
