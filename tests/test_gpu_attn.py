@@ -73,12 +73,15 @@ def test_attn_tiny_fp32_sink(dsv4):
     _case(dsv4, B=2, nq=100, H=4, c=64, m=4, w=16, k=8, dtype="f32", sink=True, what="sink")
 
 
-@pytest.fixture(params=["tc_cluster", "tc_single_cta", "cuda_cores"])
+@pytest.fixture(params=["tc_cluster", "tc_single_cta", "tc_double_buffer", "cuda_cores"])
 def attn_path(request, monkeypatch):
     """Run a case on each attention kernel: the 2-CTA-cluster tcgen05 kernel, the single-CTA
-    tcgen05 kernel (both bf16, c=512, H%64==0) and the CUDA-core kernel."""
+    tcgen05 kernel with 128-slot blocks, the double-buffered one with 64-slot blocks (all
+    bf16, c=512, H%64==0) and the CUDA-core kernel. Split lists (decode) always take the
+    128-slot kernel."""
     monkeypatch.setenv("DSV4_FORCE_SIMT", "1" if request.param == "cuda_cores" else "0")
     monkeypatch.setenv("DSV4_ATTN_CLUSTER", "1" if request.param == "tc_cluster" else "0")
+    monkeypatch.setenv("DSV4_ATTN_DB", "1" if request.param == "tc_double_buffer" else "0")
     return request.param
 
 
