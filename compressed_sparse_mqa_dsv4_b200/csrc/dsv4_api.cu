@@ -84,17 +84,16 @@ static long long scores_ld_for(int max_entries) { return round_up(max_entries > 
 
 static const long long kScoreChunkBytes = 256ll << 20;
 
-// Workspace bytes per query row: its fp32 scores and, for long rows, the candidate blocks
-// of the two-stage top-k (k scores + k entry indices per segment).
+// Workspace bytes per query row: its fp32 scores and, for long rows, the region of the
+// threshold top-k.
 static long long candidate_bytes_per_row(int max_entries, int k) {
-  const int nseg = topk_segments(max_entries);
-  return nseg > 1 ? (long long)nseg * k * 8 : 0;
+  return topk_row_bytes(max_entries, k);
 }
 
 // Workspace layout for a chunk of `rows` queries:
 //   [bf16 expansion of K^I (FP4 tensor-core path)]
 //   [scores: rows x ld fp32 (absent when the caller supplies score rows)]
-//   [candidate scores and indices of the two-stage top-k]
+//   [threshold top-k regions of long rows (histograms, counters, selected, candidates)]
 //   [bf16 expansion of the chunk's q^I rows (FP4 tensor-core path)]
 struct IxLayout {
   long long scores, cand, qx, total;
@@ -169,8 +168,9 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   a.idx = idx;
   a.counts = counts;
   a.nseg = 1;
-  a.cand_score = nullptr;
-  a.cand_idx = nullptr;
+  a.cand = nullptr;
+  a.cand_row_bytes = 0;
+  a.hist1_done = 0;
   a.q_map_q0 = 0;
   a.q_map_rows = 0;
   cudaStream_t st = (cudaStream_t)stream;
@@ -195,7 +195,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     rows = total;                                  // one chunk; single-stage top-k
     if (fp4x && ix_layout(rows, ld, 0, kx, qx, false).total > wsb) fp4x = false;
   } else {
-    // largest chunk that fits, preferring the two-stage top-k, then the FP4 expansion
+    // largest chunk that fits, preferring the threshold top-k, then the FP4 expansion
     auto fit = [&](long long c_row, long long kx_b, long long qx_row) {
       const long long per = ld * 4 + c_row + qx_row;
       long long r = (wsb - round_up(kx_b, 256)) / per;
@@ -216,9 +216,9 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     a.scores = reinterpret_cast<float*>(base + L.scores);
     a.scores_ld = ld;
     if (c_use > 0) {
-      a.nseg = topk_segments(max_entries);
-      a.cand_score = reinterpret_cast<float*>(base + L.cand);
-      a.cand_idx = reinterpret_cast<int32_t*>(base + L.cand + rows * a.nseg * k * 4);
+      a.nseg = 2;
+      a.cand = base + L.cand;
+      a.cand_row_bytes = c_use;
     }
   }
   if (scores_out) {
@@ -245,7 +245,8 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     a.score_q0 = scores_out ? 0 : q0;
     ax.score_q0 = a.score_q0;
     bool used = false;
-    int s = DSV4_OK;
+    int s = topk_prepare(a, q0, qn, st);
+    if (s != DSV4_OK) return s;
     if (fp4x) {
       const long long qrow0 = (long long)q0 * H_I;
       s = launch_fp4_expand(static_cast<const uint8_t*>(qI) + qrow0 * (c_I / 2),
@@ -266,6 +267,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
       s = launch_index_scores_simt(a, q0, qn, max_entries, st);
       if (s != DSV4_OK) return s;
     }
+    a.hist1_done = used ? 1 : 0;                  // the tensor-core kernel built hist1
     s = launch_topk(a, q0, qn, st);
     if (s != DSV4_OK) return s;
   }

@@ -25,11 +25,29 @@ struct IndexArgs {
   // (0: the whole request; the FP4 path reads a per-chunk bf16 expansion)
   int q_map_q0;
   long long q_map_rows;
-  // two-stage top-k of long rows: nseg candidate blocks of k per score row (nseg = 1: off)
+  // threshold top-k of long rows (nseg > 1): one region of cand_row_bytes per score row
+  // (int hist1[256] of key bits 31..24 at its start, then hist2, counters, the entries above
+  // the threshold, the boundary candidates); hist1_done: the score kernel built hist1
   int nseg;
-  float* cand_score;
-  int32_t* cand_idx;
+  char* cand;
+  long long cand_row_bytes;
+  int hist1_done;
 };
+
+// Order-preserving 32-bit key of a score (larger score -> larger key; -0 folded into +0).
+__device__ __forceinline__ uint32_t score_key(float s) {
+  s = s + 0.0f;                                  // fold -0 into +0
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// One histogram update per distinct bin among the warp's active lanes.
+__device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool pred) {
+  const uint32_t active = __ballot_sync(0xffffffffu, pred);
+  if (!pred) return;
+  const uint32_t same = __match_any_sync(active, bin);
+  if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
+}
 
 // Completed entries of query (b, i), clamped to the score-row capacity (flagged).
 __device__ __forceinline__ int visible_entries(const IndexArgs& a, int b, int i) {
@@ -73,8 +91,12 @@ int launch_index_scores_simt(const IndexArgs& a, int q_begin, int q_count, int m
 int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max_e,
                            cudaStream_t st, bool* used);
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
-// Segments of the two-stage top-k for rows of up to max_entries entries (1: single stage).
-int topk_segments(int max_entries);
+// Zeroes the threshold top-k headers of the score rows of queries [q_begin, q_begin +
+// q_count) (before the score kernel, which may build the first histogram).
+int topk_prepare(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
+// Workspace bytes per score row of the threshold top-k for rows of up to max_entries
+// entries and k winners (0: such rows take the single-stage select).
+long long topk_row_bytes(int max_entries, int k);
 // FP4 codes [rows, cols/2] + E4M3 scales [rows, cols/16] -> bf16 [rows, cols] (exact).
 int launch_fp4_expand(const uint8_t* codes, const uint8_t* scales, long long rows, int cols,
                       __nv_bfloat16* out, cudaStream_t st);

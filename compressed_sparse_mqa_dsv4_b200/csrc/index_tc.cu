@@ -38,6 +38,7 @@ struct IndexSmem {
   uint8_t q[2][QT * IX_HI * 128];           // K-major SW128: [QT*64 rows][64 ch] per K half
   uint8_t k[NST][2][IX_BLK * 128];          // [128 entries][64 ch] per K half
   float w[QT][IX_HI];
+  int hist[QT][256];                        // key bits 31..24 of the tile's scores (long rows)
   uint64_t q_full;
   uint64_t k_full[NST], k_empty[NST];
   uint64_t d_full[2], d_empty[2];
@@ -110,6 +111,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     s.abort = 0;
     tc::fence_barrier_init();
   }
+  for (int e = tid; e < QT * 256; e += blockDim.x) s.hist[e >> 8][e & 255] = 0;
   for (int e = tid; e < QT * IX_HI; e += blockDim.x) {
     const int u = e / IX_HI, h = e % IX_HI;
     s.w[u][h] = u < nqt ? a.w[(long long)(qlo + u) * a.H_I + h] : 0.f;
@@ -242,6 +244,10 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[32 + h], fmaxf(d3[h], 0.f), sc1);
       }
       if (sidx < Et[0]) a.scores[srow[0] + sidx] = sc0;
+      if (a.nseg > 1) {                          // first histogram of the threshold top-k
+        hist_add(s.hist[QT > 1 ? 2 * qp : 0], score_key(sc0) >> 24, sidx < Et[0]);
+        if (QT > 1) hist_add(s.hist[QT > 1 ? 2 * qp + 1 : 0], score_key(sc1) >> 24, 2 * qp + 1 < nqt && sidx < Et[1]);
+      }
       if (tid == 0) IX_TRACE(6, blk);
       if (QT > 1 && 2 * qp + 1 < nqt && sidx < Et[1]) a.scores[srow[1] + sidx] = sc1;
     }
@@ -251,6 +257,14 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   if (warp == 9) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, IX_TM_COLS);
+  }
+  if (a.nseg > 1) {
+    // add the tile's histograms to the rows' first histograms (int hist1[256] at the start
+    // of each row's top-k region)
+    for (int e = tid; e < nqt * 256; e += blockDim.x) {
+      const int u = e >> 8, v = s.hist[u][e & 255];
+      if (v) atomicAdd(reinterpret_cast<int*>(a.cand + (long long)(qlo + u - a.score_q0) * a.cand_row_bytes) + (e & 255), v);
+    }
   }
 }
 

@@ -12,24 +12,15 @@
 //   exclusive scans give every warp its output offset and its share of the ties, and the
 //   selected positions are emitted in ascending order.
 // Rows up to TOPK_SEG entries: one CTA per query (E_t <= k selects everything without
-// reading a score). Longer rows (decode over long contexts): stage 1 selects, per segment
-// of TOPK_SEG entries, that segment's top k under the same order (score descending, then
-// entry ascending) -- every entry of the query's top k is in its segment's top k, since the
-// entries ranked above it within the segment are a subset of those ranked above it overall;
-// stage 2 selects the query's top k among the concatenated segment candidates, which are
-// already in ascending entry order.
+// reading a score). Longer rows (decode over long contexts) take a threshold pipeline whose
+// passes stream the row across many CTAs (see "threshold pipeline" below).
 #include "dsv4_common.cuh"
 #include "index_common.cuh"
 
 namespace dsv4 {
 
-constexpr int TOPK_SEG = 16384;                  // longer rows take the two-stage path
+constexpr int TOPK_SEG = 16384;                  // longer rows take the threshold pipeline
 
-__device__ __forceinline__ uint32_t score_key(float s) {
-  s = s + 0.0f;                                  // fold -0 into +0
-  const uint32_t u = __float_as_uint(s);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
 
 // Block-wide exclusive prefix sum over the NT threads; also returns the total.
 template <int NT>
@@ -55,13 +46,6 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
   return before + incl - v;
 }
 
-// One histogram update per distinct bin among the warp's active lanes.
-__device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool pred) {
-  const uint32_t active = __ballot_sync(0xffffffffu, pred);
-  if (!pred) return;
-  const uint32_t same = __match_any_sync(active, bin);
-  if ((threadIdx.x & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], __popc(same));
-}
 
 struct TopkShared {
   int hist[256];
@@ -239,44 +223,185 @@ __global__ void __launch_bounds__(NT) topk_kernel(IndexArgs a, int q_begin) {
   select_topk<NT, NT == 256>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; });
 }
 
-// Stage 1 of the long-row path: grid (segment, query). Writes the segment's top
-// min(k, segment length) entries (global entry index and score) in ascending entry order to
-// its k candidate slots and pads the rest with score -inf / index -1.
+// ---------------------------------------------------------------- threshold pipeline
+// Rows longer than TOPK_SEG entries (decode over long contexts). Each pass is spread over
+// CTAs of TK_PASS entries and streams the row once:
+//   hist1  per-row histogram of key bits 31..24;
+//   hist2  the bin B1 holding the k_eff-th largest key -> histogram of bits 23..16 of the
+//          keys in B1;
+//   filter the bin B2 holding the k_eff-th largest key among those -> keys whose top 16 bits
+//          exceed (B1, B2) are selected; keys equal to it in their top 16 bits are boundary
+//          candidates, kept as (low 16 key bits, ~entry) so that a larger value means a larger
+//          score or, for equal scores, a lower entry;
+//   final  per row: the k_eff - (selected) largest boundary candidates by a radix select over
+//          those 48-bit values (all distinct), then the selected entries in ascending order.
+// A row whose boundary candidates exceed TK_CAND is selected by the single-CTA select over
+// the whole row instead (many scores sharing their top 16 bits).
+constexpr int TK_PASS = 8192;                    // entries per CTA of a pass
+constexpr int TK_CAND = 8192;                    // boundary candidates kept per row
+constexpr int TK_MAXK = 4096;                    // larger k: single-CTA select
+constexpr int TK_HDR = 4096;                     // row header: hist1, hist2, counters
+
+struct TkRow {
+  int* hist1;                                    // [256]
+  int* hist2;                                    // [256]
+  int* counters;                                 // n_sel, n_cand
+  int32_t* sel;                                  // [k]
+  unsigned long long* cand;                      // [TK_CAND]
+};
+
+__device__ __forceinline__ TkRow tk_row(const IndexArgs& a, long long row) {
+  char* base = a.cand + row * a.cand_row_bytes;
+  TkRow r;
+  r.hist1 = reinterpret_cast<int*>(base);
+  r.hist2 = reinterpret_cast<int*>(base + 1024);
+  r.counters = reinterpret_cast<int*>(base + 2048);
+  r.sel = reinterpret_cast<int32_t*>(base + TK_HDR);
+  r.cand = reinterpret_cast<unsigned long long*>(base + TK_HDR + (((long long)a.k * 4 + 255) & ~255ll));
+  return r;
+}
+
+// The bin (by thread: thread t owns bin 255 - t) where the count from the top first reaches
+// `need`; returns the bin and the count strictly above it through shared memory.
 template <int NT>
-__global__ void __launch_bounds__(NT) topk_seg_kernel(IndexArgs a, int q_begin) {
-  __shared__ TopkShared sh;
-  const int qg = q_begin + blockIdx.y, seg = blockIdx.x;
-  const int b = qg / a.nq, i = qg % a.nq;
-  const int Et = visible_entries(a, b, i);
-  const int k = a.k;
-  const long long row = qg - a.score_q0;
-  float* cs = a.cand_score + (row * a.nseg + seg) * k;
-  int32_t* ci = a.cand_idx + (row * a.nseg + seg) * k;
-  const int lo = seg * TOPK_SEG;
-  const int len = max(0, min(Et, lo + TOPK_SEG) - lo);
-  const int kseg = min(k, len);
-  const float* sc = a.scores + row * a.scores_ld + lo;
-  for (int j = kseg + threadIdx.x; j < k; j += blockDim.x) {
-    cs[j] = -INFINITY;
-    ci[j] = -1;
+__device__ __forceinline__ void tk_find_bin(const int* hist_g, int need, TopkShared& sh) {
+  if (threadIdx.x == 0) {                         // (not found: an inconsistent row, which the
+    sh.sel = -1;                                  // final stage sends to the whole-row select)
+    sh.above = 0;
   }
-  if (kseg == len) {                              // the whole segment is a candidate set
-    for (int j = threadIdx.x; j < len; j += blockDim.x) {
-      cs[j] = sc[j];
-      ci[j] = lo + j;
+  const int d = 255 - (int)threadIdx.x;
+  const int h = d >= 0 ? __ldcg(hist_g + d) : 0;
+  int tot;
+  const int above = block_exclusive_scan<NT>(h, sh.warp_tot, tot);
+  if (d >= 0 && above < need && need <= above + h) {
+    sh.sel = d;
+    sh.above = above;
+  }
+  __syncthreads();
+}
+
+// One pass over entries [lo, hi) of a score row: 32 keys per thread, loaded as float4s
+// (8 in flight per thread). f(j, key, valid) is called by whole warps.
+template <int NT, typename F>
+__device__ __forceinline__ void tk_scan(const float* sc, int lo, int hi, F f) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int j0 = lo + 128 * wid; j0 < hi; j0 += 128 * (NT / 32) * 8) {
+    float4 v[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int j = j0 + 128 * (NT / 32) * r + 4 * lane;
+      v[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j + 3 < hi) {
+        v[r] = __ldcg(reinterpret_cast<const float4*>(sc + j));
+      } else {
+        if (j < hi) v[r].x = __ldcg(sc + j);
+        if (j + 1 < hi) v[r].y = __ldcg(sc + j + 1);
+        if (j + 2 < hi) v[r].z = __ldcg(sc + j + 2);
+      }
     }
-    return;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int j = j0 + 128 * (NT / 32) * r + 4 * lane;
+      const float fv[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f(j + u, score_key(fv[u]), j + u < hi);
+    }
   }
-  select_topk<NT, false>(sc, len, kseg, sh, [&](int p, int j) {
-    cs[p] = sc[j];
-    ci[p] = lo + j;
+}
+
+// Warp-aggregated append of one value per flagged lane to list[*counter ...]; returns the
+// position of this lane's value (or -1).
+__device__ __forceinline__ int tk_append(int* counter, bool pred) {
+  const uint32_t m = __ballot_sync(0xffffffffu, pred);
+  if (m == 0) return -1;
+  const int lane = threadIdx.x & 31;
+  int base = 0;
+  if (lane == __ffs(m) - 1) base = atomicAdd(counter, __popc(m));
+  base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
+  return pred ? base + __popc(m & ((1u << lane) - 1u)) : -1;
+}
+
+struct TkCta {
+  int qg, Et, keff, lo, hi;
+  long long row;
+  bool active;
+};
+
+__device__ __forceinline__ TkCta tk_cta(const IndexArgs& a, int q_begin) {
+  TkCta c;
+  c.qg = q_begin + blockIdx.y;
+  const int b = c.qg / a.nq, i = c.qg % a.nq;
+  c.Et = visible_entries(a, b, i);
+  c.keff = min(a.k, c.Et);
+  c.row = c.qg - a.score_q0;
+  c.lo = blockIdx.x * TK_PASS;
+  c.hi = min(c.Et, c.lo + TK_PASS);
+  c.active = c.Et > a.k && c.lo < c.hi;          // shorter rows: the final kernel selects all
+  return c;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_hist1_kernel(IndexArgs a, int q_begin) {
+  __shared__ TopkShared sh;
+  const TkCta c = tk_cta(a, q_begin);
+  if (!c.active) return;
+  const TkRow r = tk_row(a, c.row);
+  if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+  __syncthreads();
+  tk_scan<NT>(a.scores + c.row * a.scores_ld, c.lo, c.hi,
+              [&](int, uint32_t key, bool valid) { hist_add(sh.hist, key >> 24, valid); });
+  __syncthreads();
+  if (threadIdx.x < 256 && sh.hist[threadIdx.x]) atomicAdd(r.hist1 + threadIdx.x, sh.hist[threadIdx.x]);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_hist2_kernel(IndexArgs a, int q_begin) {
+  __shared__ TopkShared sh;
+  const TkCta c = tk_cta(a, q_begin);
+  if (!c.active) return;
+  const TkRow r = tk_row(a, c.row);
+  tk_find_bin<NT>(r.hist1, c.keff, sh);
+  const uint32_t b1 = (uint32_t)sh.sel;
+  if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+  __syncthreads();
+  // few keys fall in bin B1 and they spread over the second byte: plain shared atomics
+  tk_scan<NT>(a.scores + c.row * a.scores_ld, c.lo, c.hi, [&](int, uint32_t key, bool valid) {
+    if (valid && (key >> 24) == b1) atomicAdd(&sh.hist[(key >> 16) & 255u], 1);
+  });
+  __syncthreads();
+  if (threadIdx.x < 256 && sh.hist[threadIdx.x]) atomicAdd(r.hist2 + threadIdx.x, sh.hist[threadIdx.x]);
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_filter_kernel(IndexArgs a, int q_begin) {
+  __shared__ TopkShared sh;
+  const TkCta c = tk_cta(a, q_begin);
+  if (!c.active) return;
+  const TkRow r = tk_row(a, c.row);
+  tk_find_bin<NT>(r.hist1, c.keff, sh);
+  const uint32_t b1 = (uint32_t)sh.sel;
+  const int above1 = sh.above;
+  __syncthreads();
+  tk_find_bin<NT>(r.hist2, c.keff - above1, sh);
+  const uint32_t t16 = (b1 << 8) | (uint32_t)sh.sel;
+  tk_scan<NT>(a.scores + c.row * a.scores_ld, c.lo, c.hi, [&](int j, uint32_t key, bool valid) {
+    const uint32_t top = key >> 16;
+    const int ps = tk_append(r.counters, valid && top > t16);
+    if (ps >= 0 && ps < a.k) r.sel[ps] = j;
+    const int pc = tk_append(r.counters + 1, valid && top == t16);
+    if (pc >= 0 && pc < TK_CAND)
+      r.cand[pc] = ((unsigned long long)(key & 0xFFFFu) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
   });
 }
 
-// Stage 2 of the long-row path: one CTA per query over its nseg * k candidates.
+// Final stage: one CTA per row. Dynamic shared memory: TK_CAND candidates + TK_MAXK outputs.
 template <int NT>
-__global__ void __launch_bounds__(NT) topk_merge_kernel(IndexArgs a, int q_begin) {
+__global__ void __launch_bounds__(NT) topk_final_kernel(IndexArgs a, int q_begin) {
   __shared__ TopkShared sh;
+  __shared__ int n_out;
+  extern __shared__ unsigned long long tk_smem[];
+  unsigned long long* cv = tk_smem;                         // [TK_CAND]
+  int* outl = reinterpret_cast<int*>(tk_smem + TK_CAND);    // [TK_MAXK]
   const int qg = q_begin + blockIdx.x;
   const int b = qg / a.nq, i = qg % a.nq;
   const int Et = visible_entries(a, b, i);
@@ -286,25 +411,102 @@ __global__ void __launch_bounds__(NT) topk_merge_kernel(IndexArgs a, int q_begin
   if (threadIdx.x == 0) a.counts[qg] = keff;
   for (int j = keff + threadIdx.x; j < k; j += blockDim.x) out[j] = -1;
   if (keff == 0) return;
-  if (Et <= k) {
+  if (Et <= k) {                                  // every visible entry is selected
     for (int j = threadIdx.x; j < Et; j += blockDim.x) out[j] = j;
     return;
   }
   const long long row = qg - a.score_q0;
-  const float* cs = a.cand_score + row * a.nseg * k;
-  const int32_t* ci = a.cand_idx + row * a.nseg * k;
-  select_topk<NT, false>(cs, a.nseg * k, keff, sh, [&](int p, int j) { out[p] = ci[j]; });
+  const TkRow r = tk_row(a, row);
+  const int n_sel = __ldcg(r.counters), n_cand = __ldcg(r.counters + 1);
+  const int need = keff - n_sel;
+  if (n_cand > TK_CAND || need < 0 || need > n_cand) {
+    // too many scores share the threshold's top 16 bits: select over the whole row
+    const float* sc = a.scores + row * a.scores_ld;
+    select_topk<NT, false>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; });
+    return;
+  }
+  for (int e = threadIdx.x; e < n_cand; e += NT) cv[e] = __ldcg(r.cand + e);
+  for (int e = threadIdx.x; e < n_sel; e += NT) outl[e] = __ldcg(r.sel + e);
+  if (threadIdx.x == 0) n_out = n_sel;
+  __syncthreads();
+  if (need > 0) {
+    // radix select of the need-th largest 48-bit candidate value, 8 bits per pass
+    unsigned long long prefix = 0, pmask = 0;
+    int remaining = need;
+    for (int pass = 0; pass < 6; ++pass) {
+      const int shift = 40 - 8 * pass;
+      if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+      __syncthreads();
+      for (int e = threadIdx.x; e < n_cand; e += NT) {
+        const unsigned long long v = cv[e];
+        if ((v & pmask) == prefix) atomicAdd(&sh.hist[(v >> shift) & 255u], 1);
+      }
+      __syncthreads();
+      const int d = 255 - (int)threadIdx.x;
+      const int h = d >= 0 ? sh.hist[d] : 0;
+      int tot;
+      const int above = block_exclusive_scan<NT>(h, sh.warp_tot, tot);
+      if (d >= 0 && above < remaining && remaining <= above + h) {
+        sh.sel = d;
+        sh.above = above;
+      }
+      __syncthreads();
+      remaining -= sh.above;
+      prefix |= (unsigned long long)sh.sel << shift;
+      pmask |= 255ull << shift;
+      __syncthreads();
+    }
+    // candidate values are distinct: exactly `need` of them are >= the threshold
+    for (int e = threadIdx.x; e < n_cand; e += NT) {
+      const unsigned long long v = cv[e];
+      if (v >= prefix) {
+        const int p = atomicAdd(&n_out, 1);
+        if (p < TK_MAXK) outl[p] = (int)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
+      }
+    }
+    __syncthreads();
+  }
+  // ascending entry order: bitonic sort of the keff selected entries (padded to a power of 2)
+  int n2 = 1;
+  while (n2 < keff) n2 <<= 1;
+  for (int e = keff + threadIdx.x; e < n2; e += NT) outl[e] = 0x7FFFFFFF;
+  __syncthreads();
+  for (int size = 2; size <= n2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int e = threadIdx.x; e < n2 / 2; e += NT) {
+        const int lo = 2 * e - (e & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const int x = outl[lo], y = outl[hi];
+        if ((x > y) == up) {
+          outl[lo] = y;
+          outl[hi] = x;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int e = threadIdx.x; e < keff; e += NT) out[e] = outl[e];
 }
 
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
   if (q_count <= 0) return DSV4_OK;
   if (a.nseg > 1) {
-    topk_seg_kernel<256><<<dim3(a.nseg, q_count), 256, 0, st>>>(a, q_begin);
-    if ((long long)a.nseg * a.k >= 4096)
-      topk_merge_kernel<1024><<<q_count, 1024, 0, st>>>(a, q_begin);
-    else
-      topk_merge_kernel<256><<<q_count, 256, 0, st>>>(a, q_begin);
-  } else if (a.max_e > TOPK_SEG) {                // long rows without candidate scratch
+    constexpr int kFinalSmem = TK_CAND * 8 + TK_MAXK * 4;
+    static bool attr_set = false;
+    if (!attr_set) {
+      const cudaError_t e = cudaFuncSetAttribute(topk_final_kernel<1024>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kFinalSmem);
+      if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "top-k: %s", cudaGetErrorString(e));
+      attr_set = true;
+    }
+    // (headers zeroed by topk_prepare; the score kernel may have built hist1 already)
+    const dim3 grid((a.max_e + TK_PASS - 1) / TK_PASS, q_count);
+    if (!a.hist1_done) topk_hist1_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
+    topk_hist2_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
+    topk_filter_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
+    topk_final_kernel<1024><<<q_count, 1024, kFinalSmem, st>>>(a, q_begin);
+  } else if (a.max_e > TOPK_SEG) {                // long rows without the pipeline's scratch
     topk_kernel<1024><<<q_count, 1024, 0, st>>>(a, q_begin);
   } else {
     topk_kernel<256><<<q_count, 256, 0, st>>>(a, q_begin);
@@ -312,8 +514,17 @@ int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
   return launch_status("top-k select");
 }
 
-int topk_segments(int max_entries) {
-  return max_entries > TOPK_SEG ? (max_entries + TOPK_SEG - 1) / TOPK_SEG : 1;
+int topk_prepare(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
+  if (a.nseg <= 1 || q_count <= 0) return DSV4_OK;
+  const long long row0 = q_begin - a.score_q0;
+  const cudaError_t e = cudaMemset2DAsync(a.cand + row0 * a.cand_row_bytes, (size_t)a.cand_row_bytes, 0,
+                                          (size_t)TK_HDR, (size_t)q_count, st);
+  return e == cudaSuccess ? DSV4_OK : fail(DSV4_ERR_CUDA, "top-k: %s", cudaGetErrorString(e));
+}
+
+long long topk_row_bytes(int max_entries, int k) {
+  if (max_entries <= TOPK_SEG || k <= 0 || k > TK_MAXK) return 0;
+  return TK_HDR + (((long long)k * 4 + 255) & ~255ll) + (long long)TK_CAND * 8;
 }
 
 }  // namespace dsv4

@@ -101,8 +101,10 @@ int dsv4_quantize_fp4(const void* x, uint8_t* codes, uint8_t* scales, int64_t ro
                       void* stream);
 
 /* Bytes of workspace dsv4_index_topk needs for a bf16 / fp32 request: per chunk of queries
- * the fp32 score rows and, for rows longer than 16384 entries, the candidates of the
- * two-stage top-k (a smaller workspace makes smaller chunks; a larger one is not used).
+ * the fp32 score rows and, for rows longer than 16384 entries (and k <= 4096), the region of
+ * the threshold top-k (histograms, the entries above the threshold and up to 8192 boundary
+ * candidates: 4 KiB + 4k bytes + 64 KiB per row). A smaller workspace makes smaller chunks;
+ * a larger one is not used.
  * max_entries = the largest number of completed entries any query of the request can see. */
 size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k);
 

@@ -115,7 +115,8 @@ def test_index_long_rows_radix_path(dsv4):
 
 def test_index_decode_long_contexts(dsv4):
     """Decode over long contexts: one query per sequence, rows of 17.5k-75k entries (the
-    workspace path selects per 16384-entry segment first, then among the candidates)."""
+    workspace path: histograms of the top 16 key bits, a filter pass, then a select among
+    the boundary candidates)."""
     shape = preset("flash_csa_prefill", B=3)
     lens = [300001, 131075, 70003]
     rows = [L // 4 for L in lens]
