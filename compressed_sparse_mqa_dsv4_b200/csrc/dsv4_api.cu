@@ -86,8 +86,8 @@ static const long long kScoreChunkBytes = 256ll << 20;
 
 // Workspace bytes per query row: its fp32 scores and, for long rows, the region of the
 // threshold top-k.
-static long long candidate_bytes_per_row(int max_entries, int k) {
-  return topk_row_bytes(max_entries, k);
+static long long candidate_bytes_per_row(int max_entries, int k, long long rows) {
+  return topk_row_bytes(max_entries, k, rows);
 }
 
 // Workspace layout for a chunk of `rows` queries:
@@ -122,7 +122,7 @@ extern "C" size_t dsv4_index_topk_workspace_size_ex(int qdtype, int B, int nq, i
   if (B <= 0 || nq <= 0 || max_entries <= 0) return 0;
   const bool fp4 = fp4_tensor_path(qdtype, H_I, c_I);
   const long long ld = scores_ld_for(max_entries);
-  const long long cand = candidate_bytes_per_row(max_entries, k > 0 ? k : 0);
+  const long long cand = candidate_bytes_per_row(max_entries, k > 0 ? k : 0, (long long)B * nq);
   const long long qx = fp4 ? (long long)H_I * c_I * 2 : 0;
   const long long kx = fp4 ? (ki_rows > 0 ? ki_rows : 0) * c_I * 2 : 0;
   const long long total = (long long)B * nq;
@@ -167,6 +167,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   a.B = B; a.nq = nq; a.H_I = H_I; a.c_I = c_I; a.m = m; a.k = k; a.max_e = max_entries;
   a.idx = idx;
   a.counts = counts;
+  a.topk_pipe = 0;
   a.nseg = 1;
   a.cand = nullptr;
   a.cand_row_bytes = 0;
@@ -184,7 +185,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   // FP4 operands take the tensor-core kernel through an exact bf16 expansion in the workspace
   // (K^I once, q^I per chunk) when the workspace has room for it; else the CUDA-core kernel.
   const long long ld = scores_ld_for(max_entries);
-  const long long cand = candidate_bytes_per_row(max_entries, k);
+  const long long cand = candidate_bytes_per_row(max_entries, k, (long long)B * nq);
   const long long wsb = ws_ok ? (long long)workspace_bytes : 0;
   bool fp4x = ws_ok && fp4_tensor_path(qdtype, H_I, c_I) && ki_rows > 0 &&
               !(reinterpret_cast<uintptr_t>(KI) & 7u) && !(reinterpret_cast<uintptr_t>(qI) & 7u);
@@ -216,7 +217,8 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     a.scores = reinterpret_cast<float*>(base + L.scores);
     a.scores_ld = ld;
     if (c_use > 0) {
-      a.nseg = 2;
+      if (topk_scheme(max_entries, k, total) == 2) a.topk_pipe = 1;
+      else a.nseg = topk_segments(max_entries);
       a.cand = base + L.cand;
       a.cand_row_bytes = c_use;
     }
@@ -227,7 +229,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   }
   IndexArgs ax = a;                                // the bf16 view of FP4 operands
   if (fp4x) {
-    const IxLayout L = ix_layout(rows, ld, scores_out ? 0 : (a.nseg > 1 ? cand : 0), kx, qx,
+    const IxLayout L = ix_layout(rows, ld, scores_out ? 0 : (a.cand ? cand : 0), kx, qx,
                                  !scores_out);
     char* base = static_cast<char*>(workspace);
     __nv_bfloat16* kbuf = reinterpret_cast<__nv_bfloat16*>(base);

@@ -25,9 +25,13 @@ struct IndexArgs {
   // (0: the whole request; the FP4 path reads a per-chunk bf16 expansion)
   int q_map_q0;
   long long q_map_rows;
-  // threshold top-k of long rows (nseg > 1): one region of cand_row_bytes per score row
-  // (int hist1[256] of key bits 31..24 at its start, then hist2, counters, the entries above
-  // the threshold, the boundary candidates); hist1_done: the score kernel built hist1
+  // top-k of long rows, one region of cand_row_bytes per score row:
+  //  * topk_pipe = 1 (few rows, decode): threshold pipeline; the region holds int hist1[256]
+  //    of key bits 31..24 at its start, then hist2, counters, the entries above the
+  //    threshold and the boundary candidates; hist1_done: the score kernel built hist1;
+  //  * nseg > 1 (many rows): per-segment selection then a merge; the region holds nseg * k
+  //    candidate scores, then their nseg * k entry indices.
+  int topk_pipe;
   int nseg;
   char* cand;
   long long cand_row_bytes;
@@ -94,9 +98,12 @@ int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
 // Zeroes the threshold top-k headers of the score rows of queries [q_begin, q_begin +
 // q_count) (before the score kernel, which may build the first histogram).
 int topk_prepare(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
-// Workspace bytes per score row of the threshold top-k for rows of up to max_entries
-// entries and k winners (0: such rows take the single-stage select).
-long long topk_row_bytes(int max_entries, int k);
+// Top-k scheme for a request of `rows` queries with up to max_entries entries and k winners:
+// 0 single CTA per row, 1 segments + merge, 2 threshold pipeline; and the workspace bytes
+// per score row it needs (0 for scheme 0).
+int topk_scheme(int max_entries, int k, long long rows);
+long long topk_row_bytes(int max_entries, int k, long long rows);
+int topk_segments(int max_entries);
 // FP4 codes [rows, cols/2] + E4M3 scales [rows, cols/16] -> bf16 [rows, cols] (exact).
 int launch_fp4_expand(const uint8_t* codes, const uint8_t* scales, long long rows, int cols,
                       __nv_bfloat16* out, cudaStream_t st);

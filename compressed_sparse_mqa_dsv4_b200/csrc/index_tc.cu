@@ -32,13 +32,15 @@ constexpr int IX_THREADS = 320;
 constexpr uint32_t IX_TM_COLS = 512;
 
 // QT queries per tile, NST key stages in flight. One-query tiles (decode) need a quarter of
-// the Q buffer and spend the room on a deeper key ring.
-template <int QT, int NST>
+// the Q buffer and spend the room on a deeper key ring. HIST: the tile also histograms its
+// scores for the threshold top-k (kept out of the layout otherwise: a few KiB more shared
+// memory cost the prefill shape ~10 % through a smaller L1).
+template <int QT, int NST, bool HIST>
 struct IndexSmem {
   uint8_t q[2][QT * IX_HI * 128];           // K-major SW128: [QT*64 rows][64 ch] per K half
   uint8_t k[NST][2][IX_BLK * 128];          // [128 entries][64 ch] per K half
   float w[QT][IX_HI];
-  int hist[QT][256];                        // key bits 31..24 of the tile's scores (long rows)
+  int hist[HIST ? QT : 1][HIST ? 256 : 1];  // key bits 31..24 of the tile's scores
   uint64_t q_full;
   uint64_t k_full[NST], k_empty[NST];
   uint64_t d_full[2], d_empty[2];
@@ -62,18 +64,18 @@ __device__ unsigned long long g_ix_trace[32][8];
   } while (0)
 #endif
 
-template <int QT, int NST>
-constexpr size_t ix_smem() { return sizeof(IndexSmem<QT, NST>) + 1024; }
-static_assert(ix_smem<4, IX_STAGES>() <= 232448 && ix_smem<1, 6>() <= 232448,
+template <int QT, int NST, bool HIST>
+constexpr size_t ix_smem() { return sizeof(IndexSmem<QT, NST, HIST>) + 1024; }
+static_assert(ix_smem<4, IX_STAGES, true>() <= 232448 && ix_smem<1, 6, true>() <= 232448,
               "shared memory of the index score kernel");
 
-template <int QT, int NST>
+template <int QT, int NST, bool HIST>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     index_tc_kernel(const IndexArgs a, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k, int q_begin, int q_count,
                     int tile0, int tiles_per_seq, int chunk, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
-  IndexSmem<QT, NST>& s = *reinterpret_cast<IndexSmem<QT, NST>*>(
+  IndexSmem<QT, NST, HIST>& s = *reinterpret_cast<IndexSmem<QT, NST, HIST>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int tile = tile0 + blockIdx.x;
@@ -111,7 +113,8 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     s.abort = 0;
     tc::fence_barrier_init();
   }
-  for (int e = tid; e < QT * 256; e += blockDim.x) s.hist[e >> 8][e & 255] = 0;
+  if constexpr (HIST)
+    for (int e = tid; e < QT * 256; e += blockDim.x) s.hist[e >> 8][e & 255] = 0;
   for (int e = tid; e < QT * IX_HI; e += blockDim.x) {
     const int u = e / IX_HI, h = e % IX_HI;
     s.w[u][h] = u < nqt ? a.w[(long long)(qlo + u) * a.H_I + h] : 0.f;
@@ -244,7 +247,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[32 + h], fmaxf(d3[h], 0.f), sc1);
       }
       if (sidx < Et[0]) a.scores[srow[0] + sidx] = sc0;
-      if (a.nseg > 1) {                          // first histogram of the threshold top-k
+      if constexpr (HIST) {                      // first histogram of the threshold top-k
         hist_add(s.hist[QT > 1 ? 2 * qp : 0], score_key(sc0) >> 24, sidx < Et[0]);
         if (QT > 1) hist_add(s.hist[QT > 1 ? 2 * qp + 1 : 0], score_key(sc1) >> 24, 2 * qp + 1 < nqt && sidx < Et[1]);
       }
@@ -258,7 +261,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, IX_TM_COLS);
   }
-  if (a.nseg > 1) {
+  if constexpr (HIST) {
     // add the tile's histograms to the rows' first histograms (int hist1[256] at the start
     // of each row's top-k region)
     for (int e = tid; e < nqt * 256; e += blockDim.x) {
@@ -304,21 +307,37 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
   if (grid.y > 65535) return DSV4_OK;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<IX_QT, IX_STAGES>,
+    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<IX_QT, IX_STAGES, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ix_smem<IX_QT, IX_STAGES>());
+                                         (int)ix_smem<IX_QT, IX_STAGES, false>());
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(index_tc_kernel<1, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)ix_smem<1, 6>());
+      e = cudaFuncSetAttribute(index_tc_kernel<IX_QT, IX_STAGES, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ix_smem<IX_QT, IX_STAGES, true>());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(index_tc_kernel<1, 6, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)ix_smem<1, 6, false>());
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(index_tc_kernel<1, 6, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)ix_smem<1, 6, true>());
     if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "index_tc: %s", cudaGetErrorString(e));
     attr_set = true;
   }
-  if (qt == 1)
-    index_tc_kernel<1, 6><<<grid, IX_THREADS, ix_smem<1, 6>(), st>>>(a, mq, mk, q_begin, q_count, t0,
-                                                                    tps, chunk, spin_limit());
-  else
-    index_tc_kernel<IX_QT, IX_STAGES><<<grid, IX_THREADS, ix_smem<IX_QT, IX_STAGES>(), st>>>(
-        a, mq, mk, q_begin, q_count, t0, tps, chunk, spin_limit());
+  const int sp = spin_limit();
+  if (qt == 1) {
+    if (a.topk_pipe)
+      index_tc_kernel<1, 6, true><<<grid, IX_THREADS, ix_smem<1, 6, true>(), st>>>(a, mq, mk, q_begin, q_count,
+                                                                                 t0, tps, chunk, sp);
+    else
+      index_tc_kernel<1, 6, false><<<grid, IX_THREADS, ix_smem<1, 6, false>(), st>>>(a, mq, mk, q_begin, q_count,
+                                                                                   t0, tps, chunk, sp);
+  } else {
+    if (a.topk_pipe)
+      index_tc_kernel<IX_QT, IX_STAGES, true><<<grid, IX_THREADS, ix_smem<IX_QT, IX_STAGES, true>(), st>>>(
+          a, mq, mk, q_begin, q_count, t0, tps, chunk, sp);
+    else
+      index_tc_kernel<IX_QT, IX_STAGES, false><<<grid, IX_THREADS, ix_smem<IX_QT, IX_STAGES, false>(), st>>>(
+          a, mq, mk, q_begin, q_count, t0, tps, chunk, sp);
+  }
   *used = true;
   return launch_status("index scores (tensor cores)");
 }

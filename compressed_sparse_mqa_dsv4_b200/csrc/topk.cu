@@ -223,8 +223,76 @@ __global__ void __launch_bounds__(NT) topk_kernel(IndexArgs a, int q_begin) {
   select_topk<NT, NT == 256>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; });
 }
 
+// ---------------------------------------------------------------- segments + merge
+// Requests with many long rows: stage 1 selects, per segment of TOPK_SEG entries, that
+// segment's top k under the same order (score descending, then entry ascending) -- every
+// entry of the query's top k is in its segment's top k, since the entries ranked above it
+// within the segment are a subset of those ranked above it overall; stage 2 selects the
+// query's top k among the concatenated segment candidates, already in ascending entry order.
+// Candidates of a row: nseg * k scores, then nseg * k entry indices, in its region.
+
+// Stage 1: grid (segment, query). Writes the segment's top min(k, segment length) entries
+// (score and global entry index) in ascending entry order to its k candidate slots and pads
+// the rest with score -inf / index -1.
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_seg_kernel(IndexArgs a, int q_begin) {
+  __shared__ TopkShared sh;
+  const int qg = q_begin + blockIdx.y, seg = blockIdx.x;
+  const int b = qg / a.nq, i = qg % a.nq;
+  const int Et = visible_entries(a, b, i);
+  const int k = a.k;
+  const long long row = qg - a.score_q0;
+  char* region = a.cand + row * a.cand_row_bytes;
+  float* cs = reinterpret_cast<float*>(region) + (long long)seg * k;
+  int32_t* ci = reinterpret_cast<int32_t*>(region + (long long)a.nseg * k * 4) + (long long)seg * k;
+  const int lo = seg * TOPK_SEG;
+  const int len = max(0, min(Et, lo + TOPK_SEG) - lo);
+  const int kseg = min(k, len);
+  const float* sc = a.scores + row * a.scores_ld + lo;
+  for (int j = kseg + threadIdx.x; j < k; j += blockDim.x) {
+    cs[j] = -INFINITY;
+    ci[j] = -1;
+  }
+  if (kseg == len) {                              // the whole segment is a candidate set
+    for (int j = threadIdx.x; j < len; j += blockDim.x) {
+      cs[j] = sc[j];
+      ci[j] = lo + j;
+    }
+    return;
+  }
+  select_topk<NT, false>(sc, len, kseg, sh, [&](int p, int j) {
+    cs[p] = sc[j];
+    ci[p] = lo + j;
+  });
+}
+
+// Stage 2: one CTA per query over its nseg * k candidates.
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_merge_kernel(IndexArgs a, int q_begin) {
+  __shared__ TopkShared sh;
+  const int qg = q_begin + blockIdx.x;
+  const int b = qg / a.nq, i = qg % a.nq;
+  const int Et = visible_entries(a, b, i);
+  const int k = a.k;
+  const int keff = min(k, Et);
+  int32_t* out = a.idx + (long long)qg * k;
+  if (threadIdx.x == 0) a.counts[qg] = keff;
+  for (int j = keff + threadIdx.x; j < k; j += blockDim.x) out[j] = -1;
+  if (keff == 0) return;
+  if (Et <= k) {
+    for (int j = threadIdx.x; j < Et; j += blockDim.x) out[j] = j;
+    return;
+  }
+  const long long row = qg - a.score_q0;
+  const char* region = a.cand + row * a.cand_row_bytes;
+  const float* cs = reinterpret_cast<const float*>(region);
+  const int32_t* ci = reinterpret_cast<const int32_t*>(region + (long long)a.nseg * k * 4);
+  select_topk<NT, false>(cs, a.nseg * k, keff, sh, [&](int p, int j) { out[p] = ci[j]; });
+}
+
 // ---------------------------------------------------------------- threshold pipeline
-// Rows longer than TOPK_SEG entries (decode over long contexts). Each pass is spread over
+// Requests with few rows longer than TOPK_SEG entries (decode over long contexts). Each pass
+// is spread over
 // CTAs of TK_PASS entries and streams the row once:
 //   hist1  per-row histogram of key bits 31..24;
 //   hist2  the bin B1 holding the k_eff-th largest key -> histogram of bits 23..16 of the
@@ -491,7 +559,7 @@ __global__ void __launch_bounds__(NT) topk_final_kernel(IndexArgs a, int q_begin
 
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
   if (q_count <= 0) return DSV4_OK;
-  if (a.nseg > 1) {
+  if (a.topk_pipe) {
     constexpr int kFinalSmem = TK_CAND * 8 + TK_MAXK * 4;
     static bool attr_set = false;
     if (!attr_set) {
@@ -506,6 +574,12 @@ int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
     topk_hist2_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
     topk_filter_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
     topk_final_kernel<1024><<<q_count, 1024, kFinalSmem, st>>>(a, q_begin);
+  } else if (a.nseg > 1) {
+    topk_seg_kernel<256><<<dim3(a.nseg, q_count), 256, 0, st>>>(a, q_begin);
+    if ((long long)a.nseg * a.k >= 4096)
+      topk_merge_kernel<1024><<<q_count, 1024, 0, st>>>(a, q_begin);
+    else
+      topk_merge_kernel<256><<<q_count, 256, 0, st>>>(a, q_begin);
   } else if (a.max_e > TOPK_SEG) {                // long rows without the pipeline's scratch
     topk_kernel<1024><<<q_count, 1024, 0, st>>>(a, q_begin);
   } else {
@@ -515,16 +589,32 @@ int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
 }
 
 int topk_prepare(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
-  if (a.nseg <= 1 || q_count <= 0) return DSV4_OK;
+  if (!a.topk_pipe || q_count <= 0) return DSV4_OK;
   const long long row0 = q_begin - a.score_q0;
   const cudaError_t e = cudaMemset2DAsync(a.cand + row0 * a.cand_row_bytes, (size_t)a.cand_row_bytes, 0,
                                           (size_t)TK_HDR, (size_t)q_count, st);
   return e == cudaSuccess ? DSV4_OK : fail(DSV4_ERR_CUDA, "top-k: %s", cudaGetErrorString(e));
 }
 
-long long topk_row_bytes(int max_entries, int k) {
-  if (max_entries <= TOPK_SEG || k <= 0 || k > TK_MAXK) return 0;
-  return TK_HDR + (((long long)k * 4 + 255) & ~255ll) + (long long)TK_CAND * 8;
+int topk_segments(int max_entries) {
+  return max_entries > TOPK_SEG ? (max_entries + TOPK_SEG - 1) / TOPK_SEG : 1;
+}
+
+// The pipeline pays its per-row final select and its extra passes only when few rows share
+// the GPU (a decode batch); many rows keep every SM busy with per-segment selects.
+constexpr long long TK_PIPE_ROWS = 1024;
+
+int topk_scheme(int max_entries, int k, long long rows) {
+  if (max_entries <= TOPK_SEG || k <= 0) return 0;
+  return (rows <= TK_PIPE_ROWS && k <= TK_MAXK) ? 2 : 1;
+}
+
+long long topk_row_bytes(int max_entries, int k, long long rows) {
+  switch (topk_scheme(max_entries, k, rows)) {
+    case 2: return TK_HDR + (((long long)k * 4 + 255) & ~255ll) + (long long)TK_CAND * 8;
+    case 1: return (long long)topk_segments(max_entries) * k * 8;
+    default: return 0;
+  }
 }
 
 }  // namespace dsv4

@@ -129,6 +129,20 @@ def test_index_decode_long_contexts(dsv4):
                    what="decode long")
 
 
+def test_index_many_long_rows(dsv4):
+    """More than 1024 queries whose rows exceed 16384 entries: the workspace path selects per
+    16384-entry segment and merges the candidates (the threshold pipeline serves requests with
+    few rows, as in decode)."""
+    shape = preset("flash_csa_prefill", H_I=4, c_I=16)
+    nq, E0 = 1100, 17000
+    pos0 = [4 * E0]
+    g = Generator(31)
+    qI, w = g.index_queries(shape, nq)
+    KI = g.index_keys(shape, (pos0[0] + nq) // 4 + 1)
+    _run_and_check(dsv4, qI, w, KI, [0], pos0, 4, 256, [(0, i) for i in (0, 1, 547, 1099)],
+                   what="many long rows")
+
+
 def test_index_flash_full_sampled(dsv4, index_path):
     """V4-Flash shape: n=8192, H_I=64, c_I=128, k=512; every query run, a sample compared."""
     shape = preset("flash_csa_prefill")
