@@ -727,16 +727,17 @@ __global__ void __maxnreg__(128)
   }
 }
 
-// Merges the nsplit partials of every (query, head group): one warp per head, the combined
-// max M over the splits and the sink, weights 2^(m_s - M), one normalisation, bf16 output,
-// LSE. Splits without candidates carry m = -inf and are not read.
+// Merges the nsplit partials of every (query, head group): one warp per head (grid: items x
+// 8 CTAs of 8 warps), the combined max M over the splits and the sink, weights 2^(m_s - M),
+// one normalisation, bf16 output, LSE. Splits without candidates carry m = -inf and are not
+// read.
 __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnArgs a, int head_groups) {
   const int base = blockIdx.x;
   const int qi = base / head_groups, hg = base % head_groups;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = a.nsplit;
-  for (int r = 0; r < AT_H / 8; ++r) {
-    const int hl = 8 * warp + r;                       // head within the group
+  {
+    const int hl = 8 * blockIdx.y + warp;              // head within the group
     const int h = hg * AT_H + hl;
     const float2 ml = lane < S ? a.part_ml[((long long)base * S + lane) * AT_H + hl]
                                : make_float2(-INFINITY, 0.f);
@@ -856,7 +857,7 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   *used = true;
   int s2 = launch_status("hybrid attention (tensor cores)");
   if (s2 != DSV4_OK || nsplit == 1) return s2;
-  attn_combine_kernel<<<(unsigned)items, 256, 0, st>>>(a, a.H / AT_H);
+  attn_combine_kernel<<<dim3((unsigned)items, AT_H / 8), 256, 0, st>>>(a, a.H / AT_H);
   return launch_status("hybrid attention split combine");
 }
 
