@@ -23,7 +23,8 @@
 //         stores.
 //   8-11  producer (one per sub-partition; each warp instruction moves one 128-byte chunk
 //         of 4 rows): resolves the block's 128 row addresses, then gathers them with 16-byte
-//         cp.async, chunk by chunk as GEMM2 of the previous block releases each chunk pair.
+//         cp.async, chunk by chunk as GEMM2 of the previous block releases each chunk pair;
+//         completion is signalled per half block (chunks 0-3, 4-7).
 //   12    watcher: waits for GEMM2's chunk releases and the Q buffer on the producers'
 //         behalf and passes them on through named-barrier gates (a producer's own mbarrier
 //         wait would queue behind its cp.async traffic and stall the gather).
@@ -69,7 +70,7 @@ struct AttnSmem {
   float inv[AT_H];
   uint64_t rowaddr[AT_BLK];
   uint64_t q_full, q_empty;
-  uint64_t ch_full[AT_CHUNKS], ch_empty[4];
+  uint64_t ch_full[AT_CHUNKS], ch_empty[4];  // ch_full[3], ch_full[7]: chunks 0-3, 4-7 landed
   uint64_t s_full, p_full, o_done, drain;
   uint32_t tmem_base;
   int abort;
@@ -310,8 +311,7 @@ __global__ void __maxnreg__(128)
             if (G > 0) pair_sync(GATE_PAIR0 + (c >> 1));
             if (pt == 0) A1_TRACE(8 + (c >> 1), k, j);
             if (tma_win && pt == 0) {
-              tc::mbar_expect_tx(&s.ch_full[c], (AT_BLK - ls) * 128);
-              tc::mbar_expect_tx(&s.ch_full[c + 1], (AT_BLK - ls) * 128);
+              tc::mbar_expect_tx(&s.ch_full[c | 3], 2 * (AT_BLK - ls) * 128);
             }
           }
           uint8_t* dst = s.kv[c];
@@ -321,10 +321,13 @@ __global__ void __maxnreg__(128)
               cp_async16(kv0 + (uint32_t)(c * AT_BLK * 128) + dsto[i], src[i] + (uint64_t)(128 * c));
           if (tma_win && pt == 0) {
             for (int r0 = ls; r0 < AT_BLK; r0 += 32)
-              tc::tma_load_2d(dst + r0 * 128, &map_local, &s.ch_full[c], 64 * c,
+              tc::tma_load_2d(dst + r0 * 128, &map_local, &s.ch_full[c | 3], 64 * c,
                               (int32_t)(first_row + (r0 - ls)));
           }
-          cp_async_arrive_noinc(&s.ch_full[c]);
+          // One completion arrival per four chunks: each such arrival stalls the issuing
+          // thread for a few hundred cycles (measured), so per-chunk arrivals throttled the
+          // gather; GEMM1 then consumes the block in two halves.
+          if ((c & 3) == 3) cp_async_arrive_noinc(&s.ch_full[c]);
           if (pt == 0 && (c & 1)) A1_TRACE(28 + (c >> 1), k, j);
         }
         if (pt == 0) A1_TRACE(1, k, j);
@@ -338,7 +341,7 @@ __global__ void __maxnreg__(128)
       volatile int never = 0;
       if (k > 0) tc::mbar_wait(&s.q_full, (uint32_t)((k - 1) & 1), spin, &never);
       if (G > 0)
-        for (int c = 0; c < AT_CHUNKS; ++c) tc::mbar_wait(&s.ch_full[c], (G - 1) & 1, spin, &never);
+        for (int c = 3; c < AT_CHUNKS; c += 4) tc::mbar_wait(&s.ch_full[c], (G - 1) & 1, spin, &never);
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------------ watcher
@@ -398,7 +401,7 @@ __global__ void __maxnreg__(128)
         for (int j = it.jb; j < it.je && ok; ++j, ++G) {
 #pragma unroll
           for (int c = 0; c < AT_CHUNKS; ++c) {
-            ok = wwait(&s.ch_full[c], G & 1);
+            if ((c & 3) == 0) ok = wwait(&s.ch_full[c | 3], G & 1);
             if (!ok) break;
             if (lane == 0 && (c & 1)) A1_TRACE(12 + (c >> 1), k, j);
             tc::fence_proxy_async_smem();          // cp.async (generic) -> tensor core (async)
