@@ -8,10 +8,11 @@
 // entry's dot products with every head of every query in the tile, and the weighted
 // ReLU head sum is a per-thread reduction in registers:
 //     D[128 entries x 64*nqt] = K^I_blk[128 x c_I] . qI_tile[64*nqt x c_I]^T
-// One CTA per (tile of <= 4 queries of one sequence, chunk of 4096-16384 entries), 10 warps:
+// CTAs walk work units (tile of <= 4 queries of one sequence, chunk of 4096-16384 entries):
+// persistent, one per SM, for multi-query tiles; one per unit for one-query tiles. 10 warps:
 //   warps 0-7  epilogue: warp w reads TMEM lane quadrant w%4 for queries 2(w/4), 2(w/4)+1
-//   warp 8     producer: the query tile once, then 128-entry key blocks by 2D TMA into a
-//              4-stage ring
+//   warp 8     producer: per unit the query tile, then 128-entry key blocks by 2D TMA into a
+//              4-stage ring (6 stages for one-query tiles) that runs on across units
 //   warp 9     MMA issuer and TMEM owner; D is double-buffered (2 x 256 columns)
 // Scores of entries a query cannot see are not written. All waits are bounded.
 #include <cstdlib>
@@ -41,7 +42,7 @@ struct IndexSmem {
   uint8_t k[NST][2][IX_BLK * 128];          // [128 entries][64 ch] per K half
   float w[QT][IX_HI];
   int hist[HIST ? QT : 1][HIST ? 256 : 1];  // key bits 31..24 of the tile's scores
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[NST], k_empty[NST];
   uint64_t d_full[2], d_empty[2];
   uint64_t drain;
@@ -69,38 +70,66 @@ constexpr size_t ix_smem() { return sizeof(IndexSmem<QT, NST, HIST>) + 1024; }
 static_assert(ix_smem<4, IX_STAGES, true>() <= 232448 && ix_smem<1, 6, true>() <= 232448,
               "shared memory of the index score kernel");
 
+// Named-barrier OR-reduction over `threads` threads (all take the same decision).
+__device__ __forceinline__ bool ix_red_or(uint32_t id, uint32_t threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n"
+      " barrier.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
+// A work unit: a tile of <= QT queries of one sequence and a chunk of its entries. Every
+// role derives the same units in the same order and skips the empty ones.
+struct IxUnit {
+  int b, qlo, nqt, e0, e1;
+  long long base;
+  bool valid;
+};
+
+// Units are numbered chunk-major (all tiles' first chunks, then their second chunks, ...), so
+// the valid units of rows of different lengths form a dense prefix that the CTAs' round robin
+// spreads evenly.
+template <int QT>
+__device__ __forceinline__ IxUnit ix_unit(const IndexArgs& a, int u, int q_begin, int q_count,
+                                          int tile0, int tiles_per_seq, int chunk, int ntiles) {
+  IxUnit r;
+  const int tile = tile0 + u % ntiles, c = u / ntiles;
+  r.b = tile / tiles_per_seq;
+  const int i0 = (tile % tiles_per_seq) * QT;
+  r.qlo = max(r.b * a.nq + i0, q_begin);
+  const int qhi = min(r.b * a.nq + min(i0 + QT, a.nq), q_begin + q_count);
+  r.nqt = qhi - r.qlo;
+  const int e_tile = r.nqt > 0 ? visible_entries(a, r.b, qhi - 1 - r.b * a.nq) : 0;
+  r.e0 = c * chunk;
+  r.e1 = min(e_tile, r.e0 + chunk);
+  r.base = r.nqt > 0 ? a.kv_row_off[r.b] : 0;
+  const bool bounds_ok = r.base >= 0 && r.base + e_tile <= a.ki_rows;
+  r.valid = r.nqt > 0 && r.e1 > r.e0 && bounds_ok;
+  if (r.nqt > 0 && !bounds_ok && c == 0 && threadIdx.x == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
+  return r;
+}
+
+// Persistent: each CTA walks the work units blockIdx.x, blockIdx.x + gridDim.x, ...; the key
+// ring, the TMEM double buffer and their barrier phases run on across units (global block
+// counter), the Q buffer is reloaded per unit once the MMAs of the previous unit are done.
 template <int QT, int NST, bool HIST>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     index_tc_kernel(const IndexArgs a, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k, int q_begin, int q_count,
-                    int tile0, int tiles_per_seq, int chunk, uint32_t spin) {
+                    int tile0, int tiles_per_seq, int chunk, int ntiles, int units, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
   IndexSmem<QT, NST, HIST>& s = *reinterpret_cast<IndexSmem<QT, NST, HIST>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = tile0 + blockIdx.x;
-  const int b = tile / tiles_per_seq;
-  const int i0 = (tile % tiles_per_seq) * QT;
-  // queries of this tile inside [q_begin, q_begin + q_count)
-  int qlo = b * a.nq + i0, qhi = b * a.nq + min(i0 + QT, a.nq);
-  qlo = max(qlo, q_begin);
-  qhi = min(qhi, q_begin + q_count);
-  const int nqt = qhi - qlo;                       // queries in the tile (may be 0)
-  int e_tile = 0;                                  // entries seen by the tile's last query
-  if (nqt > 0) e_tile = visible_entries(a, b, qhi - 1 - b * a.nq);
-  const int e0 = blockIdx.y * chunk;
-  const int e1 = min(e_tile, e0 + chunk);
-  const long long base = nqt > 0 ? a.kv_row_off[b] : 0;
-  const bool bounds_ok = base >= 0 && base + e_tile <= a.ki_rows;
-  if (nqt <= 0 || e1 <= e0 || !bounds_ok) {
-    if (nqt > 0 && !bounds_ok && tid == 0 && blockIdx.y == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
-    return;                                        // uniform exit before any barrier
-  }
-  const int nblk = (e1 - e0 + IX_BLK - 1) / IX_BLK;
   volatile int* abort = &s.abort;
 
   if (tid == 0) {
     tc::mbar_init(&s.q_full, 1);
+    tc::mbar_init(&s.q_empty, 1);
     for (int i = 0; i < NST; ++i) {
       tc::mbar_init(&s.k_full[i], 1);
       tc::mbar_init(&s.k_empty[i], 1);
@@ -115,10 +144,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   }
   if constexpr (HIST)
     for (int e = tid; e < QT * 256; e += blockDim.x) s.hist[e >> 8][e & 255] = 0;
-  for (int e = tid; e < QT * IX_HI; e += blockDim.x) {
-    const int u = e / IX_HI, h = e % IX_HI;
-    s.w[u][h] = u < nqt ? a.w[(long long)(qlo + u) * a.H_I + h] : 0.f;
-  }
   if (warp == 9) {
     tc::tmem_alloc(&s.tmem_base, IX_TM_COLS);
     tc::tmem_relinquish();
@@ -131,30 +156,66 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
-      int issued[NST];
-#pragma unroll
-      for (int st = 0; st < NST; ++st) issued[st] = 0;
       tc::prefetch_tensormap(&map_q);
       tc::prefetch_tensormap(&map_k);
-      tc::mbar_arrive_expect_tx(&s.q_full, 2 * QT * IX_HI * 128);
-      const int qrow = (qlo - a.q_map_q0) * IX_HI;
-      tc::tma_load_2d(s.q[0], &map_q, &s.q_full, 0, qrow);
-      tc::tma_load_2d(s.q[1], &map_q, &s.q_full, 64, qrow);
-      for (int blk = 0; blk < nblk; ++blk) {
-        const int st = blk % NST, use = blk / NST;
-        if (use > 0 && !tc::mbar_wait(&s.k_empty[st], (uint32_t)((use - 1) & 1), spin, abort)) break;
-        tc::mbar_arrive_expect_tx(&s.k_full[st], 2 * IX_BLK * 128);
-        const int row = (int)(base + e0 + blk * IX_BLK);
-        tc::tma_load_2d(s.k[st][0], &map_k, &s.k_full[st], 0, row);
-        tc::tma_load_2d(s.k[st][1], &map_k, &s.k_full[st], 64, row);
-        IX_TRACE(0, blk);
-        issued[st] = use + 1;
+      uint32_t gb = 0;                                 // key blocks issued so far
+      int k = 0;                                       // units loaded so far
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const IxUnit w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+        if (!w.valid) continue;
+        // The unit's Q goes into the single Q buffer once the MMAs of the previous unit have
+        // completed (q_empty). Meanwhile the unit's first key blocks already enter the ring:
+        // up to NST of them reuse stages the previous units released, so the ring stays full
+        // across the unit boundary; a later block's stage is released only by this unit's
+        // MMAs, which need its Q, so Q is loaded (waiting if need be) before that.
+        bool q_loaded = false;
+        auto load_q = [&]() {
+          tc::mbar_arrive_expect_tx(&s.q_full, 2 * QT * IX_HI * 128);
+          const int qrow = (w.qlo - a.q_map_q0) * IX_HI;
+          tc::tma_load_2d(s.q[0], &map_q, &s.q_full, 0, qrow);
+          tc::tma_load_2d(s.q[1], &map_q, &s.q_full, 64, qrow);
+          q_loaded = true;
+        };
+        auto q_free = [&](bool block) {
+          if (k == 0) return true;
+          const uint32_t par = (uint32_t)((k - 1) & 1);
+          return block ? tc::mbar_wait(&s.q_empty, par, spin, abort) : tc::mbar_test_wait(&s.q_empty, par);
+        };
+        const uint32_t gb0 = gb;
+        const int nblk = (w.e1 - w.e0 + IX_BLK - 1) / IX_BLK;
+        for (int blk = 0; blk < nblk; ++blk, ++gb) {
+          const int st = gb % NST, use = gb / NST;
+          if (!q_loaded && gb >= gb0 + NST) {
+            if (!q_free(true)) {
+              ok = false;
+              break;
+            }
+            load_q();
+          }
+          if (use > 0 && !tc::mbar_wait(&s.k_empty[st], (uint32_t)((use - 1) & 1), spin, abort)) {
+            ok = false;
+            break;
+          }
+          if (!q_loaded && q_free(false)) load_q();
+          tc::mbar_arrive_expect_tx(&s.k_full[st], 2 * IX_BLK * 128);
+          const int row = (int)(w.base + w.e0 + blk * IX_BLK);
+          tc::tma_load_2d(s.k[st][0], &map_k, &s.k_full[st], 0, row);
+          tc::tma_load_2d(s.k[st][1], &map_k, &s.k_full[st], 64, row);
+          IX_TRACE(0, (int)gb);
+        }
+        if (ok && !q_loaded) {
+          if (!q_free(true)) break;
+          load_q();
+        }
+        if (q_loaded) ++k;
       }
       if (*abort) {
+        // the consumers gave up: let this thread's own bulk copies land before exiting
         volatile int never = 0;
-        for (int st = 0; st < NST; ++st)
-          if (issued[st] > 0) tc::mbar_wait(&s.k_full[st], (uint32_t)((issued[st] - 1) & 1), spin, &never);
-        tc::mbar_wait(&s.q_full, 0, spin, &never);
+        for (uint32_t g = gb > (uint32_t)NST ? gb - NST : 0; g < gb; ++g)
+          tc::mbar_wait(&s.k_full[g % NST], (g / NST) & 1, spin, &never);
+        if (k > 0) tc::mbar_wait(&s.q_full, (uint32_t)((k - 1) & 1), spin, &never);
       }
     }
     __syncwarp();
@@ -164,31 +225,41 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     // decision, and elect.sync lets one lane issue. A single-lane branch issued the MMAs and
     // passed completed barriers several times more slowly, which capped the key stream.
     {
-      const uint32_t idesc = tc::idesc_bf16_f32(128, IX_HI * nqt, 0, 0);
       const uint64_t d_k0 = tc::sdesc_sw128(tc::smem_u32(s.k[0][0]), 16, 1024);
       const uint64_t d_q0 = tc::sdesc_sw128(tc::smem_u32(s.q[0]), 16, 1024);
       auto wwait = [&](uint64_t* bar, uint32_t parity) {
         return __all_sync(0xffffffffu, tc::mbar_wait(bar, parity, spin, abort)) != 0;
       };
-      bool ok = wwait(&s.q_full, 0);
-      for (int blk = 0; blk < nblk && ok; ++blk) {
-        const int st = blk % NST, buf = blk & 1;
-        ok = wwait(&s.k_full[st], (uint32_t)((blk / NST) & 1));
-        IX_TRACE(1, blk);
-        if (ok && blk >= 2) ok = wwait(&s.d_empty[buf], (uint32_t)(((blk >> 1) - 1) & 1));
-        IX_TRACE(2, blk);
-        if (!ok) break;
-        tc::tc_fence_after();
-        // descriptor start addresses (16-byte units): key stage st, K half kk/4, K step kk%4
+      uint32_t gb = 0;
+      int k = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const IxUnit w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+        if (!w.valid) continue;
+        ok = wwait(&s.q_full, (uint32_t)(k & 1));
+        ++k;
+        const uint32_t idesc = tc::idesc_bf16_f32(128, IX_HI * w.nqt, 0, 0);
+        const int nblk = (w.e1 - w.e0 + IX_BLK - 1) / IX_BLK;
+        for (int blk = 0; blk < nblk && ok; ++blk, ++gb) {
+          const int st = gb % NST, buf = gb & 1;
+          ok = wwait(&s.k_full[st], (uint32_t)((gb / NST) & 1));
+          IX_TRACE(1, (int)gb);
+          if (ok && gb >= 2) ok = wwait(&s.d_empty[buf], (uint32_t)(((gb >> 1) - 1) & 1));
+          IX_TRACE(2, (int)gb);
+          if (!ok) break;
+          tc::tc_fence_after();
+          // descriptor start addresses (16-byte units): key stage st, K half kk/4, K step kk%4
 #pragma unroll
-        for (int kk = 0; kk < IX_CI / 16; ++kk)
-          tc::mma_bf16_ss_warp(tmem + buf * 256,
-                               d_k0 + (uint64_t)(st * (2 * IX_BLK * 128 / 16) + (kk >> 2) * (IX_BLK * 128 / 16) + (kk & 3) * 2),
-                               d_q0 + (uint64_t)((kk >> 2) * (QT * IX_HI * 128 / 16) + (kk & 3) * 2), idesc,
-                               kk > 0 ? 1u : 0u);
-        tc::mma_commit_warp(&s.k_empty[st]);
-        tc::mma_commit_warp(&s.d_full[buf]);
-        IX_TRACE(3, blk);
+          for (int kk = 0; kk < IX_CI / 16; ++kk)
+            tc::mma_bf16_ss_warp(tmem + buf * 256,
+                                 d_k0 + (uint64_t)(st * (2 * IX_BLK * 128 / 16) + (kk >> 2) * (IX_BLK * 128 / 16) + (kk & 3) * 2),
+                                 d_q0 + (uint64_t)((kk >> 2) * (QT * IX_HI * 128 / 16) + (kk & 3) * 2), idesc,
+                                 kk > 0 ? 1u : 0u);
+          tc::mma_commit_warp(&s.k_empty[st]);
+          tc::mma_commit_warp(&s.d_full[buf]);
+          IX_TRACE(3, (int)gb);
+        }
+        if (ok) tc::mma_commit_warp(&s.q_empty);       // the unit's Q is no longer read
       }
       if (!ok) {
         // let every issued MMA finish before TMEM is released
@@ -203,56 +274,85 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     const int quad = warp & 3;                    // TMEM lane quadrant
     const int qp = warp >> 2;                     // query pair: queries 2qp, 2qp+1
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
-    int Et[2];
-    long long srow[2];
+    uint32_t gb = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const IxUnit w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+      if (!w.valid) continue;
+      // every epilogue thread has finished the previous unit; after a failed wait all of
+      // them leave here together (named barriers below need all 256)
+      if (ix_red_or(1, 256, !ok)) break;
+      // the unit's head weights
+      for (int e = tid; e < QT * IX_HI; e += 256) {
+        const int q = e / IX_HI, h = e % IX_HI;
+        s.w[q][h] = q < w.nqt ? a.w[(long long)(w.qlo + q) * a.H_I + h] : 0.f;
+      }
+      tc::named_barrier(1, 256);
+      int Et[2];
+      long long srow[2];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int qu = 2 * qp + u;
-      Et[u] = qu < nqt ? visible_entries(a, b, qlo + qu - b * a.nq) : 0;
-      srow[u] = (long long)(qlo + qu - a.score_q0) * a.scores_ld;
-    }
-    for (int blk = 0; blk < nblk; ++blk) {
-      const int buf = blk & 1;
-      if (!tc::mbar_wait(&s.d_full[buf], (uint32_t)((blk >> 1) & 1), spin, abort)) break;
-      if (tid == 0) IX_TRACE(4, blk);
-      tc::tc_fence_after();
-      float d0[32], d1[32], d2[32], d3[32];
-      const uint32_t col = tmem + lane_base + buf * 256 + qp * 128;
-      const bool two = 2 * qp < nqt;              // this warp has work in the tile
-      if (two) {
-        tc::tmem_ld32(col, d0);
-        tc::tmem_ld32(col + 32, d1);
-        if constexpr (QT > 1) {                   // one-query tiles have no second query
-          tc::tmem_ld32(col + 64, d2);
-          tc::tmem_ld32(col + 96, d3);
+      for (int v = 0; v < 2; ++v) {
+        const int qu = 2 * qp + v;
+        Et[v] = qu < w.nqt ? visible_entries(a, w.b, w.qlo + qu - w.b * a.nq) : 0;
+        srow[v] = (long long)(w.qlo + qu - a.score_q0) * a.scores_ld;
+      }
+      const int nblk = (w.e1 - w.e0 + IX_BLK - 1) / IX_BLK;
+      for (int blk = 0; blk < nblk; ++blk, ++gb) {
+        const int buf = gb & 1;
+        ok = tc::mbar_wait(&s.d_full[buf], (uint32_t)((gb >> 1) & 1), spin, abort);
+        if (!ok) break;
+        if (tid == 0) IX_TRACE(4, (int)gb);
+        tc::tc_fence_after();
+        float d0[32], d1[32], d2[32], d3[32];
+        const uint32_t col = tmem + lane_base + buf * 256 + qp * 128;
+        const bool two = 2 * qp < w.nqt;          // this warp has work in the tile
+        if (two) {
+          tc::tmem_ld32(col, d0);
+          tc::tmem_ld32(col + 32, d1);
+          if constexpr (QT > 1) {                 // one-query tiles have no second query
+            tc::tmem_ld32(col + 64, d2);
+            tc::tmem_ld32(col + 96, d3);
+          }
+          tc::tmem_wait_ld();
         }
-        tc::tmem_wait_ld();
+        tc::tc_fence_before();
+        tc::mbar_arrive(&s.d_empty[buf]);
+        if (tid == 0) IX_TRACE(5, (int)gb);
+        if (!two) continue;
+        const int sidx = w.e0 + blk * IX_BLK + 32 * quad + lane;
+        float sc0 = 0.f, sc1 = 0.f;
+        const float* w0 = s.w[QT > 1 ? 2 * qp : 0];
+        const float* w1 = s.w[QT > 1 ? 2 * qp + 1 : 0];
+#pragma unroll
+        for (int h = 0; h < 32; ++h) sc0 = fmaf(w0[h], fmaxf(d0[h], 0.f), sc0);
+#pragma unroll
+        for (int h = 0; h < 32; ++h) sc0 = fmaf(w0[32 + h], fmaxf(d1[h], 0.f), sc0);
+        if constexpr (QT > 1) {
+#pragma unroll
+          for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[h], fmaxf(d2[h], 0.f), sc1);
+#pragma unroll
+          for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[32 + h], fmaxf(d3[h], 0.f), sc1);
+        }
+        if (sidx < Et[0]) a.scores[srow[0] + sidx] = sc0;
+        if constexpr (HIST) {                    // first histogram of the threshold top-k
+          hist_add(s.hist[QT > 1 ? 2 * qp : 0], score_key(sc0) >> 24, sidx < Et[0]);
+          if (QT > 1) hist_add(s.hist[QT > 1 ? 2 * qp + 1 : 0], score_key(sc1) >> 24, 2 * qp + 1 < w.nqt && sidx < Et[1]);
+        }
+        if (tid == 0) IX_TRACE(6, (int)gb);
+        if (QT > 1 && 2 * qp + 1 < w.nqt && sidx < Et[1]) a.scores[srow[1] + sidx] = sc1;
       }
-      tc::tc_fence_before();
-      tc::mbar_arrive(&s.d_empty[buf]);
-      if (tid == 0) IX_TRACE(5, blk);
-      if (!two) continue;
-      const int sidx = e0 + blk * IX_BLK + 32 * quad + lane;
-      float sc0 = 0.f, sc1 = 0.f;
-      const float* w0 = s.w[QT > 1 ? 2 * qp : 0];
-      const float* w1 = s.w[QT > 1 ? 2 * qp + 1 : 0];
-#pragma unroll
-      for (int h = 0; h < 32; ++h) sc0 = fmaf(w0[h], fmaxf(d0[h], 0.f), sc0);
-#pragma unroll
-      for (int h = 0; h < 32; ++h) sc0 = fmaf(w0[32 + h], fmaxf(d1[h], 0.f), sc0);
-      if constexpr (QT > 1) {
-#pragma unroll
-        for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[h], fmaxf(d2[h], 0.f), sc1);
-#pragma unroll
-        for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[32 + h], fmaxf(d3[h], 0.f), sc1);
+      if constexpr (HIST) {
+        // add the unit's histograms to its rows' first histograms (int hist1[256] at the
+        // start of each row's top-k region) and clear them for the next unit
+        tc::named_barrier(1, 256);
+        for (int e = tid; e < QT * 256; e += 256) {
+          const int q = e >> 8, v = s.hist[q][e & 255];
+          if (v) {
+            atomicAdd(reinterpret_cast<int*>(a.cand + (long long)(w.qlo + q - a.score_q0) * a.cand_row_bytes) + (e & 255), v);
+            s.hist[q][e & 255] = 0;
+          }
+        }
       }
-      if (sidx < Et[0]) a.scores[srow[0] + sidx] = sc0;
-      if constexpr (HIST) {                      // first histogram of the threshold top-k
-        hist_add(s.hist[QT > 1 ? 2 * qp : 0], score_key(sc0) >> 24, sidx < Et[0]);
-        if (QT > 1) hist_add(s.hist[QT > 1 ? 2 * qp + 1 : 0], score_key(sc1) >> 24, 2 * qp + 1 < nqt && sidx < Et[1]);
-      }
-      if (tid == 0) IX_TRACE(6, blk);
-      if (QT > 1 && 2 * qp + 1 < nqt && sidx < Et[1]) a.scores[srow[1] + sidx] = sc1;
     }
   }
   tc::tc_fence_before();
@@ -260,14 +360,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   if (warp == 9) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, IX_TM_COLS);
-  }
-  if constexpr (HIST) {
-    // add the tile's histograms to the rows' first histograms (int hist1[256] at the start
-    // of each row's top-k region)
-    for (int e = tid; e < nqt * 256; e += blockDim.x) {
-      const int u = e >> 8, v = s.hist[u][e & 255];
-      if (v) atomicAdd(reinterpret_cast<int*>(a.cand + (long long)(qlo + u - a.score_q0) * a.cand_row_bytes) + (e & 255), v);
-    }
   }
 }
 
@@ -298,13 +390,27 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
   const int tps = (a.nq + qt - 1) / qt;
   auto tile_of = [&](int qg) { return (qg / a.nq) * tps + (qg % a.nq) / qt; };
   const int t0 = tile_of(q_begin), t1 = tile_of(q_begin + q_count - 1);
-  // Long rows with few query tiles (decode): larger entry chunks per CTA amortise its setup
-  // (Q tile, TMEM, pipeline fill) while keeping at least 4 CTAs per SM of work.
-  int chunk = IX_CHUNK;
+  // Work units (tile, chunk of entries); one persistent CTA per SM walks them.
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      sms = 148;
+  }
+  // Prefill tiles (several queries): persistent CTAs, one per SM, walk units of IX_CHUNK
+  // entries (per-tile CTAs paid their setup and pipeline fill on only a few key blocks).
+  // One-query tiles (decode over long rows of very different lengths): one CTA per unit, so
+  // that the hardware hands units to SMs as they free up (a static walk balanced them worse);
+  // units grow to 16384 entries while there are at least 4 per SM.
   const long long tiles = t1 - t0 + 1;
-  while (chunk < 4 * IX_CHUNK && tiles * ((max_e + 2 * chunk - 1) / (2 * chunk)) >= 4 * 148) chunk *= 2;
-  dim3 grid((unsigned)tiles, (max_e + chunk - 1) / chunk);
-  if (grid.y > 65535) return DSV4_OK;
+  int chunk = IX_CHUNK;
+  if (qt == 1)
+    while (chunk < 4 * IX_CHUNK && tiles * ((max_e + 2 * chunk - 1) / (2 * chunk)) >= 4 * sms) chunk *= 2;
+  const long long nchunk = (max_e + chunk - 1) / chunk;
+  const long long units = tiles * nchunk;
+  if (units >= (1ll << 31)) return DSV4_OK;
+  const unsigned grid = (unsigned)(qt == 1 || units < sms ? units : sms);
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<IX_QT, IX_STAGES, false>,
@@ -326,17 +432,17 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
   if (qt == 1) {
     if (a.topk_pipe)
       index_tc_kernel<1, 6, true><<<grid, IX_THREADS, ix_smem<1, 6, true>(), st>>>(a, mq, mk, q_begin, q_count,
-                                                                                 t0, tps, chunk, sp);
+                                                                                 t0, tps, chunk, (int)tiles, (int)units, sp);
     else
       index_tc_kernel<1, 6, false><<<grid, IX_THREADS, ix_smem<1, 6, false>(), st>>>(a, mq, mk, q_begin, q_count,
-                                                                                   t0, tps, chunk, sp);
+                                                                                   t0, tps, chunk, (int)tiles, (int)units, sp);
   } else {
     if (a.topk_pipe)
       index_tc_kernel<IX_QT, IX_STAGES, true><<<grid, IX_THREADS, ix_smem<IX_QT, IX_STAGES, true>(), st>>>(
-          a, mq, mk, q_begin, q_count, t0, tps, chunk, sp);
+          a, mq, mk, q_begin, q_count, t0, tps, chunk, (int)tiles, (int)units, sp);
     else
       index_tc_kernel<IX_QT, IX_STAGES, false><<<grid, IX_THREADS, ix_smem<IX_QT, IX_STAGES, false>(), st>>>(
-          a, mq, mk, q_begin, q_count, t0, tps, chunk, sp);
+          a, mq, mk, q_begin, q_count, t0, tps, chunk, (int)tiles, (int)units, sp);
   }
   *used = true;
   return launch_status("index scores (tensor cores)");
