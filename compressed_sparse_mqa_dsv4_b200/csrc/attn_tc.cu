@@ -850,7 +850,9 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   if (nsplit > 1)
     a.part_ml = reinterpret_cast<float2*>(a.part_o + items * nsplit * AT_H * (long long)AT_C);
   const long long work = items * nsplit;
-  const long long grid = work < sms ? work : sms;
+  // split lists (decode): one CTA per work item, so that the hardware hands items of very
+  // different lengths to SMs as they free up; unsplit lists: persistent, one CTA per SM
+  const long long grid = (nsplit > 1 || work < sms) ? work : sms;
   if (nsplit > 1)
     attn_tc_kernel<true><<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(
         a, mq, mlocal, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
