@@ -200,13 +200,14 @@ class Generator:
 
         visible: int tensor [Q] -- how many entries each query may choose from (the
         caller computes it). For each query, draws a uniformly random subset of size
-        min(k, visible) of [0, visible), in random order, padded with -1.
-        Returns (idx int32 [Q, k], counts int32 [Q]).
+        min(k, visible) of [0, visible), in random order, padded with -1, on the
+        generator's device. Returns (idx int32 [Q, k], counts int32 [Q]).
         """
-        visible = visible.to(torch.int64).reshape(-1)
+        dev = self.device
+        visible = visible.to(torch.int64).reshape(-1).to(dev)
         Qn = visible.numel()
-        idx = torch.full((Qn, k), -1, dtype=torch.int32)
-        counts = torch.minimum(visible, torch.tensor(k)).to(torch.int32)
+        idx = torch.full((Qn, k), -1, dtype=torch.int32, device=dev)
+        counts = torch.minimum(visible, torch.tensor(k, device=dev)).to(torch.int32)
         if k == 0 or Qn == 0:
             return idx, counts
         emax = int(visible.max().item()) if Qn else 0
@@ -216,11 +217,11 @@ class Generator:
         chunk = max(1, (1 << 24) // max(emax, 1))
         for q0 in range(0, Qn, chunk):
             q1 = min(Qn, q0 + chunk)
-            r = torch.rand(q1 - q0, emax, generator=g)
-            cols = torch.arange(emax).unsqueeze(0)
+            r = torch.rand(q1 - q0, emax, generator=g, device=dev)
+            cols = torch.arange(emax, device=dev).unsqueeze(0)
             r = torch.where(cols < visible[q0:q1].unsqueeze(1), r, torch.full_like(r, 2.0))
             kk = min(k, emax)
             order = torch.argsort(r, dim=1)[:, :kk].to(torch.int32)
-            keep = torch.arange(kk).unsqueeze(0) < counts[q0:q1].unsqueeze(1)
+            keep = torch.arange(kk, device=dev).unsqueeze(0) < counts[q0:q1].unsqueeze(1)
             idx[q0:q1, :kk] = torch.where(keep, order, torch.full_like(order, -1))
         return idx, counts
