@@ -164,3 +164,33 @@ def test_decode_attention_full_sampled(dsv4, kind):
             1 / math.sqrt(c), dense_m=m if kind == "hca" else 0, queries=[(0, 0)])
         assert_close(Og[b, 0].float().cpu(), Or[0], "bf16", f"decode {kind} b={b} O")
         assert_close(Lg[b, 0].float().cpu(), Lr[0], "bf16", f"decode {kind} b={b} LSE")
+
+
+def test_index_pro_fp4_full_sampled(dsv4):
+    """V4-Pro indexer at full size: 131072 queries over up to 32768 entries, k=1024, FP4
+    operands. The device quantises q^I and K^I with dsv4_quantize_fp4 and scores them through
+    the benchmark's call and workspace; the oracle quantises the same bf16 rows with its own
+    quantiser and scores the dequantised values in fp64 for sampled queries."""
+    s = preset("pro_csa_prefill")
+    n, m, k, HI, cI = s.n, s.m, s.k, s.H_I, s.c_I
+    E = n // m
+    g = Generator(51, device="cuda")
+    qI, w = g.index_queries(s, n)
+    KI = g.index_keys(s, E)
+    qc, qs = dsv4.dsv4_quantize_fp4(qI.reshape(-1, cI))
+    kc, ks = dsv4.dsv4_quantize_fp4(KI)
+    ws = torch.empty(dsv4.dsv4_index_topk_workspace_size_ex(dsv4.FP4, 1, n, HI, cI, E, k, E),
+                     dtype=torch.uint8, device="cuda")
+    zero64 = torch.zeros(1, dtype=torch.int64, device="cuda")
+    zero32 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx, counts = dsv4.dsv4_index_topk(qc.view(1, n, HI, cI // 2), w, kc, zero64, zero32, m, k, E,
+                                       qI_scales=qs, KI_scales=ks, c_I=cI, workspace=ws)
+    dsv4.dsv4_check_errors()
+    idx, counts = idx.cpu().numpy(), counts.cpu().numpy()
+    kc64, ks64 = O.quantize_fp4(KI.float().cpu())
+    KI64 = O.dequantize_fp4(kc64, ks64, cI)
+    for t in sample_positions(n, m, extra=[4 * k - 1, 4 * k, 4 * 16384 + 3, n - 1], count=4):
+        qct, qst = O.quantize_fp4(qI[0, t].float().cpu())
+        q64 = O.dequantize_fp4(qct, qst, cI)
+        s64 = O.index_scores_query(q64, w[0, t].cpu(), KI64, t, m)
+        check_topk_query(idx[0, t], counts[0, t], s64, k, what=f"pro fp4 index t={t}")
