@@ -202,6 +202,63 @@ __device__ __forceinline__ void select_topk(const float* sc, int n, int keff, To
   }
 }
 
+// Rows of at most R * NT entries: each thread holds its contiguous run of R keys in
+// registers for all four radix passes and the ordered compaction (the loop over global
+// loads re-read every key once per pass, one dependent load at a time).
+template <int NT, int R, typename Emit>
+__device__ __forceinline__ void select_topk_regs(const float* sc, int n, int keff, TopkShared& sh,
+                                                 Emit emit) {
+  int* hist = sh.hist;
+  const int per = (n + NT - 1) / NT;              // <= R
+  const int lo = threadIdx.x * per, hi = min(n, lo + per);
+  uint32_t key[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) key[r] = (r < hi - lo) ? score_key(__ldg(sc + lo + r)) : 0u;
+  const int cnt = max(0, hi - lo);
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = keff;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    if (threadIdx.x < 256) hist[threadIdx.x] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      if (r < cnt && (key[r] & pmask) == prefix) atomicAdd(&hist[(key[r] >> shift) & 255u], 1);
+    __syncthreads();
+    const int d = 255 - (int)threadIdx.x;
+    const int h = d >= 0 ? hist[d] : 0;
+    int tot;
+    const int above = block_exclusive_scan<NT>(h, sh.warp_tot, tot);
+    if (d >= 0 && above < remaining && remaining <= above + h) {
+      sh.sel = d;
+      sh.above = above;
+    }
+    __syncthreads();
+    remaining -= sh.above;
+    prefix |= (uint32_t)sh.sel << shift;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;
+  int n_gt = 0, n_eq = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    n_gt += r < cnt && key[r] > T;
+    n_eq += r < cnt && key[r] == T;
+  }
+  int tot;
+  const int eq_before = block_exclusive_scan<NT>(n_eq, sh.warp_tot, tot);
+  const int take_eq = max(0, min(n_eq, remaining - eq_before));
+  int pos = block_exclusive_scan<NT>(n_gt + take_eq, sh.warp_tot, tot), eq_seen = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    if (r < cnt && (key[r] > T || (key[r] == T && eq_seen++ < take_eq))) {
+      if (pos < keff) emit(pos, lo + r);
+      ++pos;
+    }
+  }
+}
+
 // Single stage: one CTA per query.
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_kernel(IndexArgs a, int q_begin) {
@@ -220,7 +277,11 @@ __global__ void __launch_bounds__(NT) topk_kernel(IndexArgs a, int q_begin) {
     return;
   }
   const float* sc = a.scores + (long long)(qg - a.score_q0) * a.scores_ld;
-  select_topk<NT, NT == 256>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; });
+  auto emit = [&](int p, int j) { out[p] = j; };
+  if (NT == 256 && Et <= 8 * NT)
+    select_topk_regs<NT, 8>(sc, Et, keff, sh, emit);
+  else
+    select_topk<NT, NT == 256>(sc, Et, keff, sh, emit);
 }
 
 // ---------------------------------------------------------------- segments + merge
