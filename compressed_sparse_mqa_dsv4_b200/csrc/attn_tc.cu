@@ -54,6 +54,7 @@ constexpr uint32_t GATE_PAIR0 = 6;          // 6..9: chunk pairs 0..3
 constexpr uint32_t TM_S = 0;
 constexpr uint32_t TM_O = 64;
 constexpr uint32_t TM_COLS = 512;
+constexpr int AT_ORDER_MAX = 256;            // split lists ranked longest first up to this many
 constexpr float TAU = 8.f;                  // log2-domain growth tolerated before rescaling
 constexpr float LOG2E = 1.4426950408889634f;
 constexpr float LN2 = 0.6931471805599453f;
@@ -74,6 +75,8 @@ struct AttnSmem {
   uint64_t s_full, p_full, o_done, drain;
   uint32_t tmem_base;
   int abort;
+  int first;                                // split lists: this CTA's work item
+  int order_nb[AT_ORDER_MAX];               // split lists: blocks per (query, head group)
 };
 constexpr size_t AT_SMEM = sizeof(AttnSmem) + 1024;
 static_assert(AT_SMEM <= 232448, "shared memory of the attention kernel");
@@ -241,6 +244,30 @@ __global__ void __maxnreg__(128)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = s.tmem_base;
+  // Split lists run one CTA per work item and the hardware dispatches CTAs in index order,
+  // so CTA r*nsplit + sp takes split sp of the list ranked r by length (longest first, ties
+  // by position): long lists start in the first wave and short ones fill the tail, as in
+  // longest-processing-time-first scheduling.
+  int first = blockIdx.x;
+  if constexpr (kSplit) {
+    const int nbase = items / a.nsplit;
+    if (nbase <= AT_ORDER_MAX) {
+      for (int t = tid; t < nbase; t += AT_THREADS) s.order_nb[t] = item_info<false>(a, t, head_groups).nb;
+      __syncthreads();
+      const int r = blockIdx.x / a.nsplit;
+      for (int t = tid; t < nbase; t += AT_THREADS) {
+        const int v = s.order_nb[t];
+        int rank = 0;
+        for (int j = 0; j < nbase; ++j) {
+          const int u = s.order_nb[j];
+          rank += (u > v || (u == v && j < t)) ? 1 : 0;
+        }
+        if (rank == r) s.first = t * a.nsplit + blockIdx.x % a.nsplit;
+      }
+      __syncthreads();
+      first = s.first;
+    }
+  }
 
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer (4 warps)
@@ -251,7 +278,7 @@ __global__ void __maxnreg__(128)
     int k = 0;
     bool ok = true;
     if (pt == 0) tc::prefetch_tensormap(&map_q);
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+    for (int item = first; item < items && ok; item += gridDim.x) {
       const ItemInfo it = item_info<kSplit>(a, item, head_groups);
       if (kSplit && it.je <= it.jb) continue;          // a split without blocks: no work
       ok = !gate(GATE_ITEM, false);                    // the Q buffer is free (or abort)
@@ -359,7 +386,7 @@ __global__ void __maxnreg__(128)
     uint32_t G = 0;
     int k = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+    for (int item = first; item < items && ok; item += gridDim.x) {
       const ItemInfo it = item_info<kSplit>(a, item, head_groups);
       if (kSplit && it.je <= it.jb) continue;
       if (k > 0) ok = wwait(&s.q_empty, (uint32_t)((k - 1) & 1));
@@ -393,7 +420,7 @@ __global__ void __maxnreg__(128)
       uint32_t G = 0;
       int k = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
+      for (int item = first; item < items && ok; item += gridDim.x) {
         const ItemInfo it = item_info<kSplit>(a, item, head_groups);
         if (kSplit && it.je <= it.jb) continue;
         ok = wwait(&s.q_full, (uint32_t)(k & 1));
@@ -453,7 +480,7 @@ __global__ void __maxnreg__(128)
     // The item's description, its sink logit and the validity of this thread's slot in the
     // next block are loaded one step ahead (global loads queue behind the producers' gather
     // traffic, so their latency is long).
-    int item = blockIdx.x;
+    int item = first;
     ItemInfo it = item_info<kSplit>(a, item < items ? item : 0, head_groups);
     float sink_h = (quad == 0 && a.sink) ? __ldg(a.sink + it.hg * AT_H + hb + lane) : 0.f;
     bool vnext = item < items && it.je > it.jb && slot_row(a, it.cs, it.nc4, it.jb * AT_BLK + slot).valid;
@@ -823,13 +850,15 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   s = encode_tensor_map_2d(&mlocal, a.local, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_local,
                            64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
-  // Few (query, head group) items: split each candidate list so that about two work items
-  // per SM exist, as far as the caller's workspace (a.nsplit = its capacity) allows.
+  // Few (query, head group) items: split each candidate list so that about one and a half
+  // work items per SM exist, as far as the caller's workspace (a.nsplit = its capacity)
+  // allows (measured on 64 dense decode lists of 9-65 blocks: 4 splits 138 us, 5 splits
+  // 151 us, 8 splits 156 us; each split pays its own Q load, setup and partial write).
   // A selected list has at most round4(k) + round4(w) candidates; a split must keep at least
-  // 4 blocks to pay for its own Q load, setup and partial write.
+  // 4 blocks.
   int nsplit = 1;
   if (a.part_o && a.nsplit > 1 && items < sms) {
-    nsplit = (int)((2 * sms + items - 1) / items);
+    nsplit = (int)((3 * sms / 2 + items - 1) / items);
     if (nsplit > a.nsplit) nsplit = a.nsplit;
     if (a.idx) {
       const int nb_max = (((a.k + 3) & ~3) + ((a.w + 3) & ~3) + AT_BLK - 1) / AT_BLK;
@@ -849,6 +878,7 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   }
   if (nsplit > 1)
     a.part_ml = reinterpret_cast<float2*>(a.part_o + items * nsplit * AT_H * (long long)AT_C);
+
   const long long work = items * nsplit;
   // split lists (decode): one CTA per work item, so that the hardware hands items of very
   // different lengths to SMs as they free up; unsplit lists: persistent, one CTA per SM
