@@ -275,9 +275,15 @@ def test_topk_brute_force(E, k):
 
 
 def test_topk_ties_prefer_lower_index():
+    """Equal scores across the k-th place: the lower entries are taken."""
     s = np.array([1.0, 3.0, 3.0, 2.0, 3.0, 0.5])
     idx, cnt = O.topk_select(s, 4)
     assert idx.tolist() == [1, 2, 3, 4] and cnt == 4
+    s = np.array([1.0, 3.0, 2.0, 3.0, 2.0, 0.5, 2.0])     # three 2.0s compete for one place
+    idx, cnt = O.topk_select(s, 3)
+    assert idx.tolist() == [1, 2, 3] and cnt == 3
+    idx, cnt = O.topk_select(np.full(9, 0.25), 4)          # all tied
+    assert idx.tolist() == [0, 1, 2, 3] and cnt == 4
 
 
 def test_index_topk_brute_force_tiny():
