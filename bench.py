@@ -40,6 +40,24 @@ ATTN_TRAFFIC = {"sources_sha1": "248722e89d10cce437e3ab7ed32df08169c2a504",
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc.cu", "dsv4_common.cuh", "tc_common.cuh")
 
 
+def max_over_ranks(value: float, world: int, device) -> float:
+    """The largest of the ranks' values (per-rank device times -> the job's time); the value
+    itself on one rank. Every rank calls it at the same point."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, max_ms: float) -> float:
+    """Units all ranks processed (the same number on each: weak scaling) per second of the
+    slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 def _attn_sources_sha1() -> str:
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "compressed_sparse_mqa_dsv4_b200", "csrc")
@@ -215,14 +233,9 @@ def run_cuda(args, rank: int, world: int):
     comp_ms = [r[0].elapsed_time(r[1]) for r in recs]
     index_ms = [r[1].elapsed_time(r[2]) for r in recs]
     attn_ms = [r[2].elapsed_time(r[3]) for r in recs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
-    tokens = s.B * s.n * args.steps * world
-    value = tokens / (total_ms / 1e3)
+    value = job_throughput(s.B * s.n * args.steps, world, total_ms)
 
     # ---- end to end through the C ABI with host buffers (pinned), copies inside the region
     pinned = {k: v.pin_memory() for k, v in host.items()}
@@ -250,12 +263,8 @@ def run_cuda(args, rank: int, world: int):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = s.B * s.n * e2e_steps * world / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = job_throughput(s.B * s.n * e2e_steps, world, e2e_ms)
 
     # ---- roofline of the dominant kernel (attention, tensor-core bound by algorithm)
     peaks, peak_src = _peaks()
