@@ -20,6 +20,8 @@ Sources (page title, then section / equation):
       s5.1 local window L_t = {max(0,t-w+1)..t} and ONE candidate list / softmax
       s5.2 logit scaled by 1/sqrt(c)
       s5.3 sink logit z'_h in the denominator only
+      s7  incremental decode state machine (local ring slot per token, bounded
+          compressor tail, entry emitted when (t+1) is a multiple of the ratio)
       s8  precision table (MXFP4 indexer operands)
   [PR-MASK] huggingface/transformers PR #45892 discussion: [S, S*top_k] gathered
       mask vs [S, compressed_len] scatter mask give identical attention.
@@ -345,6 +347,51 @@ def dequantize_fp4(codes, scales, cols: int) -> np.ndarray:
     t4 = e4m3_values()
     s = t4[scales.astype(np.int64) & 0x7F]
     return val * np.repeat(s, 16, axis=1)
+
+
+# ----------------------------------------------------------------------------- [CSA-DEF] s7
+
+
+def tail_slots(m: int, overlap: bool) -> int:
+    """Rows of the bounded compressor tail ([CSA-DEF] s7 state table): the current block,
+    plus for CSA the preceding block, whose stream-b half the next entry pools."""
+    return 2 * m if overlap else m
+
+
+def decode_append(tail, C_row, Z_row, bias, t: int, m: int, overlap: bool):
+    """One token of the compressor state machine ([CSA-DEF] s7, steps 2-4).
+
+    tail  float64 [T, 2, S*c], T = tail_slots(m, overlap): slot p mod T holds the C row
+          (tail[., 0]) and the Z row (tail[., 1]) of position p. Position t's rows are
+          written in place.
+    Returns the completed entry [c] when t + 1 is a multiple of m (it is entry
+    (t+1)/m - 1 and is eligible for the block's final token), else None: an incomplete
+    block exposes no entry. The entry is the s2.1 / s2.2 softmax over the block's
+    positions (stream a, bias[0]) and, for CSA after the first block, the preceding
+    block's positions (stream b, bias[1]).
+    """
+    T = tail.shape[0]
+    tail[t % T, 0] = as_f64(C_row)
+    tail[t % T, 1] = as_f64(Z_row)
+    if (t + 1) % m != 0:
+        return None
+    i = (t + 1) // m - 1
+    width = tail.shape[2]
+    c = width // 2 if overlap else width
+    bias = as_f64(bias)
+    pooled = [(m * i + p, 0, bias[0][p]) for p in range(m)]
+    if overlap and i > 0:
+        pooled += [(m * (i - 1) + p, 1, bias[1][p]) for p in range(m)]
+    logits = np.stack([tail[pos % T, 1, half * c:(half + 1) * c] + b for pos, half, b in pooled])
+    values = np.stack([tail[pos % T, 0, half * c:(half + 1) * c] for pos, half, _ in pooled])
+    top = logits.max(axis=0)
+    e = np.exp(logits - top)
+    return (e * values).sum(axis=0) / e.sum(axis=0)
+
+
+def ring_write(local, kv_row, t: int) -> None:
+    """[CSA-DEF] s7 step 1: the token's shared-KV entry overwrites ring slot t mod R."""
+    local[t % local.shape[0]] = as_f64(kv_row)
 
 
 # ----------------------------------------------------------------------------- layer chains

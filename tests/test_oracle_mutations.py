@@ -52,6 +52,12 @@ SLIPS = {
         ("loc = local_window(t, w) % R", "loc = (local_window(t, w) + 1) % R"),
     "attention: HCA dense read one entry too many":
         ("comp = np.arange(completed_entries(t, dense_m))", "comp = np.arange(completed_entries(t, dense_m) + 1)"),
+    "decode: entry emitted one token early":
+        ("if (t + 1) % m != 0:\n        return None", "if t % m != 0:\n        return None"),
+    "decode: preceding block read from stream a":
+        ("pooled += [(m * (i - 1) + p, 1, bias[1][p])", "pooled += [(m * (i - 1) + p, 0, bias[1][p])"),
+    "decode: ring slot off by one":
+        ("local[t % local.shape[0]] = as_f64(kv_row)", "local[(t + 1) % local.shape[0]] = as_f64(kv_row)"),
     "fp4: E4M3 exponent bias 8":
         ("vals.append((1.0 + mant / 8.0) * 2.0 ** (e - 7))", "vals.append((1.0 + mant / 8.0) * 2.0 ** (e - 8))"),
     "fp4: e2m1 subnormal 0.25":

@@ -480,6 +480,68 @@ def test_window_only_for_queries_before_first_entry():
         np.testing.assert_allclose(o[0, t], ref, rtol=1e-15)
 
 
+# ----------------------------------------------------------------------------- decode state
+
+
+@pytest.mark.parametrize("overlap,m,n", [(True, 4, 37), (True, 1, 5), (False, 16, 50), (False, 3, 11)])
+def test_decode_state_machine_reproduces_the_compressor(overlap, m, n):
+    """[CSA-DEF] s7: feeding tokens one at a time through the bounded tail emits, at
+    exactly the tokens whose t + 1 is a multiple of m, the entries the s2.1/s2.2
+    compressor pools from the whole stream (a trailing partial block emits nothing)."""
+    rng = _rng(40 + m)
+    S, c = (2 if overlap else 1), 5
+    C = rng.standard_normal((1, n, S * c))
+    Z = rng.standard_normal((1, n, S * c))
+    bias = 0.1 * rng.standard_normal((S, m, c))
+    want = O.compress(C, Z, bias, m, overlap)[0]
+    tail = np.zeros((O.tail_slots(m, overlap), 2, S * c))
+    got = {}
+    for t in range(n):
+        e = O.decode_append(tail, C[0, t], Z[0, t], bias, t, m, overlap)
+        if e is not None:
+            got[t] = e
+    assert sorted(got) == [m * (i + 1) - 1 for i in range(n // m)]
+    for t, e in got.items():
+        np.testing.assert_allclose(e, want[(t + 1) // m - 1], rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("overlap,m", [(True, 4), (False, 8)])
+def test_decode_tail_restored_from_a_prefix(overlap, m):
+    """An incomplete prefix tail restored from the prefix's last T positions (slot p mod T)
+    continues exactly like the uninterrupted stream; the state is T rows whatever n is."""
+    rng = _rng(50 + m)
+    S, c, n0, n = (2 if overlap else 1), 3, 4 * m + 2, 7 * m + 1
+    C = rng.standard_normal((1, n, S * c))
+    Z = rng.standard_normal((1, n, S * c))
+    bias = 0.1 * rng.standard_normal((S, m, c))
+    want = O.compress(C, Z, bias, m, overlap)[0]
+    T = O.tail_slots(m, overlap)
+    tail = np.full((T, 2, S * c), np.nan)              # anything not restored must not be read
+    for p in range(n0 - T, n0):
+        tail[p % T, 0], tail[p % T, 1] = C[0, p], Z[0, p]
+    for t in range(n0, n):
+        e = O.decode_append(tail, C[0, t], Z[0, t], bias, t, m, overlap)
+        assert (e is not None) == ((t + 1) % m == 0)
+        if e is not None:
+            np.testing.assert_allclose(e, want[(t + 1) // m - 1], rtol=1e-13, atol=1e-15)
+    assert tail.shape[0] == T
+
+
+def test_ring_write_keeps_the_window():
+    """s7 step 1 into an R-slot ring (R >= w): after token t the ring holds tokens
+    t-R+1..t, so the window read through slots j mod R returns tokens max(0,t-w+1)..t."""
+    rng = _rng(60)
+    n, c, w, R = 23, 4, 5, 7
+    kv = rng.standard_normal((n, c))
+    ring = np.zeros((R, c))
+    for t in range(n):
+        O.ring_write(ring, kv[t], t)
+        win = O.local_window(t, w)
+        np.testing.assert_array_equal(ring[win % R], kv[win])
+        held = np.arange(max(0, t - R + 1), t + 1)
+        np.testing.assert_array_equal(ring[held % R], kv[held])
+
+
 # ----------------------------------------------------------------------------- FP4
 
 
