@@ -18,7 +18,8 @@ import torch
 
 __all__ = [
     "DSV4Error", "lib", "LIB_PATH", "F32", "BF16", "FP4",
-    "dsv4_compress", "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
+    "dsv4_compress", "dsv4_compress_decode", "dsv4_ring_write", "decode_tail_shape",
+    "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
     "dsv4_index_topk_workspace_size_ex",
     "dsv4_hybrid_sparse_attn", "dsv4_hybrid_sparse_attn_workspace_size", "dsv4_check_errors",
 ]
@@ -42,6 +43,10 @@ lib.dsv4_check_errors.restype = _I
 lib.dsv4_check_errors.argtypes = [_P]
 lib.dsv4_compress.restype = _I
 lib.dsv4_compress.argtypes = [_I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]
+lib.dsv4_compress_decode.restype = _I
+lib.dsv4_compress_decode.argtypes = [_I, _P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _I, _I, _P]
+lib.dsv4_ring_write.restype = _I
+lib.dsv4_ring_write.argtypes = [_I, _P, _P, _I, _P, _I, _I, _P]
 lib.dsv4_quantize_fp4.restype = _I
 lib.dsv4_quantize_fp4.argtypes = [_P, _P, _P, _L, _I, _P]
 lib.dsv4_index_topk_workspace_size.restype = _S
@@ -111,6 +116,44 @@ def dsv4_compress(C: torch.Tensor, Z: torch.Tensor, bias: torch.Tensor, m: int, 
     _check(lib.dsv4_compress(_code(C.dtype), _ptr(C), _ptr(Z), _ptr(bias), _ptr(out), B, n, c, m,
                              1 if overlap else 0, _stream(stream)), "dsv4_compress")
     return out
+
+
+def decode_tail_shape(B: int, c: int, m: int, overlap: bool):
+    """Shape of the compressor tail state of dsv4_compress_decode: [B, S*m, 2, S*c]."""
+    S = 2 if overlap else 1
+    return (B, S * m, 2, S * c)
+
+
+def dsv4_compress_decode(C_new: torch.Tensor, Z_new: torch.Tensor, bias: torch.Tensor,
+                         tail: torch.Tensor, pool: torch.Tensor, pool_row_off: torch.Tensor,
+                         pos: torch.Tensor, m: int, overlap: bool, stream=None) -> None:
+    """One decode token per sequence: C_new, Z_new [B, S*c] into the tail
+    [B, S*m, 2, S*c]; completed entries are written to pool [rows, c] in place."""
+    _dev(C_new, "C_new"), _dev(Z_new, "Z_new", C_new.dtype), _dev(bias, "bias", torch.float32)
+    B, width = C_new.shape
+    S = 2 if overlap else 1
+    c = width // S
+    _dev(tail, "tail", C_new.dtype), _dev(pool, "pool", C_new.dtype)
+    _dev(pool_row_off, "pool_row_off", torch.int64), _dev(pos, "pos", torch.int32)
+    if tuple(tail.shape) != decode_tail_shape(B, c, m, overlap):
+        raise ValueError(f"tail must be {decode_tail_shape(B, c, m, overlap)}, got {tuple(tail.shape)}")
+    if pool.shape[-1] != c:
+        raise ValueError(f"pool rows must have {c} channels")
+    _check(lib.dsv4_compress_decode(_code(C_new.dtype), _ptr(C_new), _ptr(Z_new), _ptr(bias),
+                                    _ptr(tail), _ptr(pool), _ptr(pool_row_off),
+                                    pool.numel() // c, _ptr(pos), B, c, m, 1 if overlap else 0,
+                                    _stream(stream)), "dsv4_compress_decode")
+
+
+def dsv4_ring_write(kv_new: torch.Tensor, local: torch.Tensor, pos: torch.Tensor,
+                    stream=None) -> None:
+    """kv_new [B, c] into slot pos[b] mod R of local [B, R, c], in place."""
+    _dev(kv_new, "kv_new"), _dev(local, "local", kv_new.dtype), _dev(pos, "pos", torch.int32)
+    B, c = kv_new.shape
+    if local.shape[0] != B or local.shape[2] != c:
+        raise ValueError(f"local must be [{B}, R, {c}]")
+    _check(lib.dsv4_ring_write(_code(kv_new.dtype), _ptr(kv_new), _ptr(local), local.shape[1],
+                               _ptr(pos), B, c, _stream(stream)), "dsv4_ring_write")
 
 
 def dsv4_quantize_fp4(x: torch.Tensor, codes: Optional[torch.Tensor] = None,

@@ -1,0 +1,128 @@
+// Incremental decode state ("CSA And HCA: Definition, State, And Cost Model", s7): per new
+// token of every sequence, the local shared-KV ring slot write (step 1) and the compressor
+// state machine (steps 2-4): the token's (C, Z) rows go to a bounded tail, and when t + 1
+// is a multiple of the ratio m the completed entry (s2.1 / s2.2) is appended to the pool.
+//
+// The tail of a sequence holds the rows of its last T = m (HCA) or 2m (CSA: the current
+// block plus the preceding block, whose stream-b half the next entry pools) positions,
+// position p in slot p mod T. One CTA per sequence; a thread owns channel ch of both
+// streams (columns ch and c + ch), so the rows it pools at an emission include the ones it
+// has just written itself and no other thread's. Per channel the arithmetic is the one of
+// the prefill compressor: an online softmax in fp32 over the preceding block's stream-b
+// positions, then the current block's stream-a positions, in position order.
+#include "dsv4_common.cuh"
+
+namespace dsv4 {
+
+template <typename T>
+__global__ void __launch_bounds__(256) compress_decode_kernel(
+    const T* __restrict__ C_new, const T* __restrict__ Z_new, const float* __restrict__ bias,
+    T* __restrict__ tail, T* __restrict__ pool, const int64_t* __restrict__ pool_row_off,
+    long long pool_rows, const int32_t* __restrict__ pos, int c, int m, int overlap) {
+  const int b = blockIdx.x;
+  const int S = overlap ? 2 : 1;
+  const int T_slots = S * m;
+  const long long width = (long long)S * c;
+  const int t = pos[b];
+  if (t < 0) {
+    if (threadIdx.x == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  T* tail_b = tail + (long long)b * T_slots * 2 * width;     // [T, 2, S*c]
+  // steps 2-3: the token's rows into slot t mod T
+  T* slot = tail_b + (long long)(t % T_slots) * 2 * width;
+  for (long long j = threadIdx.x; j < width; j += blockDim.x) {
+    slot[j] = C_new[(long long)b * width + j];
+    slot[width + j] = Z_new[(long long)b * width + j];
+  }
+  const long long t1 = (long long)t + 1;
+  if (t1 % m != 0) return;                                   // incomplete block: no entry
+  // step 4: entry i = (t+1)/m - 1 into pool row pool_row_off[b] + i
+  const long long i = t1 / m - 1;
+  const long long row = pool_row_off[b] + i;
+  const bool row_ok = pool_row_off[b] >= 0 && row < pool_rows;
+  if (!row_ok) {
+    if (threadIdx.x == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  for (int ch = threadIdx.x; ch < c; ch += blockDim.x) {
+    float mx = -INFINITY, den = 0.f, acc = 0.f;
+    for (int half = (overlap && i > 0) ? 1 : 0; half >= 0; --half) {
+      const long long tok0 = half ? m * (i - 1) : m * i;
+      for (int p = 0; p < m; ++p) {
+        const T* r = tail_b + ((tok0 + p) % T_slots) * 2 * width + half * c + ch;
+        float l = to_f32(r[width]) + bias[((long long)half * m + p) * c + ch];
+        float x = to_f32(r[0]);
+        if (l > mx) {
+          float e = expf(mx - l);
+          den = den * e + 1.f; acc = acc * e + x; mx = l;
+        } else {
+          float e = expf(l - mx);
+          den += e; acc = fmaf(e, x, acc);
+        }
+      }
+    }
+    pool[row * c + ch] = from_f32<T>(acc / den);
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) ring_write_kernel(const T* __restrict__ kv_new,
+                                                         T* __restrict__ local, int R,
+                                                         const int32_t* __restrict__ pos, int c) {
+  const int b = blockIdx.x;
+  const int t = pos[b];
+  if (t < 0) {
+    if (threadIdx.x == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  T* dst = local + ((long long)b * R + t % R) * c;
+  for (int j = threadIdx.x; j < c; j += blockDim.x) dst[j] = kv_new[(long long)b * c + j];
+}
+
+}  // namespace dsv4
+
+extern "C" int dsv4_compress_decode(int dtype, const void* C_new, const void* Z_new,
+                                    const float* bias, void* tail, void* pool,
+                                    const int64_t* pool_row_off, int64_t pool_rows,
+                                    const int32_t* pos, int B, int c, int m, int overlap,
+                                    void* stream) {
+  using namespace dsv4;
+  if (B < 0 || c < 1 || m < 1 || (overlap != 0 && overlap != 1) || pool_rows < 0)
+    return fail(DSV4_ERR_INVALID_ARG,
+                "dsv4_compress_decode: bad sizes B=%d c=%d m=%d overlap=%d pool_rows=%lld", B, c,
+                m, overlap, (long long)pool_rows);
+  if (B == 0) return DSV4_OK;
+  if (!C_new || !Z_new || !bias || !tail || !pool || !pool_row_off || !pos)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode: NULL pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dtype == DSV4_F32)
+    compress_decode_kernel<float><<<B, 256, 0, st>>>(
+        (const float*)C_new, (const float*)Z_new, bias, (float*)tail, (float*)pool, pool_row_off,
+        pool_rows, pos, c, m, overlap);
+  else if (dtype == DSV4_BF16)
+    compress_decode_kernel<__nv_bfloat16><<<B, 256, 0, st>>>(
+        (const __nv_bfloat16*)C_new, (const __nv_bfloat16*)Z_new, bias, (__nv_bfloat16*)tail,
+        (__nv_bfloat16*)pool, pool_row_off, pool_rows, pos, c, m, overlap);
+  else
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode: dtype %d not F32/BF16", dtype);
+  return launch_status("dsv4_compress_decode");
+}
+
+extern "C" int dsv4_ring_write(int dtype, const void* kv_new, void* local, int R,
+                               const int32_t* pos, int B, int c, void* stream) {
+  using namespace dsv4;
+  if (B < 0 || R < 1 || c < 1)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_ring_write: bad sizes B=%d R=%d c=%d", B, R, c);
+  if (B == 0) return DSV4_OK;
+  if (!kv_new || !local || !pos) return fail(DSV4_ERR_INVALID_ARG, "dsv4_ring_write: NULL pointer");
+  cudaStream_t st = (cudaStream_t)stream;
+  if (dtype == DSV4_F32)
+    ring_write_kernel<float><<<B, 256, 0, st>>>((const float*)kv_new, (float*)local, R, pos, c);
+  else if (dtype == DSV4_BF16)
+    ring_write_kernel<__nv_bfloat16><<<B, 256, 0, st>>>((const __nv_bfloat16*)kv_new,
+                                                        (__nv_bfloat16*)local, R, pos, c);
+  else
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_ring_write: dtype %d not F32/BF16", dtype);
+  return launch_status("dsv4_ring_write");
+}

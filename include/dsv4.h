@@ -87,6 +87,47 @@ int dsv4_compress(int dtype, const void* C, const void* Z, const float* bias, vo
                   int B, int n, int c, int m, int overlap, void* stream);
 
 /*
+ * dsv4_compress_decode -- one token of the compressor state machine of [CSA-DEF] s7
+ * (steps 2-4: update the compressor state; when t + 1 is a multiple of m, emit and append
+ * the completed entry) for each of B sequences. The emitted entry is the s2.1 (overlap = 1)
+ * or s2.2 (overlap = 0) entry dsv4_compress computes from the whole stream; an incomplete
+ * block exposes nothing.
+ *
+ *   dtype         DSV4_F32 or DSV4_BF16: element type of C_new, Z_new, tail and pool.
+ *   C_new, Z_new  [B, S*c], S = 1 + overlap: the new token's entry and gate rows (columns
+ *                 [0,c) stream a, [c,2c) stream b, as for dsv4_compress).
+ *   bias          fp32 [S, m, c].
+ *   tail          [B, T, 2, S*c], T = S*m, caller-owned state, updated in place: slot
+ *                 p mod T holds position p's C row ([., ., 0, .]) and Z row ([., ., 1, .]).
+ *                 Before the first call for a sequence whose prefix has n0 tokens, slots
+ *                 p mod T for p in [max(0, n0 - T), n0) hold the prefix's rows (nothing
+ *                 else is read; for n0 = 0 the tail needs no initialisation).
+ *   pool          [pool_rows, c]: sequence b's entry i is row pool_row_off[b] + i.
+ *   pos           int32 [B]: position t of each sequence's new token.
+ * Writes pool row pool_row_off[b] + (t+1)/m - 1 when (t + 1) % m == 0, so that attention
+ * of token t launched after this call sees the completed entry. Device-side errors
+ * (t < 0, a pool row outside [0, pool_rows)) skip the sequence and set
+ * DSV4_ERR_DEVICE_BOUNDS. Requires B >= 0, c >= 1, m >= 1, overlap in {0,1}; B == 0 is a
+ * no-op.
+ */
+int dsv4_compress_decode(int dtype, const void* C_new, const void* Z_new, const float* bias,
+                         void* tail, void* pool, const int64_t* pool_row_off, int64_t pool_rows,
+                         const int32_t* pos, int B, int c, int m, int overlap, void* stream);
+
+/*
+ * dsv4_ring_write -- [CSA-DEF] s7 step 1: each sequence's new shared-KV entry overwrites
+ * slot t mod R of its local ring (the layout dsv4_hybrid_sparse_attn reads: position j in
+ * slot j mod R).
+ *
+ *   dtype   DSV4_F32 or DSV4_BF16.
+ *   kv_new  [B, c]; local [B, R, c]; pos int32 [B] (t; t < 0 skips the sequence and sets
+ *           DSV4_ERR_DEVICE_BOUNDS).
+ * Requires B >= 0, R >= 1, c >= 1; B == 0 is a no-op.
+ */
+int dsv4_ring_write(int dtype, const void* kv_new, void* local, int R, const int32_t* pos,
+                    int B, int c, void* stream);
+
+/*
  * dsv4_quantize_fp4 -- FP4 indexer operands ([CSA-DEF] s3.1 and s8: the indexer Q/K are
  * multiplied in 4-bit floating point). Per group of 16 consecutive elements of a row:
  *   scale = RNE_E4M3(amax / 6) (fp32 quotient, saturating at 448);

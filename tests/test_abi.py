@@ -56,6 +56,14 @@ def test_host_validation_rejects_bad_arguments(lib):
     args = [1, P(16), P(16), ctypes.c_int64(4), P(16), None, None, 0, P(16), 8, P(16), 1, 1, 64,
             512, 4, 0, None, ctypes.c_float(1.0), P(16), None, None, ctypes.c_size_t(0), None]
     assert lib.dsv4_hybrid_sparse_attn(*args) == 1
+    # decode state: m = 0 rejected; B = 0 is a no-op; a ring of R = 0 slots rejected
+    lib.dsv4_compress_decode.restype = ctypes.c_int
+    assert lib.dsv4_compress_decode(1, P(16), P(16), P(16), P(16), P(16), P(16), ctypes.c_int64(4),
+                                    P(16), 1, 8, 0, 1, None) == 1
+    assert lib.dsv4_compress_decode(1, None, None, None, None, None, None, ctypes.c_int64(0), None,
+                                    0, 8, 4, 1, None) == 0
+    lib.dsv4_ring_write.restype = ctypes.c_int
+    assert lib.dsv4_ring_write(1, P(16), P(16), 0, P(16), 1, 8, None) == 1
     # index top-k: k above the supported maximum
     lib.dsv4_index_topk.restype = ctypes.c_int
     a = [1, P(16), None, P(16), P(16), None, ctypes.c_int64(1), P(16), P(16), 1, 1, 64, 128, 4,
