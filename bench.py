@@ -303,6 +303,11 @@ def run_cuda(args, rank: int, world: int):
     if args.layers:
         res["other_layers"] = {nm: run_layer(args, dev, stream, nm)
                                for nm in ("flash_hca_prefill", "pro_csa_prefill")}
+    if not args.no_decode:
+        try:                                          # last, so that it cannot cost the line
+            res["decode"]["state_update"] = run_decode_state(args, dev, stream)
+        except Exception as e:                        # noqa: BLE001
+            res["decode"]["state_update"] = {"error": str(e)[:300]}
     return res
 
 
@@ -394,6 +399,73 @@ def run_decode(args, dev, stream):
             "ms_per_step": round(ms, 4), "bytes_per_step": nbytes, "achieved_gbs": round(gbps, 1),
             "peak_gbs": peak, "frac": round(gbps / peak, 4), "peak_source": f"{src} hbm_gbs",
             "steps": steps, "l2": "flushed (256 MiB write) before every step"}
+
+
+def run_decode_state(args, dev, stream):
+    """Per-token state updates of the batched decode step ("CSA And HCA: Definition, State,
+    And Cost Model", s7 steps 1-4) for the same 64 sequences and 4 layers: the ring slot
+    write in every layer, the main and index-key compressor states of the CSA layers and the
+    main compressor state of the HCA layers, appending the entries that complete at this
+    token (L mod m == 0) to the pools. Timed apart from the decode step above."""
+    import torch
+    import compressed_sparse_mqa_dsv4_b200 as dsv4
+    from workloads import DECODE_BATCH as D
+    B, c, w, cI = D["B"], D["c"], D["w"], D["c_I"]
+    m4, m128 = D["m_csa"], D["m_hca"]
+    g = torch.Generator(device="cpu").manual_seed(args.seed + 1)
+    L = torch.randint(D["L_lo"], D["L_hi"] + 1, (B,), generator=g)
+    E4, E128 = (L // m4).tolist(), (L // m128).tolist()
+    off4 = torch.tensor([0] + torch.cumsum(torch.tensor(E4), 0)[:-1].tolist(), dtype=torch.int64,
+                        device=dev)
+    off128 = torch.tensor([0] + torch.cumsum(torch.tensor(E128), 0)[:-1].tolist(),
+                          dtype=torch.int64, device=dev)
+    pos = (L - 1).to(torch.int32).to(dev)
+    gd = torch.Generator(device=dev).manual_seed(args.seed + 4)
+
+    def normal(*shape):
+        return torch.empty(*shape, dtype=torch.bfloat16, device=dev).normal_(0.0, 1.0, generator=gd)
+
+    pool4, KI, pool128 = normal(sum(E4), c), normal(sum(E4), cI), normal(sum(E128), c)
+    local = normal(B, w, c)
+    tail4 = normal(*dsv4.decode_tail_shape(B, c, m4, True))
+    tailI = normal(*dsv4.decode_tail_shape(B, cI, m4, True))
+    tail128 = normal(*dsv4.decode_tail_shape(B, c, m128, False))
+    kv, C4, Z4 = normal(B, c), normal(B, 2 * c), normal(B, 2 * c)
+    CI, ZI, C128, Z128 = normal(B, 2 * cI), normal(B, 2 * cI), normal(B, c), normal(B, c)
+    b4 = torch.randn(2, m4, c, device=dev, generator=gd) * 0.1
+    bI = torch.randn(2, m4, cI, device=dev, generator=gd) * 0.1
+    b128 = torch.randn(1, m128, c, device=dev, generator=gd) * 0.1
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        for kind in D["layers"]:
+            dsv4.dsv4_ring_write(kv, local, pos)
+            if kind == "csa":
+                dsv4.dsv4_compress_decode(C4, Z4, b4, tail4, pool4, off4, pos, m4, True)
+                dsv4.dsv4_compress_decode(CI, ZI, bI, tailI, KI, off4, pos, m4, True)
+            else:
+                dsv4.dsv4_compress_decode(C128, Z128, b128, tail128, pool128, off128, pos, m128,
+                                          False)
+
+    for _ in range(3):
+        step()
+    dsv4.dsv4_check_errors()
+    ts = []
+    for _ in range(max(1, min(args.steps, 10))):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    dsv4.dsv4_check_errors()
+    launches = sum(3 if kind == "csa" else 2 for kind in D["layers"])
+    return {"what": "ring writes + compressor states of the 4 layers for one token of each of "
+                    f"the {B} sequences (entries completing at this token appended)",
+            "ms_per_step": round(statistics.median(ts), 4), "launches_per_step": launches,
+            "emitting_sequences": {"csa": int((L % m4 == 0).sum()), "hca": int((L % m128 == 0).sum())},
+            "steps": len(ts), "l2": "flushed (256 MiB write) before every step"}
 
 
 # ----------------------------------------------------------------------------- other layers
