@@ -22,7 +22,8 @@ Sources (page title, then section / equation):
       s5.3 sink logit z'_h in the denominator only
       s7  incremental decode state machine (local ring slot per token, bounded
           compressor tail, entry emitted when (t+1) is a multiple of the ratio)
-      s8  precision table (MXFP4 indexer operands)
+      s8  precision table (MXFP4 indexer operands; main KV entries of 448 FP8 + 64 bf16
+          RoPE channels, 576-byte payload) and the per-layer persistent-state table
   [PR-MASK] huggingface/transformers PR #45892 discussion: [S, S*top_k] gathered
       mask vs [S, compressed_len] scatter mask give identical attention.
   [PYPTO] pypto-lib PR #834: per-query compressed counts (cmp_counts).
@@ -42,6 +43,9 @@ Readings taken where the pages are silent (each is also listed in the design not
     from the fp32 quotient, saturating at +-6; a zero scale gives zero codes.
     The sign bit follows IEEE rounding (a negative value that rounds to zero is -0,
     code 0x8). Two codes per byte, element 2j in the low nibble.
+  * Main-KV FP8 entries: the RoPE channels are the last 64; the FP8 channels carry one
+    fp32 scale per 64 channels, scale = amax / 448 (the pages leave the scale metadata
+    open).
 """
 from __future__ import annotations
 
@@ -347,6 +351,65 @@ def dequantize_fp4(codes, scales, cols: int) -> np.ndarray:
     t4 = e4m3_values()
     s = t4[scales.astype(np.int64) & 0x7F]
     return val * np.repeat(s, 16, axis=1)
+
+
+# ----------------------------------------------------------------------------- main-KV cache entry ([CSA-DEF] s8)
+
+
+def main_kv_payload_bytes(c: int = 512, rope: int = 64) -> int:
+    """Payload of one production main (or local) KV entry ([CSA-DEF] s8 precision table):
+    the c - rope non-RoPE channels in FP8 (1 byte) and the rope RoPE channels in bf16."""
+    return (c - rope) * 1 + rope * 2
+
+
+def quantize_main_kv_fp8(x, rope: int = 64, group: int = 64):
+    """Production main-KV entry format ([CSA-DEF] s8): channels [0, c - rope) in FP8 E4M3,
+    channels [c - rope, c) (the RoPE part) kept in bf16.
+
+    The pages leave the FP8 scale metadata open; reading: one fp32 scale per `group`
+    consecutive FP8 channels, scale = fp32(amax / 448) (448 = the largest E4M3 value),
+    code = RNE_E4M3(fp32(x / scale)) saturating at 448, IEEE sign (a negative value that
+    rounds to zero keeps its sign), zero scale -> zero codes.
+    x: [rows, c], values taken as fp32 (bf16 inputs are exact).
+    Returns (codes uint8 [rows, c - rope] = sign << 7 | magnitude code,
+             scales float32 [rows, (c - rope) / group], rope float64 [rows, rope] (the bf16
+             value of each RoPE channel)).
+    """
+    x32 = np.asarray(as_f64(x), dtype=np.float32)
+    rows, c = x32.shape
+    nf = c - rope
+    assert nf % group == 0, "FP8 channels must split into whole groups"
+    g = x32[:, :nf].reshape(rows, nf // group, group)
+    amax = np.abs(g).max(axis=-1)
+    scale = (amax / np.float32(448.0)).astype(np.float32)               # fp32 division
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = (g / safe[..., None]).astype(np.float32)                          # fp32 division
+    t4 = e4m3_values()
+    mag = round_to_table(np.abs(q).astype(np.float64), t4)
+    code = mag | (np.signbit(q).astype(np.int64) << 7)
+    code = np.where(scale[..., None] > 0, code, 0).reshape(rows, nf)
+    rope_vals = round_bf16(x32[:, nf:])
+    return code.astype(np.uint8), scale, rope_vals
+
+
+def round_bf16(x32: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (round to nearest, ties to even) and return them as
+    float64: keep the top 16 bits of the fp32 pattern after adding the rounding bias."""
+    u = np.asarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    bias = 0x7FFF + ((u >> 16) & 1)
+    r = ((u + bias) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def dequantize_main_kv_fp8(codes, scales, rope_vals, group: int = 64) -> np.ndarray:
+    """Exact fp64 value of a production main-KV entry: E4M3 value x its group scale, then
+    the bf16 RoPE channels -> [rows, c]."""
+    codes = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    t4 = e4m3_values()
+    mag = t4[codes & 0x7F]
+    val = np.where(codes & 0x80, -mag, mag)
+    s = np.repeat(np.asarray(scales, dtype=np.float32).astype(np.float64), group, axis=1)
+    return np.concatenate([val * s, np.asarray(rope_vals, dtype=np.float64)], axis=1)
 
 
 # ----------------------------------------------------------------------------- [CSA-DEF] s7

@@ -58,6 +58,13 @@ SLIPS = {
         ("pooled += [(m * (i - 1) + p, 1, bias[1][p])", "pooled += [(m * (i - 1) + p, 0, bias[1][p])"),
     "decode: ring slot off by one":
         ("local[t % local.shape[0]] = as_f64(kv_row)", "local[(t + 1) % local.shape[0]] = as_f64(kv_row)"),
+    "fp8 main KV: scale amax/240":
+        ("scale = (amax / np.float32(448.0)).astype(np.float32)",
+         "scale = (amax / np.float32(240.0)).astype(np.float32)"),
+    "fp8 main KV: RoPE channels taken from the front":
+        ("rope_vals = round_bf16(x32[:, nf:])", "rope_vals = round_bf16(x32[:, :rope])"),
+    "fp8 main KV: bf16 rounding truncates":
+        ("bias = 0x7FFF + ((u >> 16) & 1)", "bias = 0 * u"),
     "fp4: E4M3 exponent bias 8":
         ("vals.append((1.0 + mant / 8.0) * 2.0 ** (e - 7))", "vals.append((1.0 + mant / 8.0) * 2.0 ** (e - 8))"),
     "fp4: e2m1 subnormal 0.25":

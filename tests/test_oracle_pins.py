@@ -572,6 +572,79 @@ def test_e4m3_rounding_matches_torch():
     np.testing.assert_array_equal(ours, theirs.astype(np.int64))
 
 
+# ----------------------------------------------------------------------------- main-KV FP8 entry
+
+
+def test_main_kv_and_index_key_payloads_reproduce_state_table():
+    """Entry payloads taken from the oracle's formats (FP8 codes + bf16 RoPE channels of a
+    512-channel main entry; FP4 codes of a 128-channel index key) reproduce the pages'
+    persistent-state table and the 736-byte amortised write."""
+    rng = _rng(70)
+    codes, scales, rope = O.quantize_main_kv_fp8(rng.standard_normal((1, 512)))
+    main_b = codes.shape[1] * 1 + rope.shape[1] * 2                  # payload, no scales
+    assert main_b == O.main_kv_payload_bytes(512, 64) == 576
+    kcodes, _ = O.quantize_fp4(rng.standard_normal((1, 128)))
+    index_b = kcodes.shape[1]
+    assert index_b == 64
+    mib = float(1 << 20)
+    rows = [r for r in _rows("state_payload_flash.txt") if len(r) == 6]
+    assert len(rows) == 4
+    for L, E, main, index, local, total in rows:
+        L, E = int(L), int(E)
+        assert E == O.completed_entries(L - 1, 4)
+        got = (E * main_b / mib, E * index_b / mib, 128 * main_b / mib)
+        got = got + (sum(got),)
+        for g, want in zip(got, (main, index, local, total)):
+            assert round(g, 3) == float(want), (L, g, want)
+    (write,) = [r for r in _rows("state_payload_flash.txt") if r[0] == "write_bytes_per_token_layer"]
+    assert main_b + (main_b + index_b) / 4 == int(write[1])
+
+
+def test_main_kv_fp8_rounding_matches_torch_and_layout():
+    """FP8 codes are torch's float8_e4m3fn cast of the fp32 quotients x / scale, scale =
+    amax / 448 per 64 channels; the last 64 channels are torch's bf16 rounding of x."""
+    rng = _rng(71)
+    x = (rng.standard_normal((6, 512)) * np.exp(rng.uniform(-8, 8, (6, 1)))).astype(np.float32)
+    x[0, :64] = 0.0                                                    # an all-zero group
+    codes, scales, rope = O.quantize_main_kv_fp8(x)
+    assert codes.shape == (6, 448) and scales.shape == (6, 7) and rope.shape == (6, 64)
+    assert scales[0, 0] == 0 and (codes[0, :64] == 0).all()
+    g = x[:, :448].reshape(6, 7, 64)
+    want_scale = (np.abs(g).max(axis=-1) / np.float32(448.0)).astype(np.float32)
+    np.testing.assert_array_equal(scales, want_scale)
+    q = (g / np.where(want_scale > 0, want_scale, 1)[..., None]).astype(np.float32).reshape(6, 448)
+    theirs = torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    nz = np.repeat(want_scale > 0, 64, axis=1)
+    np.testing.assert_array_equal(codes[nz], theirs[nz])
+    np.testing.assert_array_equal(rope, torch.from_numpy(x[:, 448:]).to(torch.bfloat16).double().numpy())
+
+
+def test_main_kv_fp8_round_trip_and_error_bound():
+    """Entries built from E4M3 values times a power-of-two scale (the group maximum 448)
+    come back exactly; random entries come back within half an E4M3 step (2^-4 relative,
+    2^-10 scale below the normal range); a negative value that rounds to zero keeps its
+    sign bit."""
+    rng = _rng(72)
+    t4 = O.e4m3_values()
+    code = rng.integers(0, 0x7F, (5, 448))
+    code[:, ::64] = 0x7E                                             # 448 in every group
+    sign = rng.integers(0, 2, (5, 448))
+    sc = 2.0 ** rng.integers(-20, 5, (5, 7))
+    x = np.where(sign, -1, 1) * t4[code] * np.repeat(sc, 64, axis=1)
+    rope = torch.randn(5, 64).to(torch.bfloat16).double().numpy()
+    xe = np.concatenate([x, rope], axis=1)
+    c2, s2, r2 = O.quantize_main_kv_fp8(xe)
+    np.testing.assert_array_equal(O.dequantize_main_kv_fp8(c2, s2, r2), xe)
+    y = rng.standard_normal((8, 512)) * 3.0
+    y[1, 5] = -1e-12                                                  # underflows in its group
+    c3, s3, r3 = O.quantize_main_kv_fp8(y)
+    d = O.dequantize_main_kv_fp8(c3, s3, r3)
+    s_el = np.repeat(s3.astype(np.float64), 64, axis=1)
+    err = np.abs(d[:, :448] - y[:, :448])
+    assert (err <= 2.0 ** -4 * np.abs(y[:, :448]) * (1 + 1e-6) + 2.0 ** -10 * s_el * (1 + 1e-6)).all()
+    assert c3[1, 5] == 0x80
+
+
 def test_e2m1_rounding_ties_and_saturation():
     v = np.array([0.0, 0.24, 0.25, 0.26, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 5.01, 6.0, 7.0, 1e9])
     want = [0.0, 0.0, 0.0, 0.5, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 6.0, 6.0, 6.0, 6.0]
