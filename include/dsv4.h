@@ -142,10 +142,13 @@ int dsv4_quantize_fp4(const void* x, uint8_t* codes, uint8_t* scales, int64_t ro
                       void* stream);
 
 /* Bytes of workspace dsv4_index_topk needs for a bf16 / fp32 request: per chunk of queries
- * the fp32 score rows and, for rows longer than 16384 entries (and k <= 4096), the region of
- * the threshold top-k (histograms, the entries above the threshold and up to 8192 boundary
- * candidates: 4 KiB + 4k bytes + 64 KiB per row). A smaller workspace makes smaller chunks;
- * a larger one is not used.
+ * (at most 256 MiB of rows) the fp32 score rows (4 * round4(max_entries) bytes each) and,
+ * for rows longer than 16384 entries, a top-k region per row: with at most 1024 rows in the
+ * request and k <= 4096 the threshold top-k's (histograms, the entries above the threshold
+ * and up to 8192 boundary candidates: 4 KiB + round256(4k) + 64 KiB), otherwise the
+ * per-segment candidates (8k bytes per 16384-entry segment). Each of the two regions is
+ * rounded up to 256 bytes. A smaller workspace makes smaller chunks; a larger one is not
+ * used.
  * max_entries = the largest number of completed entries any query of the request can see. */
 size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k);
 

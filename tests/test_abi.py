@@ -79,3 +79,42 @@ def test_workspace_size_is_bounded(lib):
     assert small == 8192 * 2048 * 4
     big = lib.dsv4_index_topk_workspace_size(1, 131072, 32768, 1024)
     assert 0 < big <= (256 << 20) and big % 256 == 0
+
+
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,nq,E,k", [(64, 1, 262144, 512), (1, 4, 16385, 512), (1, 1024, 40000, 4096)])
+def test_workspace_size_threshold_topk_rows(lib, B, nq, E, k):
+    """Requests of at most 1024 rows longer than 16384 entries: score rows plus the threshold
+    top-k region of 4 KiB + round256(4k) + 64 KiB per row, as the header states."""
+    f = lib.dsv4_index_topk_workspace_size
+    f.restype = ctypes.c_size_t
+    rows = B * nq
+    per = 4 * ((E + 3) // 4 * 4) + 4096 + _r256(4 * k) + 65536
+    rows = min(rows, (256 << 20) // per)
+    want = _r256(rows * 4 * ((E + 3) // 4 * 4)) + _r256(rows * (4096 + _r256(4 * k) + 65536))
+    assert f(B, nq, E, k) == want
+
+
+@pytest.mark.parametrize("B,nq,E,k", [(1, 1100, 17000, 256), (1, 2048, 32768, 1024)])
+def test_workspace_size_segment_topk_rows(lib, B, nq, E, k):
+    """More than 1024 long rows: score rows plus 8k bytes per 16384-entry segment per row."""
+    f = lib.dsv4_index_topk_workspace_size
+    f.restype = ctypes.c_size_t
+    nseg = (E + 16383) // 16384
+    cand = nseg * k * 8
+    per = 4 * ((E + 3) // 4 * 4) + cand
+    rows = min(B * nq, (256 << 20) // per)
+    want = _r256(rows * 4 * ((E + 3) // 4 * 4)) + _r256(rows * cand)
+    assert f(B, nq, E, k) == want
+
+
+def test_workspace_size_short_rows_and_empty(lib):
+    f = lib.dsv4_index_topk_workspace_size
+    f.restype = ctypes.c_size_t
+    assert f(1, 2048, 16384, 512) == 2048 * 16384 * 4            # no top-k region
+    assert f(1, 8192, 16384, 512) == 256 << 20                    # chunks of 4096 rows
+    assert f(0, 8, 100, 4) == 0 and f(2, 0, 100, 4) == 0
+
