@@ -99,11 +99,6 @@ __device__ __forceinline__ uint32_t mapa(uint32_t local, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
 }
-__device__ __forceinline__ void st_remote_v4(uint32_t addr, float a, float b, float c, float d) {
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
-}
 // 16-byte store into the peer CTA's shared memory whose completion is counted (in bytes) on
 // the peer's mbarrier; no release fence is needed for the peer to observe it.
 __device__ __forceinline__ void st_async_v4(uint32_t addr, float a, float b, float c, float d,
