@@ -2,9 +2,11 @@
 
 `bench.py --gpus N` runs N independent replicas: each rank times its own steps on its GPU,
 the job's time is the maximum over the ranks and the value is the units all ranks processed
-per second of that time. These tests drive that reduction over a gloo process group and the
+per second of that time. These tests drive that reduction over a gloo process group, the
 reference arm under torchrun (rank 0 alone runs the oracle sample and prints one line; the
-other ranks exit 0 without work). No GPU is used.
+other ranks exit 0 without work), and a replica that fails between steps: the surviving
+rank's reduction ends with an error within the group's timeout instead of waiting. No GPU
+is used.
 """
 import datetime
 import json
@@ -71,3 +73,41 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["value"] > 0 and d["unit"] == "tokens/s" and d["higher_is_better"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def _rank_dies(rank, world, port, out):
+    """Rank 1 leaves before the reduction; rank 0 must get an error, not wait for ever."""
+    import time
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        os._exit(3)                                       # a replica that fails between steps
+    t0 = time.monotonic()
+    try:
+        bench.max_over_ranks(1.0, world, "cpu")
+        result = "no error"
+    except Exception as e:                                # noqa: BLE001
+        result = type(e).__name__
+    with open(os.path.join(out, "rank0.json"), "w") as f:
+        json.dump({"result": result, "seconds": time.monotonic() - t0}, f)
+    os._exit(0)
+
+
+def test_a_failed_rank_ends_the_reduction_with_an_error(tmp_path):
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_dies, args=(r, 2, port, str(tmp_path))) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    alive = [p for p in procs if p.is_alive()]
+    for p in alive:
+        p.kill()
+    assert not alive, "a rank was still waiting after 120 s"
+    assert procs[1].exitcode == 3 and procs[0].exitcode == 0
+    r = json.load(open(tmp_path / "rank0.json"))
+    assert r["result"] != "no error" and r["seconds"] < 60
