@@ -36,6 +36,14 @@ SLIPS = {
         ("return w @ np.maximum(dots, 0.0)", "return np.maximum(w @ dots, 0.0)"),
     "indexer: one entry past the completed ones":
         ("dots = qI @ KI[:E_t].T", "dots = qI @ KI[:E_t + 1].T"),
+    "indexer: weight inside the ReLU":
+        ("return w @ np.maximum(dots, 0.0)", "return np.maximum(w[:, None] * dots, 0.0).sum(axis=0)"),
+    "indexer: sequence key offset ignored":
+        ("KI[int(kv_row_off[b]):], t, m)", "KI, t, m)"),
+    "attention: sequence pool offset ignored":
+        ("pool_seq = pool[base:]", "pool_seq = pool"),
+    "fp8 main KV: zero-scale group keeps sign codes":
+        ("code = np.where(scale[..., None] > 0, code, 0).reshape(rows, nf)", "code = code.reshape(rows, nf)"),
     "topk: ties to the higher entry":
         ("order = np.lexsort((np.arange(E), -scores))", "order = np.lexsort((-np.arange(E), -scores))"),
     "topk: selection not in ascending entry order":

@@ -245,6 +245,44 @@ def test_index_score_relu_and_linearity():
     np.testing.assert_allclose(a - b, K @ q[0], rtol=1e-13, atol=1e-15)
 
 
+def test_index_score_negative_weight_worked_example():
+    """The weight multiplies the ReLU of the dot product (it is not inside it): with
+    q_0 = (1, 0), q_1 = (0, 1), K_0 = (2, -3), w = (-0.5, 1):
+    I_0 = -0.5 * ReLU(2) + 1 * ReLU(-3) = -1."""
+    q = np.array([[1.0, 0.0], [0.0, 1.0]])
+    K = np.array([[2.0, -3.0]])
+    assert O.index_scores_query(q, np.array([-0.5, 1.0]), K, 3, 4).tolist() == [-1.0]
+
+
+def test_stacked_sequences_read_their_own_rows():
+    """Pools and index keys of several sequences stacked row-wise: sequence b reads from
+    row kv_row_off[b], so each sequence's result equals the one-sequence call on its own
+    rows (and differs from reading sequence 0's rows)."""
+    rng = _rng(73)
+    H, c, m, w, HI, cI, k, nq = 2, 6, 4, 3, 2, 5, 3, 9
+    E = [7, 5]
+    off = [0, 7]
+    pool = rng.standard_normal((sum(E) + 1, c))
+    KI = rng.standard_normal((sum(E) + 1, cI))
+    Q = rng.standard_normal((2, nq, H, c))
+    local = rng.standard_normal((2, nq, c))
+    qI = rng.standard_normal((2, nq, HI, cI))
+    wI = rng.random((2, nq, HI))
+    pos0 = [4 * E[0] - nq, 4 * E[1] - nq]
+    o2, l2 = O.hybrid_attention(Q, pool, off, None, None, local, pos0, w, dense_m=m)
+    idx2, cnt2 = O.index_topk(qI, wI, KI, off, pos0, m, k)
+    for b in range(2):
+        ob, lb = O.hybrid_attention(Q[b:b + 1], pool[off[b]:], [0], None, None, local[b:b + 1],
+                                    [pos0[b]], w, dense_m=m)
+        np.testing.assert_array_equal(o2[b], ob[0])
+        np.testing.assert_array_equal(l2[b], lb[0])
+        ib, cb = O.index_topk(qI[b:b + 1], wI[b:b + 1], KI[off[b]:], [0], [pos0[b]], m, k)
+        np.testing.assert_array_equal(idx2[b], ib[0])
+        np.testing.assert_array_equal(cnt2[b], cb[0])
+    o0, _ = O.hybrid_attention(Q[1:2], pool, [0], None, None, local[1:2], [pos0[1]], w, dense_m=m)
+    assert not np.allclose(o0[0], o2[1])
+
+
 def test_index_scores_only_completed_entries():
     rng = _rng(10)
     q = rng.standard_normal((2, 4))
@@ -606,9 +644,10 @@ def test_main_kv_fp8_rounding_matches_torch_and_layout():
     rng = _rng(71)
     x = (rng.standard_normal((6, 512)) * np.exp(rng.uniform(-8, 8, (6, 1)))).astype(np.float32)
     x[0, :64] = 0.0                                                    # an all-zero group
+    x[0, 1:64:2] = -0.0                                                # (with negative zeros)
     codes, scales, rope = O.quantize_main_kv_fp8(x)
     assert codes.shape == (6, 448) and scales.shape == (6, 7) and rope.shape == (6, 64)
-    assert scales[0, 0] == 0 and (codes[0, :64] == 0).all()
+    assert scales[0, 0] == 0 and (codes[0, :64] == 0).all()            # zero scale: codes 0
     g = x[:, :448].reshape(6, 7, 64)
     want_scale = (np.abs(g).max(axis=-1) / np.float32(448.0)).astype(np.float32)
     np.testing.assert_array_equal(scales, want_scale)
