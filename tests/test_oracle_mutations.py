@@ -44,6 +44,8 @@ SLIPS = {
         ("pool_seq = pool[base:]", "pool_seq = pool"),
     "fp8 main KV: zero-scale group keeps sign codes":
         ("code = np.where(scale[..., None] > 0, code, 0).reshape(rows, nf)", "code = code.reshape(rows, nf)"),
+    "fp8 main KV: sign of -0 dropped":
+        ("code = mag | (np.signbit(q).astype(np.int64) << 7)", "code = mag | ((q < 0).astype(np.int64) << 7)"),
     "topk: ties to the higher entry":
         ("order = np.lexsort((np.arange(E), -scores))", "order = np.lexsort((-np.arange(E), -scores))"),
     "topk: selection not in ascending entry order":

@@ -645,6 +645,7 @@ def test_main_kv_fp8_rounding_matches_torch_and_layout():
     x = (rng.standard_normal((6, 512)) * np.exp(rng.uniform(-8, 8, (6, 1)))).astype(np.float32)
     x[0, :64] = 0.0                                                    # an all-zero group
     x[0, 1:64:2] = -0.0                                                # (with negative zeros)
+    x[1, 3] = x[2, 100] = -0.0                                         # -0 in nonzero groups: 0x80
     codes, scales, rope = O.quantize_main_kv_fp8(x)
     assert codes.shape == (6, 448) and scales.shape == (6, 7) and rope.shape == (6, 64)
     assert scales[0, 0] == 0 and (codes[0, :64] == 0).all()            # zero scale: codes 0
@@ -655,6 +656,7 @@ def test_main_kv_fp8_rounding_matches_torch_and_layout():
     theirs = torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     nz = np.repeat(want_scale > 0, 64, axis=1)
     np.testing.assert_array_equal(codes[nz], theirs[nz])
+    assert codes[1, 3] == 0x80 and codes[2, 100] == 0x80
     np.testing.assert_array_equal(rope, torch.from_numpy(x[:, 448:]).to(torch.bfloat16).double().numpy())
 
 
