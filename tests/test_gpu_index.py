@@ -22,10 +22,10 @@ def _inputs(shape, nq, rows, seed):
 
 
 def _score_bound(qI64, w64, KI64, t, m):
-    """Worst-case fp32 accumulation bound per entry: 2e-5 * sum_h w_h sum_d |q_hd k_sd|."""
+    """Worst-case fp32 accumulation bound per entry: 2e-5 * sum_h |w_h| sum_d |q_hd k_sd|."""
     E = (t + 1) // m
     mag = np.abs(qI64) @ np.abs(KI64[:E]).T            # [H_I, E]
-    return 2e-5 * (w64 @ mag) + 1e-30
+    return 2e-5 * (np.abs(w64) @ mag) + 1e-30
 
 
 def _run_and_check(dsv4, qI, w, KI, offs, pos0, m, k, positions, qI_sc=None, KI_sc=None,
@@ -85,6 +85,32 @@ def test_index_ragged_bf16(dsv4, index_path, n, k, HI, cI):
     else:
         pos = [(0, t) for t in sample_positions(n, 4, extra=[4 * 4096 - 1, 4 * 4096, 4 * k])]
     _run_and_check(dsv4, qI, w, KI, [0], [0], 4, k, pos, what=f"{index_path} n={n} k={k}")
+
+
+@pytest.mark.parametrize("n,k,HI,cI", [(4 * 600 + 1, 64, 64, 128), (523, 16, 8, 64)])
+def test_index_mixed_sign_weights(dsv4, index_path, n, k, HI, cI):
+    """Head weights of both signs (the score is a weighted sum of per-head ReLUs, so it can
+    be negative): the selection still follows the fp64 scores."""
+    shape = preset("flash_csa_prefill", n=n, k=k, H_I=HI, c_I=cI)
+    qI, w, KI = _inputs(shape, n, n // 4, 5 * n + k)
+    w = 2.0 * w - 1.0
+    pos = [(0, t) for t in sample_positions(n, 4, extra=[4 * k - 1, 4 * k, n - 1], count=64)]
+    _run_and_check(dsv4, qI, w, KI, [0], [0], 4, k, pos, what=f"{index_path} mixed-sign n={n}")
+
+
+def test_index_mixed_sign_weights_long_rows(dsv4):
+    """Decode rows longer than 16384 entries (the threshold top-k) with head weights of
+    both signs: negative scores pass through the key transform and the histograms."""
+    shape = preset("flash_csa_prefill", B=2)
+    lens = [4 * 20000 + 3, 4 * 17000]
+    rows = [L // 4 for L in lens]
+    offs = list(np.concatenate([[0], np.cumsum(rows)[:-1]]).astype(np.int64))
+    g = Generator(33)
+    qI, w = g.index_queries(shape, 1)
+    w = 2.0 * w - 1.0
+    KI = g.index_keys(shape, int(sum(rows)) + 1)
+    pos0 = [L - 1 for L in lens]
+    _run_and_check(dsv4, qI, w, KI, offs, pos0, 4, 512, [(0, 0), (1, 0)], what="mixed-sign long")
 
 
 def test_index_batched_offsets_decode_like(dsv4, index_path):
