@@ -56,6 +56,9 @@ lib.dsv4_index_topk_workspace_size_ex.argtypes = [_I, _I, _I, _I, _I, _I, _I, _L
 lib.dsv4_index_topk.restype = _I
 lib.dsv4_index_topk.argtypes = [_I, _P, _P, _P, _P, _P, _L, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                 _P, _P, _P, _L, _P, _S, _P]
+lib.dsv4_index_topk_noalloc.restype = _I
+lib.dsv4_index_topk_noalloc.argtypes = [_I, _P, _P, _P, _P, _P, _L, _P, _P, _I, _I, _I, _I, _I, _I,
+                                        _I, _P, _P, _P]
 lib.dsv4_hybrid_sparse_attn.restype = _I
 lib.dsv4_hybrid_sparse_attn.argtypes = [_I, _P, _P, _L, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
                                         _I, _I, _I, _P, _F, _P, _P, _P, _S, _P]

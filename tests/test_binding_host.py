@@ -89,3 +89,47 @@ def test_non_contiguous_views_are_refused():
     x = _FakeCuda(torch.zeros(4, 32, dtype=torch.bfloat16).t())
     with pytest.raises(ValueError, match="must be contiguous"):
         dsv4.dsv4_quantize_fp4(x)
+
+
+def _header_declarations():
+    import re
+    text = open(os.path.join(ROOT, "include", "dsv4.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    decls = {}
+    for ret, name, params in re.findall(r"\b(int|size_t|const char\*)\s+(dsv4_[a-z0-9_]+)\s*\(([^)]*)\)\s*;",
+                                        text, flags=re.S):
+        ps = [p.strip() for p in params.replace("\n", " ").split(",") if p.strip()]
+        decls[name] = (ret, [] if ps == ["void"] else ps)
+    return decls
+
+
+def _ctype_for(param: str):
+    import ctypes
+    p = " ".join(param.split())
+    if "*" in p:
+        return (ctypes.c_void_p, ctypes.c_char_p)
+    t = p.rsplit(" ", 1)[0]
+    return {"int": (ctypes.c_int,), "int64_t": (ctypes.c_int64,), "size_t": (ctypes.c_size_t,),
+            "float": (ctypes.c_float,)}[t]
+
+
+def test_binding_argtypes_match_the_header():
+    """Every entry point the binding declares has as many ctypes arguments as the header's
+    parameters, each of the same width (a 64-bit size passed as a 32-bit int would be read
+    with garbage upper bits), and the matching return type."""
+    import ctypes
+    decls = _header_declarations()
+    assert len(decls) >= 12
+    checked = 0
+    for name, (ret, params) in decls.items():
+        fn = getattr(dsv4.lib, name)
+        want_ret = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p}[ret]
+        assert fn.restype == want_ret, f"{name}: restype {fn.restype} for {ret}"
+        if fn.argtypes is None:
+            assert name == "dsv4_abi_version" or not params, f"{name}: argtypes not declared"
+            continue
+        assert len(fn.argtypes) == len(params), f"{name}: {len(fn.argtypes)} ctypes args, {len(params)} in the header"
+        for i, (have, p) in enumerate(zip(fn.argtypes, params)):
+            assert have in _ctype_for(p), f"{name} arg {i} ({p}): {have}"
+        checked += 1
+    assert checked >= 10
