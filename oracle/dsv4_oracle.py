@@ -19,6 +19,9 @@ Sources (page title, then section / equation):
       s3.2 / s4 shared-KV MQA (each entry is both key and value for every head)
       s5.1 local window L_t = {max(0,t-w+1)..t} and ONE candidate list / softmax
       s5.2 logit scaled by 1/sqrt(c)
+      s5.2 RMSNorm of query heads and the shared KV head; RoPE on the last 64 channels
+           (query at t, compressed entry s at m*s, local entry j at j); inverse RoPE
+           of the output's last 64 channels at t
       s5.3 sink logit z'_h in the denominator only
       s7  incremental decode state machine (local ring slot per token, bounded
           compressor tail, entry emitted when (t+1) is a multiple of the ratio)
@@ -43,6 +46,8 @@ Readings taken where the pages are silent (each is also listed in the design not
     from the fp32 quotient, saturating at +-6; a zero scale gives zero codes.
     The sign bit follows IEEE rounding (a negative value that rounds to zero is -0,
     code 0x8). Two codes per byte, element 2j in the low nibble.
+  * RMSNorm without a learned gain, eps = 1e-6; RoPE on adjacent channel pairs of the
+    last 64 channels with base 10000 (the pages fix the rotated channels and positions).
   * Main-KV FP8 entries: the RoPE channels are the last 64; the FP8 channels carry one
     fp32 scale per 64 channels, scale = amax / 448 (the pages leave the scale metadata
     open).
@@ -351,6 +356,51 @@ def dequantize_fp4(codes, scales, cols: int) -> np.ndarray:
     t4 = e4m3_values()
     s = t4[scales.astype(np.int64) & 0x7F]
     return val * np.repeat(s, 16, axis=1)
+
+
+# ----------------------------------------------------------------------------- [CSA-DEF] s5.2
+
+
+def rms_norm(x, eps: float = 1e-6) -> np.ndarray:
+    """RMS normalisation over the last axis ([CSA-DEF] s5.2: every query head and the shared
+    KV head, right before core attention): x / sqrt(mean(x^2) + eps). Reading: no learned
+    gain (a per-channel gain would be an upstream weight), eps = 1e-6."""
+    x = as_f64(x)
+    return x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)
+
+
+def rope_rotate(x, pos, rope: int = 64, base: float = 10000.0, inverse: bool = False):
+    """rho_p of [CSA-DEF] s5.2 on the last `rope` channels of x [..., c]: channel pairs
+    (c - rope + 2i, c - rope + 2i + 1) rotate by the angle p * base^(-2i / rope); the other
+    channels are unchanged; inverse=True rotates by minus the angle. `pos` broadcasts over
+    the leading axes of x. Reading: adjacent channel pairs and base 10000 (the pages fix
+    only which channels rotate and the positions)."""
+    x = np.array(as_f64(x), copy=True)
+    c = x.shape[-1]
+    half = rope // 2
+    freq = base ** (-2.0 * np.arange(half) / rope)                  # [rope/2]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * freq       # [..., rope/2]
+    if inverse:
+        ang = -ang
+    a = x[..., c - rope::2].copy()
+    b = x[..., c - rope + 1::2].copy()
+    cs, sn = np.cos(ang), np.sin(ang)
+    x[..., c - rope::2] = a * cs - b * sn
+    x[..., c - rope + 1::2] = a * sn + b * cs
+    return x
+
+
+def attend_query_rope(q, t: int, entries, entry_pos, sink=None, scale: float = None,
+                      rope: int = 64):
+    """One query's core attention with the s5.2 contract: the query heads q [H, c] and the
+    candidate entries [N, c] are RMS-normalised, q is rotated at its position t and entry j
+    at entry_pos[j] (compressed entry s: m*s for CSA, m'*s for HCA; local entry j: j), one
+    softmax as in attend_query, and the output's last `rope` channels are rotated back at t
+    (inverse RoPE). Returns (o [H, c], lse [H])."""
+    qn = rope_rotate(rms_norm(q), np.full(as_f64(q).shape[0], t), rope)
+    kv = rope_rotate(rms_norm(entries), np.asarray(entry_pos), rope)
+    o, lse = attend_query(qn, kv, sink, scale)
+    return rope_rotate(o, np.full(o.shape[0], t), rope, inverse=True), lse
 
 
 # ----------------------------------------------------------------------------- main-KV cache entry ([CSA-DEF] s8)

@@ -46,6 +46,18 @@ SLIPS = {
         ("code = np.where(scale[..., None] > 0, code, 0).reshape(rows, nf)", "code = code.reshape(rows, nf)"),
     "fp8 main KV: sign of -0 dropped":
         ("code = mag | (np.signbit(q).astype(np.int64) << 7)", "code = mag | ((q < 0).astype(np.int64) << 7)"),
+    "rope: rotation sign":
+        ("x[..., c - rope::2] = a * cs - b * sn", "x[..., c - rope::2] = a * cs + b * sn"),
+    "rope: frequency exponent":
+        ("freq = base ** (-2.0 * np.arange(half) / rope)", "freq = base ** (-1.0 * np.arange(half) / rope)"),
+    "rope: output not rotated back":
+        ("return rope_rotate(o, np.full(o.shape[0], t), rope, inverse=True), lse", "return o, lse"),
+    "rms norm: sum instead of mean":
+        ("return x / np.sqrt((x * x).mean(axis=-1, keepdims=True) + eps)",
+         "return x / np.sqrt((x * x).sum(axis=-1, keepdims=True) + eps)"),
+    "rope: entries rotated at the query position":
+        ("kv = rope_rotate(rms_norm(entries), np.asarray(entry_pos), rope)",
+         "kv = rope_rotate(rms_norm(entries), np.full(len(entry_pos), t), rope)"),
     "topk: ties to the higher entry":
         ("order = np.lexsort((np.arange(E), -scores))", "order = np.lexsort((-np.arange(E), -scores))"),
     "topk: selection not in ascending entry order":

@@ -518,6 +518,64 @@ def test_window_only_for_queries_before_first_entry():
         np.testing.assert_allclose(o[0, t], ref, rtol=1e-15)
 
 
+# ----------------------------------------------------------------------------- RMSNorm / RoPE
+
+
+def test_rms_norm_closed_form_and_scale_invariance():
+    """RMSNorm output has mean square 1 (up to eps) and ignores a positive scale of its input;
+    a constant row a maps to a / sqrt(a^2 + eps)."""
+    rng = _rng(80)
+    x = rng.standard_normal((4, 512))
+    y = O.rms_norm(x, eps=0.0)
+    np.testing.assert_allclose((y * y).mean(axis=-1), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(O.rms_norm(7.5 * x, eps=0.0), y, rtol=1e-13)
+    np.testing.assert_allclose(O.rms_norm(np.full((1, 8), 3.0), eps=1e-6), 3.0 / np.sqrt(9.0 + 1e-6),
+                               rtol=1e-15)
+
+
+def test_rope_rotation_properties():
+    """rho_p is a rotation of the last 64 channels only: norm preserving, rho_a o rho_b =
+    rho_(a+b), its inverse undoes it; in each pair the 2-D rotation by p * base^(-2i/64) maps
+    (1, 0) to (cos, sin) of that angle."""
+    rng = _rng(81)
+    x = rng.standard_normal((3, 512))
+    y = O.rope_rotate(x, [3, 40, 1000])
+    np.testing.assert_array_equal(y[:, :448], x[:, :448])
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-14)
+    np.testing.assert_allclose(O.rope_rotate(O.rope_rotate(x, [3, 40, 1000]), [4, 2, 17]),
+                               O.rope_rotate(x, [7, 42, 1017]), rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(O.rope_rotate(y, [3, 40, 1000], inverse=True), x, rtol=1e-12, atol=1e-12)
+    e = np.zeros((1, 64))
+    e[0, 2 * 5] = 1.0                                        # pair i = 5
+    r = O.rope_rotate(e, [9])
+    ang = 9 * 10000.0 ** (-2 * 5 / 64)
+    np.testing.assert_allclose(r[0, 10:12], [np.cos(ang), np.sin(ang)], rtol=1e-14)
+    assert np.count_nonzero(r) == 2
+
+
+def test_rope_logits_and_output_depend_on_relative_positions():
+    """[CSA-DEF] s5.2: q at t against entry j at p_j gives a logit that depends on t - p_j
+    only, and the inverse rotation at t puts the output in relative form: shifting the
+    query and every entry position by the same amount changes neither the output nor the
+    LSE; without the inverse rotation the output would carry the absolute rotation."""
+    rng = _rng(82)
+    H, c, N, t = 3, 128, 9, 50
+    q = rng.standard_normal((H, c))
+    ent = rng.standard_normal((N, c))
+    pos = np.array([0, 4, 8, 12, 46, 47, 48, 49, 50])          # compressed (m*s) then local
+    o1, l1 = O.attend_query_rope(q, t, ent, pos)
+    o2, l2 = O.attend_query_rope(q, t + 777, ent, pos + 777)
+    np.testing.assert_allclose(o1, o2, rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(l1, l2, rtol=1e-12)
+    # the same attention weights as plain attention over the rotated, normalised inputs
+    qn = O.rope_rotate(O.rms_norm(q), np.full(H, t))
+    kv = O.rope_rotate(O.rms_norm(ent), pos)
+    o_abs, l_abs = O.attend_query(qn, kv)
+    np.testing.assert_allclose(l1, l_abs, rtol=1e-14)
+    np.testing.assert_allclose(o1[:, :c - 64], o_abs[:, :c - 64], rtol=1e-13)
+    assert not np.allclose(o1[:, c - 64:], o_abs[:, c - 64:])
+
+
 # ----------------------------------------------------------------------------- decode state
 
 
