@@ -7,7 +7,7 @@ with the CUDA kernels.
 
 Everything is computed in float64 (numpy). Storage formats are decoded exactly
 (bf16 -> fp32 -> fp64 is exact; an FP4 e2m1 code times its E4M3 scale is exact).
-Library primitives used as single steps: numpy matmul, exp/log, max, lexsort.
+Library primitives used as single steps: numpy matmul, exp/log, sqrt, cos/sin, max, lexsort.
 
 Sources (page title, then section / equation):
   [CSA-DEF] "CSA And HCA: Definition, State, And Cost Model"
