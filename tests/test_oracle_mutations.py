@@ -96,6 +96,19 @@ SLIPS = {
          "packed = (code[:, 1::2] | (code[:, 0::2] << 4)).astype(np.uint8)"),
     "fp4: block scale amax/4":
         ("s32 = (amax / np.float32(6.0)).astype(np.float32)", "s32 = (amax / np.float32(4.0)).astype(np.float32)"),
+    "csa layer: main pool fed to the indexer":
+        ("idx, counts = index_topk(qI64, w, KI.reshape(B * E, -1)",
+         "idx, counts = index_topk(qI64, w, pool.reshape(B * E, -1)"),
+    "csa layer: index keys compressed without overlap":
+        ("KI = compress(CI, ZI, biasI, m, overlap=True)",
+         "KI = compress(CI[..., :CI.shape[-1] // 2], ZI[..., :ZI.shape[-1] // 2], biasI[:1], m, overlap=False)"),
+    "csa layer: FP4 branch leaves the keys unquantised":
+        ("KI = dequantize_fp4(kc, ks, KI.shape[-1]).reshape(KI.shape)", "KI = KI.reshape(KI.shape)"),
+    "csa layer: FP4 branch leaves the queries unquantised":
+        ("qI64 = dequantize_fp4(qc, qs, cI).reshape(Bq, nq, HI, cI)", "qI64 = qI64.reshape(Bq, nq, HI, cI)"),
+    "csa layer: attention window one position wider":
+        ("O, LSE = hybrid_attention(Q, pool.reshape(B * E, -1), off, idx, counts, local, pos0,\n                              wwin, sink, scale, 0, queries)",
+         "O, LSE = hybrid_attention(Q, pool.reshape(B * E, -1), off, idx, counts, local, pos0,\n                              wwin + 1, sink, scale, 0, queries)"),
     "fp4: sign lost on rounding to zero":
         ("code = (mag | (sign.astype(np.int64) << 3))",
          "code = (mag | ((sign & (mag > 0)).astype(np.int64) << 3))"),

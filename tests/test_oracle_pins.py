@@ -794,3 +794,128 @@ def test_fp4_negative_underflow_keeps_sign():
     x[0, 1] = -0.2                                   # -0.2 rounds to -0
     c, s = O.quantize_fp4(x)
     assert c[0, 0] == (0x7 | (0x8 << 4))
+
+
+# ----------------------------------------------------------------------------- the layer chain
+
+
+def _csa_layer_inputs(rng, B, n, H, c, cI, HI, m):
+    C, Z, bias = _compress_inputs(rng, B, n, c, m, 2)
+    CI, ZI, biasI = _compress_inputs(rng, B, n, cI, m, 2)
+    qI = rng.standard_normal((B, n, HI, cI))
+    w = rng.random((B, n, HI))
+    Q = rng.standard_normal((B, n, H, c))
+    local = rng.standard_normal((B, n, c))
+    return dict(C=C, Z=Z, bias=bias, CI=CI, ZI=ZI, biasI=biasI, qI=qI, w=w, Q=Q, local=local)
+
+
+def _layer(inp, m, k, wwin, **kw):
+    return O.csa_prefill_layer(inp["C"], inp["Z"], inp["bias"], inp["CI"], inp["ZI"], inp["biasI"],
+                               inp["qI"], inp["w"], inp["Q"], inp["local"], m, k, wwin, **kw)
+
+
+def test_csa_layer_full_budget_equals_masked_sdpa():
+    """Sections 3-5.1: with k >= floor(n/m) TopK keeps every completed entry, so the layer's
+    output is one softmax over [all entries s < floor((t+1)/m) ; window] -- masked SDPA
+    (library) over the layer's own pool and the local stream, for every sequence."""
+    rng = _rng(31)
+    B, n, H, c, m, wwin = 2, 45, 3, 8, 4, 6
+    inp = _csa_layer_inputs(rng, B, n, H, c, c, 2, m)
+    res = _layer(inp, m, n // m + 3, wwin)
+    E = n // m
+    scale = 1 / math.sqrt(c)
+    for b in range(B):
+        assert (res["counts"][b] == [(t + 1) // m for t in range(n)]).all()
+        kv = np.concatenate([res["pool"][b], inp["local"][b]], axis=0)
+        mask = np.zeros((n, E + n), dtype=bool)
+        for t in range(n):
+            mask[t, :(t + 1) // m] = True
+            mask[t, E + max(0, t - wwin + 1):E + t + 1] = True
+        for h in range(H):
+            ref = _sdpa(inp["Q"][b, :, h], kv, mask, scale)
+            np.testing.assert_allclose(res["O"][b, :, h], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_csa_layer_indexer_reads_only_its_own_stream():
+    """Section 3.1: the indexer scores separate index keys K^I (a second compressor instance
+    over its own stream), not the main entries. Changing the main stream C leaves every
+    selection unchanged and changes the output; changing stream b of the index stream in
+    block 0 (pooled only into index key 1, by the overlap of section 2.1) changes some
+    selection. Main and index widths are equal here, so feeding the main pool to the indexer
+    would run and be caught by value."""
+    rng = _rng(32)
+    B, n, H, c, m, k, wwin = 2, 64, 2, 8, 4, 3, 5
+    inp = _csa_layer_inputs(rng, B, n, H, c, c, 2, m)
+    base = _layer(inp, m, k, wwin)
+    pert = dict(inp, C=inp["C"] + 3.0 * rng.standard_normal(inp["C"].shape))
+    r1 = _layer(pert, m, k, wwin)
+    np.testing.assert_array_equal(r1["idx"], base["idx"])
+    assert np.abs(r1["O"] - base["O"]).max() > 1e-3
+    CI = inp["CI"].copy()
+    CI[:, :m, c:] = 5.0 + 5.0 * rng.standard_normal(CI[:, :m, c:].shape)
+    r2 = _layer(dict(inp, CI=CI), m, k, wwin)
+    changed = np.nonzero((r2["idx"] != base["idx"]).any(axis=-1))
+    assert len(changed[0]) > 0
+    # only queries that can see index key 1 (t >= 2m - 1) may change
+    assert changed[1].min() >= 2 * m - 1
+
+
+def _fp4_grid_rows(rng, rows, cols, exp):
+    """Rows whose 16-element groups are e2m1 grid points times 2^exp with one element at 6
+    (so amax / 6 = 2^exp is the exact E4M3 scale and quantisation is the identity)."""
+    grid = O.e2m1_values()
+    mags = grid[rng.integers(0, 8, size=(rows, cols))]
+    mags[:, ::16] = 6.0
+    sgn = np.where(rng.random((rows, cols)) < 0.5, -1.0, 1.0)
+    return sgn * mags * 2.0 ** exp
+
+
+def test_csa_layer_fp4_is_exact_on_representable_operands():
+    """Section 8 precision table (indexer in FP4): quantisation is the identity on operands
+    that are already FP4 values with exact E4M3 block scales, so the FP4 layer selects what
+    the unquantised layer selects. The index keys are made representable by constant blocks:
+    every position pooled into key i carries the same row, and softmax weights sum to one."""
+    rng = _rng(33)
+    B, n, H, c, cI, HI, m, k, wwin = 1, 48, 2, 8, 32, 3, 4, 3, 4
+    inp = _csa_layer_inputs(rng, B, n, H, c, cI, HI, m)
+    E = n // m
+    u = _fp4_grid_rows(rng, E + 1, cI, -3)                 # key i = row u[i]
+    CI = np.empty((B, n, 2 * cI))
+    for j in range(E):
+        CI[0, m * j:m * (j + 1), :cI] = u[j]               # stream a of block j -> key j
+        CI[0, m * j:m * (j + 1), cI:] = u[j + 1]           # stream b of block j -> key j + 1
+    qI = _fp4_grid_rows(rng, B * n * HI, cI, -2).reshape(B, n, HI, cI)
+    inp = dict(inp, CI=CI, qI=qI)
+    r32 = _layer(inp, m, k, wwin)
+    r4 = _layer(inp, m, k, wwin, index_fp4=True)
+    np.testing.assert_allclose(r32["KI"][0], u[:E], rtol=1e-15, atol=0)
+    np.testing.assert_array_equal(r4["KI"][0], u[:E])
+    np.testing.assert_array_equal(r4["idx"], r32["idx"])
+    np.testing.assert_allclose(r4["O"], r32["O"], rtol=1e-13, atol=1e-14)
+
+
+def test_csa_layer_fp4_scores_the_quantised_operands():
+    """The FP4 layer's selection is the TopK (brute force here) of the scores of the
+    quantise -> dequantise images of both q^I and K^I; the quantiser and the compressor
+    are pinned on their own above, so this pins how the layer wires them."""
+    rng = _rng(34)
+    B, n, H, c, cI, HI, m, k, wwin = 1, 40, 2, 8, 32, 3, 4, 4, 4
+    inp = _csa_layer_inputs(rng, B, n, H, c, cI, HI, m)
+    res = _layer(inp, m, k, wwin, index_fp4=True)
+    KI = O.compress(inp["CI"], inp["ZI"], inp["biasI"], m, True)[0]
+    kc, ks = O.quantize_fp4(KI)
+    K4 = O.dequantize_fp4(kc, ks, cI)
+    qc, qs = O.quantize_fp4(inp["qI"].reshape(-1, cI))
+    q4 = O.dequantize_fp4(qc, qs, cI).reshape(n, HI, cI)
+    differs = 0
+    for t in range(n):
+        E = (t + 1) // m
+        sc = [sum(inp["w"][0, t, h] * max(float(q4[t, h] @ K4[s]), 0.0) for h in range(HI))
+              for s in range(E)]
+        want = sorted(sorted(range(E), key=lambda j: (-sc[j], j))[:k])
+        assert res["idx"][0, t, :res["counts"][0, t]].tolist() == want, t
+        sc32 = [sum(inp["w"][0, t, h] * max(float(inp["qI"][0, t, h] @ KI[s]), 0.0)
+                    for h in range(HI)) for s in range(E)]
+        differs += int(sorted(sorted(range(E), key=lambda j: (-sc32[j], j))[:k]) != want)
+    # the quantisation is visible: some query selects differently than unquantised scores
+    assert differs > 0
