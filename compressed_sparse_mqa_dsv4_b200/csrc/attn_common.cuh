@@ -87,8 +87,5 @@ int launch_attn_tc(const AttnArgs& a, cudaStream_t st, bool* used);
 // (query, 64-head group) item.
 constexpr int ATTN_MAX_SPLIT = 8;
 long long attn_split_bytes_per_item(int c);
-int launch_attn_tc2(const AttnArgs& a, cudaStream_t st, bool* used);
-// Double-buffered 64-slot kernel for unsplit lists (c = 512, 64-head groups).
-int launch_attn_db(const AttnArgs& a, cudaStream_t st, bool* used);
 
 }  // namespace dsv4

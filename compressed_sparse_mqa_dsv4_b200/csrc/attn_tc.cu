@@ -269,13 +269,16 @@ __global__ void __maxnreg__(128)
     }
   }
 
+  // blocks and items the producers loaded (their bulk copies are drained before exit)
+  uint32_t prod_G = 0;
+  int prod_k = 0;
   if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------------ producer (4 warps)
     const int pt = tid - AT_SOFT;
     const uint64_t pool_addr = reinterpret_cast<uint64_t>(a.pool);
     const uint64_t local_addr = reinterpret_cast<uint64_t>(a.local);
-    uint32_t G = 0;
-    int k = 0;
+    uint32_t& G = prod_G;
+    int& k = prod_k;
     bool ok = true;
     if (pt == 0) tc::prefetch_tensormap(&map_q);
     for (int item = first; item < items && ok; item += gridDim.x) {
@@ -363,13 +366,6 @@ __global__ void __maxnreg__(128)
       ++k;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    if (pt == 0 && *abort) {
-      // the consumers gave up: let this thread's own bulk copies land before exiting
-      volatile int never = 0;
-      if (k > 0) tc::mbar_wait(&s.q_full, (uint32_t)((k - 1) & 1), spin, &never);
-      if (G > 0)
-        for (int c = 3; c < AT_CHUNKS; c += 4) tc::mbar_wait(&s.ch_full[c], (G - 1) & 1, spin, &never);
-    }
   } else if (warp == 12) {
     // ------------------------------------------------------------------ watcher
     // Performs the producers' mbarrier waits and passes each result on; both sides take
@@ -462,9 +458,8 @@ __global__ void __maxnreg__(128)
         }
       }
       if (!ok) {
-        tc::mma_commit_warp(&s.drain);
-        volatile int never = 0;
-        tc::mbar_wait(&s.drain, 0, spin, &never);
+        tc::mma_commit_warp(&s.drain);               // every issued MMA completes before
+        tc::mbar_drain(&s.drain, 0);                 // TMEM is released
       }
     }
     __syncwarp();
@@ -755,6 +750,14 @@ __global__ void __maxnreg__(128)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, TM_COLS);
   }
+  if (tid == AT_SOFT && *abort) {
+    // After an abort (final now: every thread has passed the barrier) the last item's Q and
+    // the last block's TMA boxes and cp.async arrivals may still be landing: let them land
+    // before the CTA's shared memory is released. Without an abort they were all consumed.
+    if (prod_k > 0) tc::mbar_drain(&s.q_full, (uint32_t)((prod_k - 1) & 1));
+    if (prod_G > 0)
+      for (int c = 3; c < AT_CHUNKS; c += 4) tc::mbar_drain(&s.ch_full[c], (prod_G - 1) & 1);
+  }
 }
 
 // Merges the nsplit partials of every (query, head group): one warp per head (grid: items x
@@ -866,16 +869,6 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
     }
   }
   a.nsplit = nsplit;
-  if (nsplit == 1) {
-    // DSV4_ATTN_DB=1: unsplit lists go to the double-buffered 64-slot kernel (slower on the
-    // flash CSA prefill workload: its gather and its tensor-core operand reads compete for
-    // shared-memory bandwidth; kept as a measured alternative)
-    const char* db = std::getenv("DSV4_ATTN_DB");
-    if (db && db[0] == '1') {
-      const int s3 = launch_attn_db(a, st, used);
-      if (s3 != DSV4_OK || *used) return s3;
-    }
-  }
   if (nsplit > 1)
     a.part_ml = reinterpret_cast<float2*>(a.part_o + items * nsplit * AT_H * (long long)AT_C);
 

@@ -338,12 +338,7 @@ extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* poo
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == DSV4_BF16) {
     bool used = false;
-    int s = launch_attn_tc2(a, st, &used);
-    if (s != DSV4_OK || used) {
-      trace_path("hybrid attention: tcgen05, 2-CTA cluster");
-      return s;
-    }
-    s = launch_attn_tc(a, st, &used);
+    int s = launch_attn_tc(a, st, &used);
     if (s != DSV4_OK || used) {
       trace_path("hybrid attention: tcgen05, single CTA");
       return s;

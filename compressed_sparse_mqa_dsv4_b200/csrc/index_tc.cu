@@ -153,13 +153,15 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   tc::tc_fence_after();
   const uint32_t tmem = s.tmem_base;
 
+  uint32_t prod_gb = 0;                                // key blocks the producer issued
+  int prod_k = 0;                                      // units whose Q it loaded
   if (warp == 8) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       tc::prefetch_tensormap(&map_q);
       tc::prefetch_tensormap(&map_k);
-      uint32_t gb = 0;                                 // key blocks issued so far
-      int k = 0;                                       // units loaded so far
+      uint32_t& gb = prod_gb;                          // key blocks issued so far
+      int& k = prod_k;                                 // units loaded so far
       bool ok = true;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const IxUnit w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
@@ -210,13 +212,6 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         }
         if (q_loaded) ++k;
       }
-      if (*abort) {
-        // the consumers gave up: let this thread's own bulk copies land before exiting
-        volatile int never = 0;
-        for (uint32_t g = gb > (uint32_t)NST ? gb - NST : 0; g < gb; ++g)
-          tc::mbar_wait(&s.k_full[g % NST], (g / NST) & 1, spin, &never);
-        if (k > 0) tc::mbar_wait(&s.q_full, (uint32_t)((k - 1) & 1), spin, &never);
-      }
     }
     __syncwarp();
   } else if (warp == 9) {
@@ -264,8 +259,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       if (!ok) {
         // let every issued MMA finish before TMEM is released
         tc::mma_commit_warp(&s.drain);
-        volatile int never = 0;
-        tc::mbar_wait(&s.drain, 0, spin, &never);
+        tc::mbar_drain(&s.drain, 0);
       }
     }
     __syncwarp();
@@ -360,6 +354,14 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
   if (warp == 9) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, IX_TM_COLS);
+  }
+  if (tid == 8 * 32 && *abort) {
+    // After an abort (final now: every thread has passed the barrier) the producer's last
+    // key blocks and Q may still be landing: let them land before the CTA's shared memory
+    // is released. Without an abort the MMAs consumed them all.
+    for (uint32_t g = prod_gb > (uint32_t)NST ? prod_gb - NST : 0; g < prod_gb; ++g)
+      tc::mbar_drain(&s.k_full[g % NST], (g / NST) & 1);
+    if (prod_k > 0) tc::mbar_drain(&s.q_full, (uint32_t)((prod_k - 1) & 1));
   }
 }
 

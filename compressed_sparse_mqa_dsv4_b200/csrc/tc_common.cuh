@@ -1,5 +1,5 @@
 // sm_100a building blocks for the tensor-core kernels: mbarriers with bounded waits,
-// TMA (tiled and row-gather) loads, tcgen05 (TMEM alloc, MMA, commit, ld/st) and the
+// TMA tiled loads and stores, tcgen05 (TMEM alloc, MMA, commit, ld/st) and the
 // shared-memory / instruction descriptors of the 5th-generation tensor core.
 //
 // Every wait is bounded: after `spin_limit` unsuccessful polls the waiter records
@@ -87,6 +87,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+// Polls allowed to a drain wait (below). A drain waits for this CTA's own copies or MMAs,
+// which always complete within microseconds; the bound only keeps the wait finite.
+constexpr uint32_t kDrainPolls = 1u << 24;
+
+// Wait for the CTA's own in-flight asynchronous work (bulk copies, MMAs) before it releases
+// TMEM or exits after an abort. Unlike mbar_wait it ignores the abort flag and the device
+// status word -- an abort is why it runs -- and it does not flag a timeout of its own.
+__device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
+  if (mbar_test_wait(bar, parity)) return true;
+  for (uint32_t i = 0; i < kDrainPolls; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -105,19 +119,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Row gather: four rows y0..y3 of a 2D tensor (box = {width, 1}) into four consecutive
-// box-sized slots of shared memory.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y0, int32_t y1, int32_t y2,
-                                            int32_t y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
-      "r"(y2), "r"(y3)
       : "memory");
 }
 

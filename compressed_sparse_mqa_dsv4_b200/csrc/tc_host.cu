@@ -42,11 +42,15 @@ int encode_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType
   return DSV4_OK;
 }
 
+// DSV4_SPIN_LIMIT=N sets the polls of every bounded wait (read once per process). N = 0
+// leaves only the non-blocking first test, so any wait whose phase has not completed when
+// it starts gives up at once: the way to exercise the abort path of the kernels.
 uint32_t spin_limit() {
   static uint32_t lim = [] {
     const char* e = std::getenv("DSV4_SPIN_LIMIT");
-    long long v = e ? std::atoll(e) : 0;
-    return v > 0 ? (uint32_t)v : (uint32_t)(1u << 22);
+    if (!e || !*e) return (uint32_t)(1u << 22);
+    const long long v = std::atoll(e);
+    return v >= 0 && v < (1ll << 32) ? (uint32_t)v : (uint32_t)(1u << 22);
   }();
   return lim;
 }

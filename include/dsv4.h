@@ -203,6 +203,12 @@ int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_scales, const 
  * scores_out, scores_ld, workspace and workspace_bytes.
  *   - max_entries above 2,097,152 (one score row larger than the scratch) is rejected
  *     with DSV4_ERR_INVALID_ARG before anything is enqueued.
+ *   - Queries are processed in chunks whose score rows fit in the scratch; long rows
+ *     (more than 16384 entries) also need their top-k region there and get smaller chunks.
+ *   - DSV4_FP4 operands are scored on the tensor cores only while the exact bf16 expansion
+ *     of the whole key pool (256 bytes per key row at c_I = 128) fits in the scratch beside
+ *     at least one score row: above roughly 32,000 key rows such requests are scored on
+ *     CUDA cores instead (same results up to fp32 rounding order, lower throughput).
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
  *   - Every call on a device shares the one array. The scratch holds score rows that

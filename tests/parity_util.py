@@ -1,7 +1,11 @@
 """Comparison rules shared by the GPU parity tests.
 
 Tolerances (from the stated targets; written here once):
-  * floating point outputs stored in bf16: max |gpu - oracle| <= 2e-2 (absolute);
+  * floating point outputs stored in bf16: max |gpu - oracle| <= 2e-2 (absolute, the stated
+    bound) AND max |gpu - oracle| <= 1e-2 * max |oracle| (norm-wise). The second bound keeps
+    the check meaningful where the outputs themselves are far below 2e-2 (long candidate
+    lists of small rows average to |O| ~ 1e-3): a zeroed or wrongly gathered output fails it.
+    bf16 storage of O contributes 2^-9 relative, the bf16 softmax weights about as much;
   * fp32 outputs: max |gpu - oracle| <= 1e-4 * max |oracle| (norm-wise relative);
   * LSE: the same rule as the output of that dtype;
   * integer / byte outputs (FP4 codes, scale bytes, top-k indices, counts): bit-exact,
@@ -14,22 +18,29 @@ import numpy as np
 import torch
 
 BF16_ABS = 2e-2
+BF16_REL = 1e-2
 F32_REL = 1e-4
 TIE_REL = 1e-6
 
 
-def assert_close(gpu, ref, dtype: str, what: str):
+def assert_close(gpu, ref, dtype: str, what: str, verbose: bool = False):
+    """Compare under the rule of `dtype` ("bf16" or "f32"); returns max |diff|. With verbose,
+    prints the observed error, the reference scale and the relative error."""
     g = gpu.detach().to("cpu").to(torch.float64).numpy() if isinstance(gpu, torch.Tensor) else np.asarray(gpu, np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (what, g.shape, r.shape)
     mask = ~np.isnan(r)
     assert np.isfinite(g[mask]).all(), f"{what}: non-finite GPU values"
     err = np.abs(g[mask] - r[mask]).max() if mask.any() else 0.0
+    rmax = np.abs(r[mask]).max() if mask.any() else 0.0
+    if verbose:
+        print(f"[parity] {what}: max|diff| {err:.3e}, max|ref| {rmax:.3e}, "
+              f"rel {err / max(rmax, 1e-30):.3e}")
     if dtype == "bf16":
-        bound = BF16_ABS
+        bound = min(BF16_ABS, BF16_REL * max(rmax, 1e-30))
     else:
-        bound = F32_REL * max(np.abs(r[mask]).max() if mask.any() else 0.0, 1e-30)
-    assert err <= bound, f"{what}: max |diff| {err:.3e} > {bound:.3e}"
+        bound = F32_REL * max(rmax, 1e-30)
+    assert err <= bound, f"{what}: max |diff| {err:.3e} > {bound:.3e} (max |ref| {rmax:.3e})"
     return err
 
 

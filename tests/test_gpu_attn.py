@@ -54,8 +54,8 @@ def _case(dsv4, *, B, nq, H, c, m, w, k, dtype, pos0=None, R=None, sink=False, d
                                 None if dense else counts.numpy(), local, pos0, w, sk, scale,
                                 dense_m=m if dense else 0, queries=positions)
     bi = tuple(np.array(positions).T)
-    assert_close(Og.cpu()[bi], Or, dtype, what + " O")
-    assert_close(Lg.cpu()[bi], Lr, "f32" if dtype == "f32" else "bf16", what + " LSE")
+    assert_close(Og.cpu()[bi], Or, dtype, what + " O", verbose=True)
+    assert_close(Lg.cpu()[bi], Lr, "f32" if dtype == "f32" else "bf16", what + " LSE", verbose=True)
 
 
 def test_attn_tiny_fp32_csa(dsv4):
@@ -73,15 +73,11 @@ def test_attn_tiny_fp32_sink(dsv4):
     _case(dsv4, B=2, nq=100, H=4, c=64, m=4, w=16, k=8, dtype="f32", sink=True, what="sink")
 
 
-@pytest.fixture(params=["tc_cluster", "tc_single_cta", "tc_double_buffer", "cuda_cores"])
+@pytest.fixture(params=["tensor_cores", "cuda_cores"])
 def attn_path(request, monkeypatch):
-    """Run a case on each attention kernel: the 2-CTA-cluster tcgen05 kernel, the single-CTA
-    tcgen05 kernel with 128-slot blocks, the double-buffered one with 64-slot blocks (all
-    bf16, c=512, H%64==0) and the CUDA-core kernel. Split lists (decode) always take the
-    128-slot kernel."""
+    """Run a case on each attention kernel: the tcgen05 kernel (bf16, c=512, H%64==0; split
+    candidate lists when the request has fewer items than SMs) and the CUDA-core kernel."""
     monkeypatch.setenv("DSV4_FORCE_SIMT", "1" if request.param == "cuda_cores" else "0")
-    monkeypatch.setenv("DSV4_ATTN_CLUSTER", "1" if request.param == "tc_cluster" else "0")
-    monkeypatch.setenv("DSV4_ATTN_DB", "1" if request.param == "tc_double_buffer" else "0")
     return request.param
 
 
@@ -119,12 +115,16 @@ def test_attn_decode_ring(dsv4, attn_path):
           pos0=[L - 1 for L in lens], R=128, q_std=1.0, what="decode hca")
 
 
-def test_attn_flash_full_sampled(dsv4, attn_path):
-    """V4-Flash CSA prefill shape (n=8192, H=64, c=512, k=512, w=128, sink) -- sampled."""
+@pytest.mark.parametrize("unit", [False, True], ids=["model_scale", "unit_scale"])
+def test_attn_flash_full_sampled(dsv4, attn_path, unit):
+    """V4-Flash CSA prefill shape (n=8192, H=64, c=512, k=512, w=128, sink) -- sampled; at
+    the workload's scale (N(0,1)/sqrt(c)) and at unit scale (logits of std 1), where a wrong
+    row set or a zeroed output cannot hide under the absolute bound."""
     s = preset("flash_csa_prefill")
     pos = [(0, t) for t in sample_positions(s.n, 4, extra=[2046, 2047, 2048, 127, 128])]
     _case(dsv4, B=1, nq=s.n, H=64, c=512, m=4, w=128, k=512, dtype="bf16", sink=True,
-          kv_std=1 / math.sqrt(512), positions=pos, what="flash full")
+          q_std=1.0 if unit else None, kv_std=1.0 if unit else 1 / math.sqrt(512), positions=pos,
+          what="flash full" + (" unit" if unit else ""))
 
 
 def test_attn_out_of_range_index_is_flagged(dsv4, attn_path):
