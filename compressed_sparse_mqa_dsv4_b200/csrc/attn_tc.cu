@@ -46,7 +46,10 @@ constexpr int AT_H = 64;
 constexpr int AT_BLK = 128;
 constexpr int AT_CHUNKS = AT_C / 64;
 constexpr int AT_SOFT = 256;
-constexpr int AT_PROD = 128;
+constexpr int AT_PROD_WARPS = 4;                   // 6 were measured slower
+constexpr int AT_PROD = 32 * AT_PROD_WARPS;
+constexpr int AT_WATCH_WARP = 8 + AT_PROD_WARPS;   // warps 0-7 softmax, then the producers
+constexpr int AT_MMA_WARP = AT_WATCH_WARP + 1;
 constexpr int AT_THREADS = AT_SOFT + AT_PROD + 64;
 // Named barriers: 1-3 softmax warps, 5 producers, and the producer/watcher gates.
 constexpr uint32_t GATE_ITEM = 10;
@@ -214,7 +217,6 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int item, int h
 template <bool kSplit>
 __global__ void __maxnreg__(128)
     attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q,
-                   const __grid_constant__ CUtensorMap map_local,
                    const __grid_constant__ CUtensorMap map_o, int head_groups,
                    int items, float scale_log2, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
@@ -236,7 +238,7 @@ __global__ void __maxnreg__(128)
     tc::fence_barrier_init();
   }
   if (tid < AT_H) s.mcur[tid] = -INFINITY;
-  if (warp == 13) {
+  if (warp == AT_MMA_WARP) {
     tc::tmem_alloc(&s.tmem_base, TM_COLS);
     tc::tmem_relinquish();
   }
@@ -272,7 +274,7 @@ __global__ void __maxnreg__(128)
   // blocks and items the producers loaded (their bulk copies are drained before exit)
   uint32_t prod_G = 0;
   int prod_k = 0;
-  if (warp >= 8 && warp < 12) {
+  if (warp >= 8 && warp < AT_WATCH_WARP) {
     // ------------------------------------------------------------------ producer (4 warps)
     const int pt = tid - AT_SOFT;
     const uint64_t pool_addr = reinterpret_cast<uint64_t>(a.pool);
@@ -292,25 +294,12 @@ __global__ void __maxnreg__(128)
         for (int c = 0; c < AT_CHUNKS; ++c) tc::tma_load_2d(s.q[c], &map_q, &s.q_full, 64 * c, qrow);
       }
       for (int j = it.jb; j < it.je && ok; ++j, ++G) {
-        // Local-window slots of this block whose rows are contiguous (no ring wrap) and start
-        // on a 32-slot boundary come in by 2D TMA boxes of 32 rows; the rest by cp.async.
+        // Every slot of the block comes in by cp.async, local-window rows included (2D TMA
+        // boxes of 32 contiguous window rows were measured slower here: the TMA issue of
+        // small boxes paced the window block's gather at about half the cp.async rate).
         const int bs = j * AT_BLK;
-        int ls = it.nc4 - bs;
-        if (ls < 0) ls = 0;
-        bool tma_win = false;
-        long long first_row = 0;
-        if (ls < AT_BLK && (ls & 31) == 0) {
-          const long long jl0 = bs + ls - it.nc4;         // window index of slot ls
-          if (jl0 < it.cs.n_local) {
-            const long long p0 = it.cs.win0 + jl0;
-            const long long last = it.cs.win0 + it.cs.n_local - 1;
-            tma_win = (p0 % a.R) + (last - p0) < a.R;
-            first_row = it.cs.local_base + p0 % a.R;
-          }
-        }
-        const int cp_end = tma_win ? ls : AT_BLK;        // slots [0, cp_end) by cp.async
         // the block's row addresses (one index load per slot)
-        for (int u = pt; u < cp_end; u += AT_PROD) {
+        for (int u = pt; u < AT_BLK; u += AT_PROD) {
           const SlotRow r = slot_row(a, it.cs, it.nc4, bs + u);
           if (r.bad_index) flag_status(DSV4_ERR_DEVICE_BOUNDS);
           s.rowaddr[u] = (r.part == 0 && r.valid)
@@ -321,7 +310,7 @@ __global__ void __maxnreg__(128)
         if (pt == 0) A1_TRACE(0, k, j);
         // this thread's copies of every chunk: rows/pieces e = pt + 96 i (same for each chunk)
         constexpr int NPER = (AT_BLK * 8 + AT_PROD - 1) / AT_PROD;
-        const int ncopy = cp_end * 8;
+        constexpr int ncopy = AT_BLK * 8;
         uint64_t src[NPER];
         uint32_t dsto[NPER];
 #pragma unroll
@@ -340,20 +329,11 @@ __global__ void __maxnreg__(128)
             // queue behind this thread's own cp.async traffic and starve the gather.
             if (G > 0) pair_sync(GATE_PAIR0 + (c >> 1));
             if (pt == 0) A1_TRACE(8 + (c >> 1), k, j);
-            if (tma_win && pt == 0) {
-              tc::mbar_expect_tx(&s.ch_full[c | 3], 2 * (AT_BLK - ls) * 128);
-            }
           }
-          uint8_t* dst = s.kv[c];
 #pragma unroll
           for (int i = 0; i < NPER; ++i)
             if (pt + AT_PROD * i < ncopy)
               cp_async16(kv0 + (uint32_t)(c * AT_BLK * 128) + dsto[i], src[i] + (uint64_t)(128 * c));
-          if (tma_win && pt == 0) {
-            for (int r0 = ls; r0 < AT_BLK; r0 += 32)
-              tc::tma_load_2d(dst + r0 * 128, &map_local, &s.ch_full[c | 3], 64 * c,
-                              (int32_t)(first_row + (r0 - ls)));
-          }
           // One completion arrival per four chunks: each such arrival stalls the issuing
           // thread for a few hundred cycles (measured), so per-chunk arrivals throttled the
           // gather; GEMM1 then consumes the block in two halves.
@@ -366,7 +346,7 @@ __global__ void __maxnreg__(128)
       ++k;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-  } else if (warp == 12) {
+  } else if (warp == AT_WATCH_WARP) {
     // ------------------------------------------------------------------ watcher
     // Performs the producers' mbarrier waits and passes each result on; both sides take
     // the same sequence of gates (one per item, four per block after the first).
@@ -398,7 +378,7 @@ __global__ void __maxnreg__(128)
         }
       }
     }
-  } else if (warp == 13) {
+  } else if (warp == AT_MMA_WARP) {
     // ------------------------------------------------------------------ MMA issuer (converged)
     {
       const uint32_t id1 = tc::idesc_bf16_f32(128, AT_H, 0, 0);   // A, B K-major
@@ -746,13 +726,13 @@ __global__ void __maxnreg__(128)
   }
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 13) {
+  if (warp == AT_MMA_WARP) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, TM_COLS);
   }
   if (tid == AT_SOFT && *abort) {
     // After an abort (final now: every thread has passed the barrier) the last item's Q and
-    // the last block's TMA boxes and cp.async arrivals may still be landing: let them land
+    // the last block's cp.async arrivals may still be landing: let them land
     // before the CTA's shared memory is released. Without an abort they were all consumed.
     if (prod_k > 0) tc::mbar_drain(&s.q_full, (uint32_t)((prod_k - 1) & 1));
     if (prod_G > 0)
@@ -843,15 +823,12 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   }
   const long long nrows_local = (long long)a.B * a.R;
   if (nrows_local >= (1ll << 31) || !aligned16(a.O)) return DSV4_OK;
-  CUtensorMap mq, mlocal, mo;
+  CUtensorMap mq, mo;
   int s = encode_tensor_map_2d(&mq, a.Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_q, 64,
                                AT_H, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
   s = encode_tensor_map_2d(&mo, a.O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_q, 64, AT_H,
                            CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != DSV4_OK) return s;
-  s = encode_tensor_map_2d(&mlocal, a.local, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_local,
-                           64, 32, CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
   // Few (query, head group) items: split each candidate list so that about one and a half
   // work items per SM exist, as far as the caller's workspace (a.nsplit = its capacity)
@@ -878,10 +855,10 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   const long long grid = (nsplit > 1 || work < sms) ? work : sms;
   if (nsplit > 1)
     attn_tc_kernel<true><<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(
-        a, mq, mlocal, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
+        a, mq, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
   else
     attn_tc_kernel<false><<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(
-        a, mq, mlocal, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
+        a, mq, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
   *used = true;
   int s2 = launch_status("hybrid attention (tensor cores)");
   if (s2 != DSV4_OK || nsplit == 1) return s2;
