@@ -22,6 +22,7 @@ __all__ = [
     "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
     "dsv4_index_topk_workspace_size_ex",
     "dsv4_hybrid_sparse_attn", "dsv4_hybrid_sparse_attn_workspace_size", "dsv4_check_errors",
+    "dsv4_norm_rope",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsv4.so")
@@ -62,6 +63,10 @@ lib.dsv4_index_topk_noalloc.argtypes = [_I, _P, _P, _P, _P, _P, _L, _P, _P, _I, 
 lib.dsv4_hybrid_sparse_attn.restype = _I
 lib.dsv4_hybrid_sparse_attn.argtypes = [_I, _P, _P, _L, _P, _P, _P, _I, _P, _I, _P, _I, _I, _I,
                                         _I, _I, _I, _P, _F, _P, _P, _P, _S, _P]
+lib.dsv4_hybrid_sparse_attn_rope.restype = _I
+lib.dsv4_hybrid_sparse_attn_rope.argtypes = lib.dsv4_hybrid_sparse_attn.argtypes[:-1] + [_I, _P]
+lib.dsv4_norm_rope.restype = _I
+lib.dsv4_norm_rope.argtypes = [_I, _P, _P, _L, _I, _I, _I, _I, _I, _F, _P]
 lib.dsv4_hybrid_sparse_attn_workspace_size.restype = _S
 lib.dsv4_hybrid_sparse_attn_workspace_size.argtypes = [_I, _I, _I, _I]
 
@@ -237,13 +242,15 @@ def dsv4_hybrid_sparse_attn(Q: torch.Tensor, pool: torch.Tensor, kv_row_off: tor
                             sink: Optional[torch.Tensor] = None, scale: Optional[float] = None,
                             O: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                             want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
-                            stream=None):
+                            rope_dims: int = 0, stream=None):
     """Hybrid shared-KV MQA. Q [B, nq, H, c]; pool [rows, c]; local [B, R, c].
 
     idx/counts: int32 [B, nq, k] / [B, nq] (CSA) or None (HCA dense read with ratio m).
     Returns (O [B, nq, H, c], lse fp32 [B, nq, H] or None).
     workspace: uint8 device scratch for split candidate lists (decode); allocated here when
     the request would use it and none is given.
+    rope_dims > 0: the output's last rope_dims channels are rotated back by each query's
+    position (dsv4_hybrid_sparse_attn_rope).
     """
     _dev(Q, "Q"), _dev(pool, "pool", Q.dtype), _dev(local, "local", Q.dtype)
     _dev(kv_row_off, "kv_row_off", torch.int64), _dev(q_pos0, "q_pos0", torch.int32)
@@ -269,13 +276,29 @@ def dsv4_hybrid_sparse_attn(Q: torch.Tensor, pool: torch.Tensor, kv_row_off: tor
     if ws_bytes and (workspace is None or workspace.numel() < ws_bytes):
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=Q.device)
     ws_bytes = workspace.numel() if workspace is not None else 0
-    _check(lib.dsv4_hybrid_sparse_attn(_code(Q.dtype), _ptr(Q), _ptr(pool), pool.shape[0],
-                                       _ptr(kv_row_off), idx_p, _ptr(counts), k, _ptr(local),
-                                       R, _ptr(q_pos0), B, nq, H, c, m, w, _ptr(sink),
-                                       float(scale), _ptr(O), _ptr(lse), _ptr(workspace),
-                                       ws_bytes, _stream(stream)),
-           "dsv4_hybrid_sparse_attn")
+    args = (_code(Q.dtype), _ptr(Q), _ptr(pool), pool.shape[0], _ptr(kv_row_off), idx_p,
+            _ptr(counts), k, _ptr(local), R, _ptr(q_pos0), B, nq, H, c, m, w, _ptr(sink),
+            float(scale), _ptr(O), _ptr(lse), _ptr(workspace), ws_bytes)
+    if rope_dims:
+        _check(lib.dsv4_hybrid_sparse_attn_rope(*args, rope_dims, _stream(stream)),
+               "dsv4_hybrid_sparse_attn_rope")
+    else:
+        _check(lib.dsv4_hybrid_sparse_attn(*args, _stream(stream)), "dsv4_hybrid_sparse_attn")
     return O, lse
+
+
+def dsv4_norm_rope(x: torch.Tensor, pos: torch.Tensor, rows_per_pos: int = 1, rope: int = 64,
+                   norm: bool = True, inverse: bool = False, eps: float = 1e-6,
+                   stream=None) -> torch.Tensor:
+    """In place on x [..., c]: RMS-normalise each row (norm) and rotate its last `rope`
+    channels by pos[row // rows_per_pos] (inverse: by minus the angle). Returns x."""
+    _dev(x, "x"), _dev(pos, "pos", torch.int32)
+    c = x.shape[-1]
+    rows = x.numel() // max(c, 1)
+    _check(lib.dsv4_norm_rope(_code(x.dtype), _ptr(x), _ptr(pos), rows, rows_per_pos, c, rope,
+                              1 if norm else 0, 1 if inverse else 0, float(eps), _stream(stream)),
+           "dsv4_norm_rope")
+    return x
 
 
 def dsv4_hybrid_sparse_attn_workspace_size(B: int, nq: int, H: int, c: int) -> int:

@@ -1,6 +1,7 @@
 // Shared declarations of the hybrid sparse attention kernels.
 #pragma once
 #include "dsv4_common.cuh"
+#include "rope.cuh"
 
 namespace dsv4 {
 
@@ -20,6 +21,9 @@ struct AttnArgs {
   float scale;
   void* O;
   float* lse;
+  // > 0: rotate the output's last rope_out channels back by the query's position (inverse
+  // RoPE of "CSA And HCA: Definition, State, And Cost Model", s5.2) before it is stored
+  int rope_out;
   // split candidate lists (tensor-core path): nsplit partials per (query, head group) in
   // part_o [items * nsplit][64 heads][c] fp32 and part_ml [items * nsplit][64] (m, L)
   int nsplit;

@@ -137,22 +137,41 @@ __global__ void __launch_bounds__(AS_THREADS) attn_simt_kernel(AttnArgs a) {
     }
   }
   __syncthreads();
-  if (ah < hn) {
-    float mx = mrun[ah], den = lrun[ah];
-    if (a.sink) {
-      const float s = a.sink[h0 + ah];
-      const float mnew = fmaxf(mx, s);
-      den = den * expf(mx - mnew) + expf(s - mnew);
+  float mx = mrun[ah], den = lrun[ah];
+  if (ah < hn && a.sink) {
+    const float s = a.sink[h0 + ah];
+    const float mnew = fmaxf(mx, s);
+    den = den * expf(mx - mnew) + expf(s - mnew);
 #pragma unroll
-      for (int u = 0; u < AS_MAXC / 16; ++u) acc[u] *= expf(mx - mnew);
-      mx = mnew;
+    for (int u = 0; u < AS_MAXC / 16; ++u) acc[u] *= expf(mx - mnew);
+    mx = mnew;
+  }
+  const float inv = ah < hn ? 1.f / den : 0.f;
+#pragma unroll
+  for (int u = 0; u < AS_MAXC / 16; ++u) acc[u] *= inv;
+  if (a.rope_out) {
+    // inverse RoPE of the last rope_out channels at the query's position: the partner of
+    // channel d (= ac + 16u) is d^1, held by thread ac^1 (c even, so both lie below c)
+    const long long tpos = (long long)a.q_pos0[b] + i;
+#pragma unroll
+    for (int u = 0; u < AS_MAXC / 16; ++u) {
+      if (u < nu) {
+        const int d = ac + 16 * u;
+        const float other = __shfl_xor_sync(0xffffffffu, acc[u], 1);
+        if (d < c && d >= c - a.rope_out) {
+          float cs, sn;
+          rope_cos_sin(tpos, (d - (c - a.rope_out)) >> 1, a.rope_out, cs, sn);
+          acc[u] = (d & 1) ? fmaf(acc[u], cs, -other * sn) : fmaf(acc[u], cs, other * sn);
+        }
+      }
     }
-    const float inv = 1.f / den;
+  }
+  if (ah < hn) {
     T* O = reinterpret_cast<T*>(a.O) + ((long long)qi * a.H + h0 + ah) * c;
 #pragma unroll
     for (int u = 0; u < AS_MAXC / 16; ++u) {
       const int d = ac + 16 * u;
-      if (u < nu && d < c) O[d] = from_f32<T>(acc[u] * inv);
+      if (u < nu && d < c) O[d] = from_f32<T>(acc[u]);
     }
     if (a.lse && ac == 0) a.lse[(long long)qi * a.H + h0 + ah] = mx + logf(den);
   }

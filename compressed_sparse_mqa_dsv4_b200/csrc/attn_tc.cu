@@ -72,6 +72,7 @@ struct AttnSmem {
   float moff[AT_H];                         // exp2 offset: mcur, or 0 while mcur = -inf
   float fac[AT_H];
   float inv[AT_H];
+  float rcos[32], rsin[32];                 // inverse RoPE of O: the item's pair angles
   uint64_t rowaddr[AT_BLK];
   uint64_t q_full, q_empty;
   uint64_t ch_full[AT_CHUNKS], ch_empty[4];  // ch_full[3], ch_full[7]: chunks 0-3, 4-7 landed
@@ -662,6 +663,11 @@ __global__ void __maxnreg__(128)
         if (a.lse) a.lse[(long long)it.qi * a.H + h0 + h] = lse;
         s.mcur[h] = -INFINITY;                         // the next item starts fresh
       }
+      if (a.rope_out && tid < 32) {                    // pair tid of the last 64 channels
+        const int qb = it.qi / a.nq;
+        const long long tpos = (long long)a.q_pos0[qb] + (it.qi - qb * a.nq);
+        rope_cos_sin(tpos, tid, 64, s.rcos[tid], s.rsin[tid]);
+      }
       tc::named_barrier(1, AT_SOFT);
       if (tid == 0) A1_TRACE(22, k, 0);
       // O^T tiles of 128 channels. Each warp reads its 32 channels x 32 heads as two 16-lane
@@ -684,8 +690,29 @@ __global__ void __maxnreg__(128)
           tc::tmem_wait_ld_dep16(v);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            pk[hh][2 * kk] = pack_bf16(v[4 * kk] * inv2[kk].x, v[4 * kk + 1] * inv2[kk].y);
-            pk[hh][2 * kk + 1] = pack_bf16(v[4 * kk + 2] * inv2[kk].x, v[4 * kk + 3] * inv2[kk].y);
+            v[4 * kk] *= inv2[kk].x;
+            v[4 * kk + 1] *= inv2[kk].y;
+            v[4 * kk + 2] *= inv2[kk].x;
+            v[4 * kk + 3] *= inv2[kk].y;
+          }
+          if (a.rope_out && q == 3 && quad >= 2) {
+            // channels 448..511 (TMEM lanes 64..127 of the last M-tile): the pair partner of
+            // lane L is lane L^1, held by thread lane^4 in the same register
+            const bool odd = (lane >> 2) & 1;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+              const float other = __shfl_xor_sync(0xffffffffu, v[r], 4);
+              const int ch = 32 * quad + 16 * hh + (lane >> 2) + 8 * ((r & 3) >> 1);   // 64..127
+              const int pr = (ch - 64) >> 1;
+              const float cs = s.rcos[pr], sn = s.rsin[pr];
+              // rotation by minus the angle: a' = a cos + b sin, b' = b cos - a sin
+              v[r] = odd ? fmaf(v[r], cs, -other * sn) : fmaf(v[r], cs, other * sn);
+            }
+          }
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            pk[hh][2 * kk] = pack_bf16(v[4 * kk], v[4 * kk + 1]);
+            pk[hh][2 * kk + 1] = pack_bf16(v[4 * kk + 2], v[4 * kk + 3]);
           }
         }
         if (q > 0) {                                   // the previous tile's stores read P
@@ -782,6 +809,16 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(const AttnArgs a, int
         acc[4 * v + 3] = fmaf(es, x.w, acc[4 * v + 3]);
       }
     }
+    if (a.rope_out && lane >= (AT_C - 64) / 16) {      // channels 448..511: inverse RoPE
+      const int qb = qi / a.nq;
+      const long long tpos = (long long)a.q_pos0[qb] + (qi - qb * a.nq);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float cs, sn;
+        rope_cos_sin(tpos, 8 * (lane - (AT_C - 64) / 16) + j, 64, cs, sn);
+        rope_apply(acc[2 * j], acc[2 * j + 1], cs, sn, true);
+      }
+    }
     uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.O) +
                                           ((long long)qi * a.H + h) * AT_C + 16 * lane);
     dst[0] = make_uint4(pack_bf16(acc[0] * inv, acc[1] * inv), pack_bf16(acc[2] * inv, acc[3] * inv),
@@ -803,7 +840,7 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   *used = false;
   const char* force = std::getenv("DSV4_FORCE_SIMT");
   if (force && force[0] == '1') return DSV4_OK;
-  if (a.c != AT_C || a.H % AT_H != 0) return DSV4_OK;
+  if (a.c != AT_C || a.H % AT_H != 0 || (a.rope_out != 0 && a.rope_out != 64)) return DSV4_OK;
   if (!aligned16(a.Q) || !aligned16(a.local) || (a.pool && !aligned16(a.pool))) return DSV4_OK;
   const long long nrows_q = (long long)a.B * a.nq * a.H;
   const long long items = (long long)a.B * a.nq * (a.H / AT_H);

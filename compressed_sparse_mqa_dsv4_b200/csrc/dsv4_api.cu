@@ -297,15 +297,16 @@ extern "C" size_t dsv4_hybrid_sparse_attn_workspace_size(int B, int nq, int H, i
   return (size_t)round_up(items * ATTN_MAX_SPLIT * attn_split_bytes_per_item(c), 256);
 }
 
-extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* pool,
-                                       int64_t pool_rows, const int64_t* kv_row_off,
-                                       const int32_t* idx, const int32_t* counts, int k,
-                                       const void* local, int R, const int32_t* q_pos0, int B,
-                                       int nq, int H, int c, int m, int w, const float* sink,
-                                       float scale, void* O, float* lse, void* workspace,
-                                       size_t workspace_bytes, void* stream) {
+static int hybrid_sparse_attn(int dtype, const void* Q, const void* pool, int64_t pool_rows,
+                              const int64_t* kv_row_off, const int32_t* idx, const int32_t* counts,
+                              int k, const void* local, int R, const int32_t* q_pos0, int B,
+                              int nq, int H, int c, int m, int w, const float* sink, float scale,
+                              void* O, float* lse, void* workspace, size_t workspace_bytes,
+                              int rope_out, void* stream) {
   if (dtype != DSV4_F32 && dtype != DSV4_BF16)
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_hybrid_sparse_attn: dtype %d", dtype);
+  if (rope_out < 0 || rope_out > c || (rope_out & 1))
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_hybrid_sparse_attn_rope: rope_dims %d (c=%d)", rope_out, c);
   if (B < 0 || nq < 0 || H < 1 || c < 1 || m < 1 || w < 1 || R < 1 || pool_rows < 0 ||
       (idx && k < 0))
     return fail(DSV4_ERR_INVALID_ARG,
@@ -321,6 +322,7 @@ extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* poo
   a.counts = counts; a.k = idx ? k : 0; a.local = local; a.R = R; a.q_pos0 = q_pos0; a.B = B;
   a.nq = nq; a.H = H; a.c = c; a.m = m; a.w = w; a.sink = sink; a.scale = scale; a.O = O;
   a.lse = lse;
+  a.rope_out = rope_out;
   a.nsplit = 1;
   a.part_o = nullptr;
   a.part_ml = nullptr;
@@ -346,4 +348,29 @@ extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* poo
   }
   trace_path("hybrid attention: CUDA cores");
   return launch_attn_simt(a, dtype, st);
+}
+
+extern "C" int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* pool,
+                                       int64_t pool_rows, const int64_t* kv_row_off,
+                                       const int32_t* idx, const int32_t* counts, int k,
+                                       const void* local, int R, const int32_t* q_pos0, int B,
+                                       int nq, int H, int c, int m, int w, const float* sink,
+                                       float scale, void* O, float* lse, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  return hybrid_sparse_attn(dtype, Q, pool, pool_rows, kv_row_off, idx, counts, k, local, R,
+                            q_pos0, B, nq, H, c, m, w, sink, scale, O, lse, workspace,
+                            workspace_bytes, 0, stream);
+}
+
+extern "C" int dsv4_hybrid_sparse_attn_rope(int dtype, const void* Q, const void* pool,
+                                            int64_t pool_rows, const int64_t* kv_row_off,
+                                            const int32_t* idx, const int32_t* counts, int k,
+                                            const void* local, int R, const int32_t* q_pos0,
+                                            int B, int nq, int H, int c, int m, int w,
+                                            const float* sink, float scale, void* O, float* lse,
+                                            void* workspace, size_t workspace_bytes,
+                                            int rope_dims, void* stream) {
+  return hybrid_sparse_attn(dtype, Q, pool, pool_rows, kv_row_off, idx, counts, k, local, R,
+                            q_pos0, B, nq, H, c, m, w, sink, scale, O, lse, workspace,
+                            workspace_bytes, rope_dims, stream);
 }

@@ -263,6 +263,41 @@ int dsv4_hybrid_sparse_attn(int dtype, const void* Q, const void* pool, int64_t 
                             const float* sink, float scale, void* O, float* lse,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * dsv4_hybrid_sparse_attn_rope -- dsv4_hybrid_sparse_attn with the output side of the
+ * [CSA-DEF] s5.2 contract fused in: the last rope_dims channels of every output row O_{t,h}
+ * are rotated back by the query's position t (inverse RoPE; the channel pairing and angles
+ * of dsv4_norm_rope) before O is stored. Q, pool and local hold rows that dsv4_norm_rope
+ * (or an upstream kernel) already normalised and rotated: the query at t, compressed entry
+ * s at m*s (m' for HCA), local entry j at j. LSE is unchanged by the rotation.
+ *   rope_dims  even, 0 <= rope_dims <= c (0: same as dsv4_hybrid_sparse_attn). The tensor-core
+ *              path takes rope_dims = 64 at c = 512; other values run on CUDA cores.
+ * All other arguments, layouts and errors are those of dsv4_hybrid_sparse_attn.
+ */
+int dsv4_hybrid_sparse_attn_rope(int dtype, const void* Q, const void* pool, int64_t pool_rows,
+                                 const int64_t* kv_row_off, const int32_t* idx,
+                                 const int32_t* counts, int k, const void* local, int R,
+                                 const int32_t* q_pos0, int B, int nq, int H, int c, int m, int w,
+                                 const float* sink, float scale, void* O, float* lse,
+                                 void* workspace, size_t workspace_bytes, int rope_dims,
+                                 void* stream);
+
+/*
+ * dsv4_norm_rope -- [CSA-DEF] s5.2: RMS normalisation of attention rows and rotary position
+ * embedding of their last `rope` channels, in place. For each row r of x [rows, c]:
+ *   norm = 1:  x_r <- x_r / sqrt(mean(x_r^2) + eps)      (fp32, no learned gain)
+ *   then channel pair i (channels c - rope + 2i, c - rope + 2i + 1) is rotated by the angle
+ *   p * 10000^(-2i / rope), p = pos[r / rows_per_pos] (inverse = 1: by minus that angle).
+ * The angle is formed and reduced in double precision; the result is rounded once to dtype.
+ * Uses: query heads (rows_per_pos = H, pos = query positions), compressed entries (pos = m*s),
+ * local entries (pos = j), and the inverse rotation of an output (norm = 0, inverse = 1).
+ *   dtype  DSV4_F32 or DSV4_BF16.   pos  int32 [ceil(rows / rows_per_pos)], >= 0 (a negative
+ *   position skips its rows and sets DSV4_ERR_DEVICE_BOUNDS).
+ *   Requires rows >= 0, rows_per_pos >= 1, c >= 1, 0 <= rope <= c, rope even, eps >= 0.
+ */
+int dsv4_norm_rope(int dtype, void* x, const int32_t* pos, int64_t rows, int rows_per_pos, int c,
+                   int rope, int norm, int inverse, float eps, void* stream);
+
 /* Workspace bytes for dsv4_hybrid_sparse_attn to split every candidate list of a request of
  * B x nq queries with H heads of dimension c (0 when no split would be used). */
 size_t dsv4_hybrid_sparse_attn_workspace_size(int B, int nq, int H, int c);
