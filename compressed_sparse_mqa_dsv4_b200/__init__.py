@@ -22,7 +22,9 @@ __all__ = [
     "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
     "dsv4_index_topk_workspace_size_ex",
     "dsv4_hybrid_sparse_attn", "dsv4_hybrid_sparse_attn_workspace_size", "dsv4_check_errors",
-    "dsv4_norm_rope",
+    "dsv4_norm_rope", "dsv4_quantize_main_kv", "dsv4_dequantize_main_kv",
+    "dsv4_compress_decode_fp8", "dsv4_hybrid_sparse_attn_fp8",
+    "dsv4_hybrid_sparse_attn_fp8_workspace_size",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libdsv4.so")
@@ -67,6 +69,18 @@ lib.dsv4_hybrid_sparse_attn_rope.restype = _I
 lib.dsv4_hybrid_sparse_attn_rope.argtypes = lib.dsv4_hybrid_sparse_attn.argtypes[:-1] + [_I, _P]
 lib.dsv4_norm_rope.restype = _I
 lib.dsv4_norm_rope.argtypes = [_I, _P, _P, _L, _I, _I, _I, _I, _I, _F, _P]
+lib.dsv4_quantize_main_kv.restype = _I
+lib.dsv4_quantize_main_kv.argtypes = [_I, _P, _P, _P, _P, _L, _I, _I, _P]
+lib.dsv4_dequantize_main_kv.restype = _I
+lib.dsv4_dequantize_main_kv.argtypes = [_P, _P, _P, _P, _L, _I, _I, _P]
+lib.dsv4_compress_decode_fp8.restype = _I
+lib.dsv4_compress_decode_fp8.argtypes = [_I, _P, _P, _P, _P, _P, _P, _P, _I, _P, _L, _P, _I, _I, _I,
+                                         _I, _P]
+lib.dsv4_hybrid_sparse_attn_fp8_workspace_size.restype = _S
+lib.dsv4_hybrid_sparse_attn_fp8_workspace_size.argtypes = [_I, _I, _I, _I]
+lib.dsv4_hybrid_sparse_attn_fp8.restype = _I
+lib.dsv4_hybrid_sparse_attn_fp8.argtypes = [_P, _P, _P, _P, _L, _P, _P, _P, _I, _P, _I, _P, _I, _I,
+                                            _I, _I, _I, _I, _P, _F, _P, _P, _P, _S, _P]
 lib.dsv4_hybrid_sparse_attn_workspace_size.restype = _S
 lib.dsv4_hybrid_sparse_attn_workspace_size.argtypes = [_I, _I, _I, _I]
 
@@ -308,3 +322,88 @@ def dsv4_hybrid_sparse_attn_workspace_size(B: int, nq: int, H: int, c: int) -> i
 def dsv4_check_errors(stream=None):
     """Synchronise the stream and raise DSV4Error if a kernel flagged a device-side error."""
     _check(lib.dsv4_check_errors(_stream(stream)), "dsv4_check_errors")
+
+
+# ----------------------------------------------------------------------------- FP8 main-KV entries
+
+
+def dsv4_quantize_main_kv(x: torch.Tensor, rope: int = 64, stream=None):
+    """x [rows, c] (fp32 / bf16) -> (codes uint8 [rows, c-rope], scales fp32 [rows, (c-rope)/64],
+    rope bf16 [rows, rope]): the FP8 main-KV entry format."""
+    _dev(x, "x")
+    c = x.shape[-1]
+    rows = x.numel() // max(c, 1)
+    codes = torch.empty(rows, c - rope, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(rows, (c - rope) // 64, dtype=torch.float32, device=x.device)
+    rp = torch.empty(rows, rope, dtype=torch.bfloat16, device=x.device)
+    _check(lib.dsv4_quantize_main_kv(_code(x.dtype), _ptr(x), _ptr(codes), _ptr(scales), _ptr(rp),
+                                     rows, c, rope, _stream(stream)), "dsv4_quantize_main_kv")
+    return codes, scales, rp
+
+
+def dsv4_dequantize_main_kv(codes: torch.Tensor, scales: torch.Tensor, rope: torch.Tensor,
+                            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """FP8 entries -> bf16 rows [rows, c]."""
+    _dev(codes, "codes", torch.uint8), _dev(scales, "scales", torch.float32)
+    _dev(rope, "rope", torch.bfloat16)
+    rows, nf = codes.shape
+    r = rope.shape[-1]
+    if out is None:
+        out = torch.empty(rows, nf + r, dtype=torch.bfloat16, device=codes.device)
+    _check(lib.dsv4_dequantize_main_kv(_ptr(codes), _ptr(scales), _ptr(rope), _ptr(out), rows, nf + r,
+                                       r, _stream(stream)), "dsv4_dequantize_main_kv")
+    return out
+
+
+def dsv4_compress_decode_fp8(C_new, Z_new, bias, tail, codes, scales, rope, pool_row_off, pos, m: int,
+                             overlap: bool, stream=None) -> None:
+    """dsv4_compress_decode emitting completed entries into an FP8 pool (codes, scales, rope)."""
+    _dev(C_new, "C_new"), _dev(Z_new, "Z_new", C_new.dtype), _dev(bias, "bias", torch.float32)
+    _dev(tail, "tail", C_new.dtype), _dev(codes, "codes", torch.uint8)
+    _dev(scales, "scales", torch.float32), _dev(rope, "rope", torch.bfloat16)
+    _dev(pool_row_off, "pool_row_off", torch.int64), _dev(pos, "pos", torch.int32)
+    B, width = C_new.shape
+    S = 2 if overlap else 1
+    c = width // S
+    if tuple(tail.shape) != decode_tail_shape(B, c, m, overlap):
+        raise ValueError(f"tail must be {decode_tail_shape(B, c, m, overlap)}")
+    _check(lib.dsv4_compress_decode_fp8(_code(C_new.dtype), _ptr(C_new), _ptr(Z_new), _ptr(bias),
+                                        _ptr(tail), _ptr(codes), _ptr(scales), _ptr(rope),
+                                        rope.shape[-1], _ptr(pool_row_off), codes.shape[0], _ptr(pos),
+                                        B, c, m, 1 if overlap else 0, _stream(stream)),
+           "dsv4_compress_decode_fp8")
+
+
+def dsv4_hybrid_sparse_attn_fp8_workspace_size(B: int, H: int, c: int, k: int) -> int:
+    return int(lib.dsv4_hybrid_sparse_attn_fp8_workspace_size(B, H, c, k))
+
+
+def dsv4_hybrid_sparse_attn_fp8(Q, codes, scales, rope, kv_row_off, idx, counts, local, q_pos0,
+                                m: int, w: int, sink=None, scale=None, O=None, lse=None,
+                                workspace=None, stream=None):
+    """Decode attention over an FP8 pool. Q [B, 1, H, c] bf16; (codes, scales, rope) the pool;
+    idx/counts [B, 1, k] / [B, 1]; local [B, R, c] bf16. Returns (O, lse)."""
+    _dev(Q, "Q", torch.bfloat16), _dev(local, "local", torch.bfloat16)
+    _dev(codes, "codes", torch.uint8), _dev(scales, "scales", torch.float32)
+    _dev(rope, "rope", torch.bfloat16), _dev(idx, "idx", torch.int32), _dev(counts, "counts", torch.int32)
+    _dev(kv_row_off, "kv_row_off", torch.int64), _dev(q_pos0, "q_pos0", torch.int32)
+    B, nq, H, c = Q.shape
+    if nq != 1:
+        raise ValueError("dsv4_hybrid_sparse_attn_fp8 takes one query per sequence")
+    k = idx.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(c)
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None:
+        lse = torch.empty(B, 1, H, dtype=torch.float32, device=Q.device)
+    need = dsv4_hybrid_sparse_attn_fp8_workspace_size(B, H, c, k)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    _check(lib.dsv4_hybrid_sparse_attn_fp8(_ptr(Q), _ptr(codes), _ptr(scales), _ptr(rope), codes.shape[0],
+                                           _ptr(kv_row_off), _ptr(idx), _ptr(counts), k, _ptr(local),
+                                           local.shape[1], _ptr(q_pos0), B, H, c, rope.shape[-1], m, w,
+                                           _ptr(sink), float(scale), _ptr(O), _ptr(lse), _ptr(workspace),
+                                           workspace.numel(), _stream(stream)),
+           "dsv4_hybrid_sparse_attn_fp8")
+    return O, lse

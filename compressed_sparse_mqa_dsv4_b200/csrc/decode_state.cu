@@ -11,14 +11,21 @@
 // the prefill compressor: an online softmax in fp32 over the preceding block's stream-b
 // positions, then the current block's stream-a positions, in position order.
 #include "dsv4_common.cuh"
+#include "fp8_kv.cuh"
 
 namespace dsv4 {
 
-template <typename T>
+// The emitted entry goes to `pool` (dtype T), or -- FP8 -- through shared memory into the
+// production main-KV format (fp8_kv.cuh): the entry rounded to T, then quantised, so an FP8
+// pool holds exactly the quantisation of the T pool's row.
+template <typename T, bool FP8>
 __global__ void __launch_bounds__(256) compress_decode_kernel(
     const T* __restrict__ C_new, const T* __restrict__ Z_new, const float* __restrict__ bias,
     T* __restrict__ tail, T* __restrict__ pool, const int64_t* __restrict__ pool_row_off,
-    long long pool_rows, const int32_t* __restrict__ pos, int c, int m, int overlap) {
+    long long pool_rows, const int32_t* __restrict__ pos, int c, int m, int overlap,
+    uint8_t* __restrict__ codes, float* __restrict__ scales, __nv_bfloat16* __restrict__ rope_out,
+    int rope) {
+  extern __shared__ float entry[];                          // FP8: the entry, c values
   const int b = blockIdx.x;
   const int S = overlap ? 2 : 1;
   const int T_slots = S * m;
@@ -62,7 +69,24 @@ __global__ void __launch_bounds__(256) compress_decode_kernel(
         }
       }
     }
-    pool[row * c + ch] = from_f32<T>(acc / den);
+    if constexpr (FP8)
+      entry[ch] = to_f32(from_f32<T>(acc / den));
+    else
+      pool[row * c + ch] = from_f32<T>(acc / den);
+  }
+  if constexpr (FP8) {
+    __syncthreads();
+    const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int nf = c - rope, ng = nf / kFp8Group;
+    for (int g = threadIdx.x >> 5; g < ng; g += nw) {
+      const int ch = g * kFp8Group + 2 * lane;
+      uint32_t code2;
+      const float sc = fp8_group_quantize(entry[ch], entry[ch + 1], code2);
+      *reinterpret_cast<uint16_t*>(codes + row * nf + ch) = (uint16_t)code2;
+      if (lane == 0) scales[row * ng + g] = sc;
+    }
+    for (int d = threadIdx.x; d < rope; d += blockDim.x)
+      rope_out[row * rope + d] = __float2bfloat16_rn(entry[nf + d]);
   }
 }
 
@@ -97,13 +121,14 @@ extern "C" int dsv4_compress_decode(int dtype, const void* C_new, const void* Z_
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode: NULL pointer");
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == DSV4_F32)
-    compress_decode_kernel<float><<<B, 256, 0, st>>>(
+    compress_decode_kernel<float, false><<<B, 256, 0, st>>>(
         (const float*)C_new, (const float*)Z_new, bias, (float*)tail, (float*)pool, pool_row_off,
-        pool_rows, pos, c, m, overlap);
+        pool_rows, pos, c, m, overlap, nullptr, nullptr, nullptr, 0);
   else if (dtype == DSV4_BF16)
-    compress_decode_kernel<__nv_bfloat16><<<B, 256, 0, st>>>(
+    compress_decode_kernel<__nv_bfloat16, false><<<B, 256, 0, st>>>(
         (const __nv_bfloat16*)C_new, (const __nv_bfloat16*)Z_new, bias, (__nv_bfloat16*)tail,
-        (__nv_bfloat16*)pool, pool_row_off, pool_rows, pos, c, m, overlap);
+        (__nv_bfloat16*)pool, pool_row_off, pool_rows, pos, c, m, overlap, nullptr, nullptr,
+        nullptr, 0);
   else
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode: dtype %d not F32/BF16", dtype);
   return launch_status("dsv4_compress_decode");
@@ -125,4 +150,38 @@ extern "C" int dsv4_ring_write(int dtype, const void* kv_new, void* local, int R
   else
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_ring_write: dtype %d not F32/BF16", dtype);
   return launch_status("dsv4_ring_write");
+}
+
+extern "C" int dsv4_compress_decode_fp8(int dtype, const void* C_new, const void* Z_new,
+                                        const float* bias, void* tail, uint8_t* codes,
+                                        float* scales, void* rope_out, int rope,
+                                        const int64_t* pool_row_off, int64_t pool_rows,
+                                        const int32_t* pos, int B, int c, int m, int overlap,
+                                        void* stream) {
+  using namespace dsv4;
+  if (B < 0 || c < 1 || m < 1 || (overlap != 0 && overlap != 1) || pool_rows < 0 || rope < 0 ||
+      rope > c || (rope & 1) || (c - rope) % kFp8Group != 0 || c > 12 * 1024)
+    return fail(DSV4_ERR_INVALID_ARG,
+                "dsv4_compress_decode_fp8: bad sizes B=%d c=%d rope=%d m=%d overlap=%d pool_rows=%lld",
+                B, c, rope, m, overlap, (long long)pool_rows);
+  if (B == 0) return DSV4_OK;
+  if (!C_new || !Z_new || !bias || !tail || !codes || !scales || (rope > 0 && !rope_out) ||
+      !pool_row_off || !pos)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode_fp8: NULL pointer");
+  if (reinterpret_cast<uintptr_t>(codes) & 1u)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode_fp8: codes must be 2-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t smem = sizeof(float) * (size_t)c;
+  if (dtype == DSV4_F32)
+    compress_decode_kernel<float, true><<<B, 256, smem, st>>>(
+        (const float*)C_new, (const float*)Z_new, bias, (float*)tail, nullptr, pool_row_off,
+        pool_rows, pos, c, m, overlap, codes, scales, (__nv_bfloat16*)rope_out, rope);
+  else if (dtype == DSV4_BF16)
+    compress_decode_kernel<__nv_bfloat16, true><<<B, 256, smem, st>>>(
+        (const __nv_bfloat16*)C_new, (const __nv_bfloat16*)Z_new, bias, (__nv_bfloat16*)tail,
+        nullptr, pool_row_off, pool_rows, pos, c, m, overlap, codes, scales,
+        (__nv_bfloat16*)rope_out, rope);
+  else
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode_fp8: dtype %d not F32/BF16", dtype);
+  return launch_status("dsv4_compress_decode_fp8");
 }

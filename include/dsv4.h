@@ -298,6 +298,65 @@ int dsv4_hybrid_sparse_attn_rope(int dtype, const void* Q, const void* pool, int
 int dsv4_norm_rope(int dtype, void* x, const int32_t* pos, int64_t rows, int rows_per_pos, int c,
                    int rope, int norm, int inverse, float eps, void* stream);
 
+/*
+ * Production main-KV entries, [CSA-DEF] s8 precision table ("main KV: 448 FP8 + 64 BF16 RoPE
+ * channels"). The pages leave the FP8 scale metadata open; this library keeps one fp32 scale
+ * per 64 consecutive FP8 channels. A pool of `rows` entries of c channels whose last `rope`
+ * channels carry RoPE ((c - rope) % 64 == 0) is three caller-owned arrays:
+ *   codes   uint8 [rows, c - rope]  E4M3 (fn) bytes, sign << 7 | magnitude code
+ *   scales  fp32  [rows, (c - rope) / 64]
+ *   rope    bf16  [rows, rope]
+ * V4 shapes: c = 512, rope = 64 -> 448 + 28 + 128 = 604 bytes per entry (bf16: 1024).
+ */
+
+/* dsv4_quantize_main_kv -- rows x [rows, c] (dtype F32 or BF16) into the FP8 entry format:
+ * per 64-channel group scale = fp32(amax / 448), code = RNE_E4M3(fp32(x / scale)) saturating
+ * at 448 with the IEEE sign (a negative value that rounds to zero is 0x80); a zero scale gives
+ * zero codes; the RoPE channels are rounded to bf16. codes 2-byte aligned, x 4-byte aligned. */
+int dsv4_quantize_main_kv(int dtype, const void* x, uint8_t* codes, float* scales, void* rope,
+                          int64_t rows, int c, int rope_dims, void* stream);
+
+/* dsv4_dequantize_main_kv -- FP8 entries back to bf16 rows out [rows, c]: each FP8 channel is
+ * RNE_bf16(E4M3 value * scale) (the product carries up to 28 significant bits, so it is
+ * rounded once), the RoPE channels are copied. */
+int dsv4_dequantize_main_kv(const uint8_t* codes, const float* scales, const void* rope,
+                            void* out, int64_t rows, int c, int rope_dims, void* stream);
+
+/* dsv4_compress_decode_fp8 -- dsv4_compress_decode with the completed entry emitted in the
+ * FP8 entry format (quantise on emission, [CSA-DEF] s7 step 4 + s8): the entry is rounded to
+ * dtype and then quantised exactly as dsv4_quantize_main_kv would quantise that row, into
+ * row pool_row_off[b] + (t+1)/m - 1 of (codes, scales, rope). Tail, positions, errors and
+ * requirements are those of dsv4_compress_decode, plus (c - rope_dims) % 64 == 0 and
+ * c <= 12288. */
+int dsv4_compress_decode_fp8(int dtype, const void* C_new, const void* Z_new, const float* bias,
+                             void* tail, uint8_t* codes, float* scales, void* rope,
+                             int rope_dims, const int64_t* pool_row_off, int64_t pool_rows,
+                             const int32_t* pos, int B, int c, int m, int overlap, void* stream);
+
+/* Workspace bytes of dsv4_hybrid_sparse_attn_fp8: the gathered bf16 rows (B*k*c*2), their
+ * candidate lists and row offsets, and the split-list partials. */
+size_t dsv4_hybrid_sparse_attn_fp8_workspace_size(int B, int H, int c, int k);
+
+/*
+ * dsv4_hybrid_sparse_attn_fp8 -- decode attention (one query per sequence, t = q_pos0[b])
+ * over a compressed pool stored as FP8 entries: the selected entries idx[b, 0..counts[b])
+ * are read in the FP8 format (604 bytes per V4 entry instead of 1024), expanded to bf16 rows
+ * as in dsv4_dequantize_main_kv next to the query, and attended with the bf16 local ring
+ * exactly as dsv4_hybrid_sparse_attn attends bf16 rows (selected entries, then the window,
+ * one softmax, sink, LSE). Q, local, O: bf16 [B, H, c], [B, R, c], [B, H, c]; lse fp32 [B, H]
+ * or NULL. A selection outside [0, floor((t+1)/m)) or beyond pool_rows is skipped and
+ * reported (DSV4_ERR_DEVICE_BOUNDS). workspace: >= dsv4_hybrid_sparse_attn_fp8_workspace_size
+ * bytes, 256-byte aligned (DSV4_ERR_WORKSPACE otherwise). Requires k >= 1, w >= 1, R >= w,
+ * (c - rope_dims) % 64 == 0.
+ */
+int dsv4_hybrid_sparse_attn_fp8(const void* Q, const uint8_t* pool_codes, const float* pool_scales,
+                                const void* pool_rope, int64_t pool_rows,
+                                const int64_t* kv_row_off, const int32_t* idx,
+                                const int32_t* counts, int k, const void* local, int R,
+                                const int32_t* q_pos0, int B, int H, int c, int rope_dims, int m,
+                                int w, const float* sink, float scale, void* O, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* Workspace bytes for dsv4_hybrid_sparse_attn to split every candidate list of a request of
  * B x nq queries with H heads of dimension c (0 when no split would be used). */
 size_t dsv4_hybrid_sparse_attn_workspace_size(int B, int nq, int H, int c);
