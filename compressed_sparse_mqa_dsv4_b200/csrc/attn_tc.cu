@@ -123,6 +123,9 @@ __device__ __forceinline__ void pair_sync(uint32_t id) {
 __device__ __forceinline__ void cp_async16(uint32_t dst, uint64_t src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
+__device__ __forceinline__ void bulk_prefetch_l2(uint64_t src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(tc::smem_u32(bar))
                : "memory");
@@ -303,9 +306,22 @@ __global__ void __maxnreg__(128)
         for (int u = pt; u < AT_BLK; u += AT_PROD) {
           const SlotRow r = slot_row(a, it.cs, it.nc4, bs + u);
           if (r.bad_index) flag_status(DSV4_ERR_DEVICE_BOUNDS);
-          s.rowaddr[u] = (r.part == 0 && r.valid)
-                             ? pool_addr + (uint64_t)r.row * AT_C * 2
-                             : local_addr + (uint64_t)(r.part == 1 ? r.row : it.cs.local_base) * AT_C * 2;
+          const uint64_t ra = (r.part == 0 && r.valid)
+                                  ? pool_addr + (uint64_t)r.row * AT_C * 2
+                                  : local_addr + (uint64_t)(r.part == 1 ? r.row : it.cs.local_base) * AT_C * 2;
+          s.rowaddr[u] = ra;
+          if constexpr (kSplit) {
+            // Split lists (decode) read their rows from HBM: the next block's rows start
+            // toward L2 now, a block ahead of their gather (which waits for GEMM2 to free the
+            // buffer), and an item's first block its own rows.
+            if (j == it.jb) bulk_prefetch_l2(ra, AT_C * 2);
+            if (j + 1 < it.je) {
+              const SlotRow r2 = slot_row(a, it.cs, it.nc4, bs + AT_BLK + u);
+              if (r2.valid)
+                bulk_prefetch_l2((r2.part == 0 ? pool_addr : local_addr) + (uint64_t)r2.row * AT_C * 2,
+                                 AT_C * 2);
+            }
+          }
         }
         tc::named_barrier(5, AT_PROD);
         if (pt == 0) A1_TRACE(0, k, j);
