@@ -88,9 +88,11 @@ def test_attn_bf16_ragged(dsv4, attn_path, H, nq, k, w):
           what=f"{attn_path} H={H} nq={nq}")
 
 
-@pytest.mark.parametrize("scale_mul", [1.0, 4.0])
+@pytest.mark.parametrize("scale_mul", [1.0, 4.0, 16.0])
 def test_attn_bf16_stress_logits(dsv4, attn_path, scale_mul):
-    """Unscaled N(0,1) activations: logits with std 1 and 4 (peaky softmax)."""
+    """Unscaled N(0,1) activations: logits with std 1, 4 and 16 (peaky softmax; at 16 the
+    maxima of later blocks exceed the running max by far more than the kernel's bound, so
+    blocks are sent back for the exact path and accumulators rescaled)."""
     _case(dsv4, B=1, nq=600, H=64, c=512, m=4, w=128, k=64, dtype="bf16", sink=True,
           q_std=1.0, kv_std=1.0, scale=scale_mul / math.sqrt(512), seed=7,
           what=f"stress x{scale_mul}")
