@@ -37,9 +37,9 @@ UNIT = "tokens/s"
 # DRAM traffic of the attention kernel per launch, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the attention
 # sources it was measured on; reported as null once those sources change.
-ATTN_TRAFFIC = {"sources_sha1": "248722e89d10cce437e3ab7ed32df08169c2a504",
-                "bytes_per_launch": 562_623_488 + 494_860_544}
-ATTN_SOURCES = ("attn_common.cuh", "attn_tc.cu", "dsv4_common.cuh", "tc_common.cuh")
+ATTN_TRAFFIC = {"sources_sha1": "9890563d8dc0c640b60fdd719480dd30dc5e509d",
+                "bytes_per_launch": 562_333_440 + 494_402_048}
+ATTN_SOURCES = ("attn_common.cuh", "attn_tc.cu", "dsv4_common.cuh", "rope.cuh", "tc_common.cuh")
 
 
 def max_over_ranks(value: float, world: int, device) -> float:

@@ -1,13 +1,13 @@
 // dsv4_compress: learned softmax-gated pooling ("CSA And HCA: Definition, State, And Cost
 // Model", s2.1 overlapping two-stream CSA compressor, s2.2 one-stream HCA compressor).
 //
-// HBM-bound streaming pass. One thread owns one 16-byte channel vector (8 bf16 / 4 fp32
-// channels) of one output entry and walks the entry's positions with an online softmax
-// per channel (running max, running denominator, running weighted sum; all fp32).
+// HBM-bound streaming pass. One thread owns four consecutive channels of one output entry
+// and walks the entry's positions with an online softmax per channel (running max, running
+// denominator, running weighted sum; all fp32), with up to eight positions' loads in flight.
 // Reads every input byte once (stream a of block i by entry i, stream b of block i by
-// entry i+1), writes each entry once. Consecutive threads own consecutive channel
-// vectors of the same entry, so each position row is read as contiguous 16-byte
-// vectors across the warp.
+// entry i+1), writes each entry once. Consecutive threads own consecutive channel groups of
+// the same entry, so each position row is read contiguously across the warp. (Eight
+// channels per thread needed 189 registers, one CTA per SM and reached ~0.7 TB/s.)
 #include "dsv4_common.cuh"
 
 namespace dsv4 {
@@ -37,12 +37,43 @@ struct OnlinePool {
   }
 };
 
-// Vectorised kernel: requires c % V == 0 and 16-byte aligned C, Z, out, bias rows.
+// Four consecutive channels of T as raw bits (8 bytes of bf16, 16 of fp32), converted to fp32
+// only where they are consumed, so the loads in flight cost 2 (4) registers each.
+template <typename T> struct Raw4;
+template <> struct Raw4<__nv_bfloat16> {
+  uint2 r;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { r = __ldg(reinterpret_cast<const uint2*>(p)); }
+  __device__ __forceinline__ void to_f32(float (&v)[4]) const {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+  }
+};
+template <> struct Raw4<float> {
+  uint4 r;
+  __device__ __forceinline__ void load(const float* p) { r = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void to_f32(float (&v)[4]) const {
+    v[0] = __uint_as_float(r.x); v[1] = __uint_as_float(r.y); v[2] = __uint_as_float(r.z); v[3] = __uint_as_float(r.w);
+  }
+};
+
+__device__ __forceinline__ void store4(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, const float (&v)[4]) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]), b = __floats2bfloat162_rn(v[2], v[3]);
+  *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+}
+
+// Vectorised kernel: requires c % 4 == 0 and C, Z, out aligned to 4 elements, bias to 16
+// bytes. A thread owns 4 channels of one entry; CHUNK positions' C and Z vectors are loaded
+// before any is consumed (memory-level parallelism per thread) and stay raw until use, and the
+// bias is read at use: a small kernel, so that many CTAs per SM hide the rest of the latency.
 template <typename T, int CHUNK>
-__global__ void __launch_bounds__(256) compress_vec_kernel(
+__global__ void __launch_bounds__(256, 3) compress_vec_kernel(
     const T* __restrict__ C, const T* __restrict__ Z, const float* __restrict__ bias,
     T* __restrict__ out, int B, int n, int c, int m, int overlap, long long total_vecs) {
-  constexpr int V = Vec16<T>::N;
+  constexpr int V = 4;
   const int vecs_per_entry = c / V;
   const int E = n / m;
   const int S = overlap ? 2 : 1;
@@ -56,36 +87,47 @@ __global__ void __launch_bounds__(256) compress_vec_kernel(
     const int ch = v * V;
     OnlinePool<T, V> pool;
     pool.init();
-    // the preceding block from stream b (CSA, i > 0) then the current block from stream a
-    for (int half = (overlap && i > 0) ? 1 : 0; half >= 0; --half) {
-      const int tok0 = half ? m * (i - 1) : m * i;
-      const T* zrow = Z + ((long long)b * n + tok0) * row_stride + half * c + ch;
-      const T* crow = C + ((long long)b * n + tok0) * row_stride + half * c + ch;
-      const float* brow = bias + (long long)half * m * c + ch;
-      for (int p0 = 0; p0 < m; p0 += CHUNK) {
-        float z[CHUNK][V], x[CHUNK][V], bb[CHUNK][V];
-        const int cnt = min(CHUNK, m - p0);
+    // positions in order: the preceding block from stream b (CSA, i > 0), then the current
+    // block from stream a; flattened, so that a chunk of loads spans both blocks when m is
+    // small (CSA m = 4: all eight positions' loads are in flight at once)
+    const int mb = (overlap && i > 0) ? m : 0;
+    const long long tb = (long long)b * n + (long long)m * (i > 0 ? i - 1 : 0);
+    const T* zb = Z + tb * row_stride + c + ch;                                 // stream b rows
+    const T* cb = C + tb * row_stride + c + ch;
+    const T* za = Z + ((long long)b * n + m * i) * row_stride + ch;             // stream a rows
+    const T* ca = C + ((long long)b * n + m * i) * row_stride + ch;
+    const int P = mb + m;
+    for (int p0 = 0; p0 < P; p0 += CHUNK) {
+      Raw4<T> zr[CHUNK], xr[CHUNK];
 #pragma unroll
-        for (int u = 0; u < CHUNK; ++u) {
-          if (u < cnt) {
-            load16_f32(zrow + (long long)(p0 + u) * row_stride, z[u]);
-            load16_f32(crow + (long long)(p0 + u) * row_stride, x[u]);
-#pragma unroll
-            for (int j = 0; j < V; j += 4) {
-              float4 t = __ldg(reinterpret_cast<const float4*>(brow + (long long)(p0 + u) * c + j));
-              bb[u][j] = t.x; bb[u][j + 1] = t.y; bb[u][j + 2] = t.z; bb[u][j + 3] = t.w;
-            }
-          }
+      for (int u = 0; u < CHUNK; ++u) {
+        const int q = p0 + u;
+        if (q < P) {
+          const bool sb = q < mb;
+          const long long off = (long long)(sb ? q : q - mb) * row_stride;
+          zr[u].load((sb ? zb : za) + off);
+          xr[u].load((sb ? cb : ca) + off);
         }
+      }
 #pragma unroll
-        for (int u = 0; u < CHUNK; ++u)
-          if (u < cnt) pool.add(z[u], bb[u], x[u]);
+      for (int u = 0; u < CHUNK; ++u) {
+        const int q = p0 + u;
+        if (q < P) {
+          const bool sb = q < mb;
+          float z[V], x[V], bb[V];
+          zr[u].to_f32(z);
+          xr[u].to_f32(x);
+          const float4 t = __ldg(reinterpret_cast<const float4*>(
+              bias + ((long long)(sb ? m + q : q - mb)) * c + ch));
+          bb[0] = t.x; bb[1] = t.y; bb[2] = t.z; bb[3] = t.w;
+          pool.add(z, bb, x);
+        }
       }
     }
     float o[V];
 #pragma unroll
     for (int j = 0; j < V; ++j) o[j] = pool.acc[j] / pool.den[j];
-    store16_f32(out + ((long long)b * E + i) * c + ch, o);
+    store4(out + ((long long)b * E + i) * c + ch, o);
   }
 }
 
@@ -126,21 +168,18 @@ __global__ void __launch_bounds__(256) compress_scalar_kernel(
 template <typename T>
 static int launch_compress(const void* C, const void* Z, const float* bias, void* out, int B,
                            int n, int c, int m, int overlap, cudaStream_t st) {
-  constexpr int V = Vec16<T>::N;
   const long long E = n / m;
-  const bool vec_ok = (c % V == 0) && (c % 4 == 0) && aligned16(C) && aligned16(Z) &&
-                      aligned16(out) && aligned16(bias);
+  const uintptr_t al = 4 * sizeof(T) - 1;          // 4 elements
+  const bool vec_ok = (c % 4 == 0) && !(reinterpret_cast<uintptr_t>(C) & al) &&
+                      !(reinterpret_cast<uintptr_t>(Z) & al) && !(reinterpret_cast<uintptr_t>(out) & al) &&
+                      aligned16(bias);
   int sms = 148;
   if (vec_ok) {
-    const long long total = (long long)B * E * (c / V);
+    const long long total = (long long)B * E * (c / 4);
     long long blocks = (total + 255) / 256;
-    blocks = blocks < (long long)sms * 16 ? blocks : (long long)sms * 16;
-    if (m >= 16)
-      compress_vec_kernel<T, 8><<<(int)blocks, 256, 0, st>>>(
-          (const T*)C, (const T*)Z, bias, (T*)out, B, n, c, m, overlap, total);
-    else
-      compress_vec_kernel<T, 4><<<(int)blocks, 256, 0, st>>>(
-          (const T*)C, (const T*)Z, bias, (T*)out, B, n, c, m, overlap, total);
+    blocks = blocks < (long long)sms * 32 ? blocks : (long long)sms * 32;
+    compress_vec_kernel<T, 8><<<(int)blocks, 256, 0, st>>>(
+        (const T*)C, (const T*)Z, bias, (T*)out, B, n, c, m, overlap, total);
   } else {
     const long long total = (long long)B * E * c;
     long long blocks = (total + 255) / 256;
