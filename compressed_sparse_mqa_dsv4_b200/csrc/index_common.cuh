@@ -90,6 +90,12 @@ __device__ __forceinline__ float load_elem(const void* p, const uint8_t* scales,
   return e2m1_decode(nib) * e4m3_decode(scales[row * (cols / 16) + d / 16]);
 }
 
+// Row header of the threshold top-k's per-row region, zeroed before each score launch:
+// hist1 [256] at byte 0, hist2 [256] at byte 1024, the pipeline's counters at byte 2048. The
+// int at byte TK_WORK_BYTE of a launch's first row hands out the score kernel's work units.
+constexpr int TK_HDR = 4096;
+constexpr int TK_WORK_BYTE = 3072;
+
 int launch_index_scores_simt(const IndexArgs& a, int q_begin, int q_count, int max_e,
                              cudaStream_t st);
 int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max_e,

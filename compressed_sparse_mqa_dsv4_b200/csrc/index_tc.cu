@@ -8,8 +8,11 @@
 // entry's dot products with every head of every query in the tile, and the weighted
 // ReLU head sum is a per-thread reduction in registers:
 //     D[128 entries x 64*nqt] = K^I_blk[128 x c_I] . qI_tile[64*nqt x c_I]^T
-// CTAs walk work units (tile of <= 4 queries of one sequence, chunk of 4096-16384 entries):
-// persistent, one per SM, for multi-query tiles; one per unit for one-query tiles. 10 warps:
+// CTAs walk work units (tile of <= 4 queries of one sequence, chunk of 2048-16384 entries):
+// persistent, one per SM, for multi-query tiles; for one-query tiles (decode) either one CTA
+// per unit or -- with the threshold top-k's zeroed row headers at hand -- persistent CTAs
+// that draw units from a global counter (dynamic scheduling over rows of very different
+// lengths without a CTA start per unit). 10 warps:
 //   warps 0-7  epilogue: warp w reads TMEM lane quadrant w%4 for queries 2(w/4), 2(w/4)+1
 //   warp 8     producer: per unit the query tile, then 128-entry key blocks by 2D TMA into a
 //              4-stage ring (6 stages for one-query tiles) that runs on across units
@@ -36,12 +39,23 @@ constexpr uint32_t IX_TM_COLS = 512;
 // the Q buffer and spend the room on a deeper key ring. HIST: the tile also histograms its
 // scores for the threshold top-k (kept out of the layout otherwise: a few KiB more shared
 // memory cost the prefill shape ~10 % through a smaller L1).
-template <int QT, int NST, bool HIST>
+// DYN: units come from a global counter through a shared-memory FIFO; pre[] holds the dense
+// unit list's per-tile offsets.
+constexpr int IX_DYN_TILES = 1024;     // tiles of one launch the dynamic scheduler indexes
+constexpr int IX_DYN_CHUNK = 2048;     // entries per dynamically scheduled unit
+constexpr int IX_UQ = 4;               // unit FIFO depth
+
+template <int QT, int NST, bool HIST, bool DYN>
 struct IndexSmem {
   uint8_t q[2][QT * IX_HI * 128];           // K-major SW128: [QT*64 rows][64 ch] per K half
   uint8_t k[NST][2][IX_BLK * 128];          // [128 entries][64 ch] per K half
   float w[QT][IX_HI];
   int hist[HIST ? QT : 1][HIST ? 256 : 1];  // key bits 31..24 of the tile's scores
+  int pre[DYN ? IX_DYN_TILES : 1];          // first dense unit of each tile
+  int wsum[8];
+  int n_dense;                              // units in the dense list
+  int uid[IX_UQ];                           // unit FIFO (-1: no more units)
+  uint64_t u_full[IX_UQ], u_empty[IX_UQ];
   uint64_t q_full, q_empty;
   uint64_t k_full[NST], k_empty[NST];
   uint64_t d_full[2], d_empty[2];
@@ -65,9 +79,9 @@ __device__ unsigned long long g_ix_trace[32][8];
   } while (0)
 #endif
 
-template <int QT, int NST, bool HIST>
-constexpr size_t ix_smem() { return sizeof(IndexSmem<QT, NST, HIST>) + 1024; }
-static_assert(ix_smem<4, IX_STAGES, true>() <= 232448 && ix_smem<1, 6, true>() <= 232448,
+template <int QT, int NST, bool HIST, bool DYN>
+constexpr size_t ix_smem() { return sizeof(IndexSmem<QT, NST, HIST, DYN>) + 1024; }
+static_assert(ix_smem<4, IX_STAGES, true, false>() <= 232448 && ix_smem<1, 6, true, true>() <= 232448,
               "shared memory of the index score kernel");
 
 // Named-barrier OR-reduction over `threads` threads (all take the same decision).
@@ -85,44 +99,70 @@ __device__ __forceinline__ bool ix_red_or(uint32_t id, uint32_t threads, bool pr
 // A work unit: a tile of <= QT queries of one sequence and a chunk of its entries. Every
 // role derives the same units in the same order and skips the empty ones.
 struct IxUnit {
-  int b, qlo, nqt, e0, e1;
+  int b, qlo, nqt, e0, e1, e_tile;
   long long base;
   bool valid;
 };
 
-// Units are numbered chunk-major (all tiles' first chunks, then their second chunks, ...), so
-// the valid units of rows of different lengths form a dense prefix that the CTAs' round robin
-// spreads evenly.
+// Chunk c of tile `tile`; `flag`: report a key-row range outside the key buffer.
 template <int QT>
-__device__ __forceinline__ IxUnit ix_unit(const IndexArgs& a, int u, int q_begin, int q_count,
-                                          int tile0, int tiles_per_seq, int chunk, int ntiles) {
+__device__ __forceinline__ IxUnit ix_tile_unit(const IndexArgs& a, int tile, int c, int q_begin,
+                                               int q_count, int tiles_per_seq, int chunk, bool flag) {
   IxUnit r;
-  const int tile = tile0 + u % ntiles, c = u / ntiles;
   r.b = tile / tiles_per_seq;
   const int i0 = (tile % tiles_per_seq) * QT;
   r.qlo = max(r.b * a.nq + i0, q_begin);
   const int qhi = min(r.b * a.nq + min(i0 + QT, a.nq), q_begin + q_count);
   r.nqt = qhi - r.qlo;
   const int e_tile = r.nqt > 0 ? visible_entries(a, r.b, qhi - 1 - r.b * a.nq) : 0;
+  r.e_tile = e_tile;
   r.e0 = c * chunk;
   r.e1 = min(e_tile, r.e0 + chunk);
   r.base = r.nqt > 0 ? a.kv_row_off[r.b] : 0;
   const bool bounds_ok = r.base >= 0 && r.base + e_tile <= a.ki_rows;
   r.valid = r.nqt > 0 && r.e1 > r.e0 && bounds_ok;
-  if (r.nqt > 0 && !bounds_ok && c == 0 && threadIdx.x == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
+  if (r.nqt > 0 && !bounds_ok && flag) flag_status(DSV4_ERR_DEVICE_BOUNDS);
   return r;
 }
 
-// Persistent: each CTA walks the work units blockIdx.x, blockIdx.x + gridDim.x, ...; the key
-// ring, the TMEM double buffer and their barrier phases run on across units (global block
-// counter), the Q buffer is reloaded per unit once the MMAs of the previous unit are done.
-template <int QT, int NST, bool HIST>
+// Static schedule: units are numbered chunk-major (all tiles' first chunks, then their second
+// chunks, ...), so the valid units of rows of different lengths form a dense prefix that the
+// CTAs' round robin spreads evenly.
+template <int QT>
+__device__ __forceinline__ IxUnit ix_unit(const IndexArgs& a, int u, int q_begin, int q_count,
+                                          int tile0, int tiles_per_seq, int chunk, int ntiles) {
+  const int c = u / ntiles;
+  return ix_tile_unit<QT>(a, tile0 + u % ntiles, c, q_begin, q_count, tiles_per_seq, chunk,
+                          c == 0 && threadIdx.x == 0);
+}
+
+// Dynamic schedule: unit d of the dense tile-major list of valid units (tile i owns units
+// pre[i] .. pre[i+1] - 1, one per chunk).
+template <int QT, int NST, bool HIST, bool DYN>
+__device__ __forceinline__ IxUnit ix_dense_unit(const IndexArgs& a, const IndexSmem<QT, NST, HIST, DYN>& s,
+                                                int d, int q_begin, int q_count, int tile0,
+                                                int tiles_per_seq, int chunk, int ntiles) {
+  int lo = 0, hi = ntiles - 1;                 // the last tile i with pre[i] <= d
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s.pre[mid] <= d) lo = mid;
+    else hi = mid - 1;
+  }
+  return ix_tile_unit<QT>(a, tile0 + lo, d - s.pre[lo], q_begin, q_count, tiles_per_seq, chunk, false);
+}
+
+// Persistent: each CTA walks the work units blockIdx.x, blockIdx.x + gridDim.x, ... (DYN:
+// the units the producer draws from *work, passed on through a FIFO); the key ring, the TMEM
+// double buffer and their barrier phases run on across units (global block counter), the Q
+// buffer is reloaded per unit once the MMAs of the previous unit are done.
+template <int QT, int NST, bool HIST, bool DYN>
 __global__ void __launch_bounds__(IX_THREADS, 1)
     index_tc_kernel(const IndexArgs a, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_k, int q_begin, int q_count,
-                    int tile0, int tiles_per_seq, int chunk, int ntiles, int units, uint32_t spin) {
+                    int tile0, int tiles_per_seq, int chunk, int ntiles, int units, int* work,
+                    uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
-  IndexSmem<QT, NST, HIST>& s = *reinterpret_cast<IndexSmem<QT, NST, HIST>*>(
+  IndexSmem<QT, NST, HIST, DYN>& s = *reinterpret_cast<IndexSmem<QT, NST, HIST, DYN>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   volatile int* abort = &s.abort;
@@ -139,11 +179,49 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       tc::mbar_init(&s.d_empty[i], 256);
     }
     tc::mbar_init(&s.drain, 1);
+    for (int i = 0; i < IX_UQ; ++i) {
+      tc::mbar_init(&s.u_full[i], 1);
+      tc::mbar_init(&s.u_empty[i], 2);             // the MMA warp and the epilogue
+    }
     s.abort = 0;
     tc::fence_barrier_init();
   }
   if constexpr (HIST)
     for (int e = tid; e < QT * 256; e += blockDim.x) s.hist[e >> 8][e & 255] = 0;
+  if constexpr (DYN) {
+    // The dense unit list: every epilogue thread counts the chunks of four consecutive tiles,
+    // then a block scan turns the counts into each tile's first unit.
+    if (warp < 8) {
+      int cnt[4], sum = 0;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = 4 * tid + r;
+        cnt[r] = 0;
+        if (i < ntiles) {
+          const IxUnit w0 = ix_tile_unit<QT>(a, tile0 + i, 0, q_begin, q_count, tiles_per_seq,
+                                             chunk, blockIdx.x == 0);
+          if (w0.valid) cnt[r] = (w0.e_tile + chunk - 1) / chunk;
+        }
+        sum += cnt[r];
+      }
+      int inc = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (lane == 31) s.wsum[warp] = inc;
+      tc::named_barrier(1, 256);
+      int run = inc - sum;
+      for (int w2 = 0; w2 < warp; ++w2) run += s.wsum[w2];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        if (4 * tid + r < ntiles) s.pre[4 * tid + r] = run;
+        run += cnt[r];
+      }
+      if (tid == 255) s.n_dense = run;
+    }
+  }
   if (warp == 9) {
     tc::tmem_alloc(&s.tmem_base, IX_TM_COLS);
     tc::tmem_relinquish();
@@ -163,9 +241,28 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       uint32_t& gb = prod_gb;                          // key blocks issued so far
       int& k = prod_k;                                 // units loaded so far
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const IxUnit w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
-        if (!w.valid) continue;
+      int d = 0;                                       // DYN: this unit's ticket
+      if constexpr (DYN) d = atomicAdd(work, 1);
+      for (int it = 0, u = blockIdx.x; ok; ++it, u += gridDim.x) {
+        IxUnit w;
+        if constexpr (DYN) {
+          // publish the unit (or the end) to the MMA warp and the epilogue; the next ticket is
+          // drawn now and arrives while this unit's blocks stream
+          const bool more = d < s.n_dense;
+          const int nd = more ? atomicAdd(work, 1) : 0;
+          const int slot = it % IX_UQ;
+          if (it >= IX_UQ && !tc::mbar_wait(&s.u_empty[slot], (uint32_t)((it / IX_UQ - 1) & 1), spin, abort))
+            break;
+          s.uid[slot] = more ? d : -1;
+          tc::mbar_arrive(&s.u_full[slot]);
+          if (!more) break;
+          w = ix_dense_unit(a, s, d, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+          d = nd;
+        } else {
+          if (u >= units) break;
+          w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+          if (!w.valid) continue;
+        }
         // The unit's Q goes into the single Q buffer once the MMAs of the previous unit have
         // completed (q_empty). Meanwhile the unit's first key blocks already enter the ring:
         // up to NST of them reuse stages the previous units released, so the ring stays full
@@ -228,9 +325,22 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
       uint32_t gb = 0;
       int k = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const IxUnit w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
-        if (!w.valid) continue;
+      for (int it = 0, u = blockIdx.x; ok; ++it, u += gridDim.x) {
+        IxUnit w;
+        if constexpr (DYN) {
+          const int slot = it % IX_UQ;
+          ok = wwait(&s.u_full[slot], (uint32_t)((it / IX_UQ) & 1));
+          if (!ok) break;
+          const int d = s.uid[slot];
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&s.u_empty[slot]);
+          if (d < 0) break;
+          w = ix_dense_unit(a, s, d, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+        } else {
+          if (u >= units) break;
+          w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+          if (!w.valid) continue;
+        }
         ok = wwait(&s.q_full, (uint32_t)(k & 1));
         ++k;
         const uint32_t idesc = tc::idesc_bf16_f32(128, IX_HI * w.nqt, 0, 0);
@@ -270,12 +380,27 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
     uint32_t gb = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      const IxUnit w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
-      if (!w.valid) continue;
-      // every epilogue thread has finished the previous unit; after a failed wait all of
-      // them leave here together (named barriers below need all 256)
-      if (ix_red_or(1, 256, !ok)) break;
+    for (int it = 0, u = blockIdx.x;; ++it, u += gridDim.x) {
+      IxUnit w;
+      if constexpr (DYN) {
+        const int slot = it % IX_UQ;
+        int d = 0;
+        if (ok) ok = tc::mbar_wait(&s.u_full[slot], (uint32_t)((it / IX_UQ) & 1), spin, abort);
+        if (ok) d = s.uid[slot];
+        // every epilogue thread has finished the previous unit and read this slot; after a
+        // failed wait all of them leave here together (named barriers below need all 256)
+        if (ix_red_or(1, 256, !ok)) break;
+        if (tid == 0) tc::mbar_arrive(&s.u_empty[slot]);
+        if (d < 0) break;
+        w = ix_dense_unit(a, s, d, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+      } else {
+        if (u >= units) break;
+        w = ix_unit<QT>(a, u, q_begin, q_count, tile0, tiles_per_seq, chunk, ntiles);
+        if (!w.valid) continue;
+        // every epilogue thread has finished the previous unit; after a failed wait all of
+        // them leave here together (named barriers below need all 256)
+        if (ix_red_or(1, 256, !ok)) break;
+      }
       // the unit's head weights
       for (int e = tid; e < QT * IX_HI; e += 256) {
         const int q = e / IX_HI, h = e % IX_HI;
@@ -402,50 +527,53 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
   }
   // Prefill tiles (several queries): persistent CTAs, one per SM, walk units of IX_CHUNK
   // entries (per-tile CTAs paid their setup and pipeline fill on only a few key blocks).
-  // One-query tiles (decode over long rows of very different lengths): one CTA per unit, so
-  // that the hardware hands units to SMs as they free up (a static walk balanced them worse);
-  // units grow to 16384 entries while there are at least 4 per SM.
+  // One-query tiles (decode over long rows of very different lengths) with the threshold
+  // top-k's row headers: persistent CTAs draw IX_DYN_CHUNK-entry units from a counter in the
+  // first row's header (zeroed before this launch) -- finely balanced, no CTA start per unit
+  // (2048-entry units: 469 us for the 2.35 GB of keys of 64 rows of 32k-262k entries; 4096:
+  // 475 us; 8192: 485 us; one CTA per 16384-entry unit: 530 us, top-k passes included).
+  // Otherwise one CTA per unit, so that the hardware hands units to SMs as they free up (a
+  // static walk balanced them worse); units grow to 16384 entries while there are at least 4
+  // per SM.
   const long long tiles = t1 - t0 + 1;
-  int chunk = IX_CHUNK;
-  if (qt == 1)
+  const bool dyn = qt == 1 && a.topk_pipe && a.cand && tiles <= IX_DYN_TILES;
+  int chunk = dyn ? IX_DYN_CHUNK : IX_CHUNK;
+  if (qt == 1 && !dyn)
     while (chunk < 4 * IX_CHUNK && tiles * ((max_e + 2 * chunk - 1) / (2 * chunk)) >= 4 * sms) chunk *= 2;
   const long long nchunk = (max_e + chunk - 1) / chunk;
   const long long units = tiles * nchunk;
   if (units >= (1ll << 31)) return DSV4_OK;
-  const unsigned grid = (unsigned)(qt == 1 || units < sms ? units : sms);
+  const unsigned grid = (unsigned)((qt == 1 && !dyn) || units < sms ? units : sms);
+  int* work = dyn ? reinterpret_cast<int*>(a.cand + (long long)(q_begin - a.score_q0) * a.cand_row_bytes +
+                                           TK_WORK_BYTE)
+                  : nullptr;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<IX_QT, IX_STAGES, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ix_smem<IX_QT, IX_STAGES, false>());
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(index_tc_kernel<IX_QT, IX_STAGES, true>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ix_smem<IX_QT, IX_STAGES, true>());
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(index_tc_kernel<1, 6, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)ix_smem<1, 6, false>());
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(index_tc_kernel<1, 6, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)ix_smem<1, 6, true>());
+    cudaError_t e = cudaSuccess;
+    auto smem_attr = [&](const void* fn, size_t bytes) {
+      if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    };
+    smem_attr((const void*)index_tc_kernel<IX_QT, IX_STAGES, false, false>, ix_smem<IX_QT, IX_STAGES, false, false>());
+    smem_attr((const void*)index_tc_kernel<IX_QT, IX_STAGES, true, false>, ix_smem<IX_QT, IX_STAGES, true, false>());
+    smem_attr((const void*)index_tc_kernel<1, 6, false, false>, ix_smem<1, 6, false, false>());
+    smem_attr((const void*)index_tc_kernel<1, 6, true, false>, ix_smem<1, 6, true, false>());
+    smem_attr((const void*)index_tc_kernel<1, 6, true, true>, ix_smem<1, 6, true, true>());
     if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "index_tc: %s", cudaGetErrorString(e));
     attr_set = true;
   }
   const int sp = spin_limit();
+#define IX_LAUNCH(QT_, NST_, HIST_, DYN_)                                                          \
+  index_tc_kernel<QT_, NST_, HIST_, DYN_><<<grid, IX_THREADS, ix_smem<QT_, NST_, HIST_, DYN_>(), st>>>( \
+      a, mq, mk, q_begin, q_count, t0, tps, chunk, (int)tiles, (int)units, work, sp)
   if (qt == 1) {
-    if (a.topk_pipe)
-      index_tc_kernel<1, 6, true><<<grid, IX_THREADS, ix_smem<1, 6, true>(), st>>>(a, mq, mk, q_begin, q_count,
-                                                                                 t0, tps, chunk, (int)tiles, (int)units, sp);
-    else
-      index_tc_kernel<1, 6, false><<<grid, IX_THREADS, ix_smem<1, 6, false>(), st>>>(a, mq, mk, q_begin, q_count,
-                                                                                   t0, tps, chunk, (int)tiles, (int)units, sp);
+    if (dyn) IX_LAUNCH(1, 6, true, true);
+    else if (a.topk_pipe) IX_LAUNCH(1, 6, true, false);
+    else IX_LAUNCH(1, 6, false, false);
   } else {
-    if (a.topk_pipe)
-      index_tc_kernel<IX_QT, IX_STAGES, true><<<grid, IX_THREADS, ix_smem<IX_QT, IX_STAGES, true>(), st>>>(
-          a, mq, mk, q_begin, q_count, t0, tps, chunk, (int)tiles, (int)units, sp);
-    else
-      index_tc_kernel<IX_QT, IX_STAGES, false><<<grid, IX_THREADS, ix_smem<IX_QT, IX_STAGES, false>(), st>>>(
-          a, mq, mk, q_begin, q_count, t0, tps, chunk, (int)tiles, (int)units, sp);
+    if (a.topk_pipe) IX_LAUNCH(IX_QT, IX_STAGES, true, false);
+    else IX_LAUNCH(IX_QT, IX_STAGES, false, false);
   }
+#undef IX_LAUNCH
   *used = true;
   return launch_status("index scores (tensor cores)");
 }

@@ -369,7 +369,6 @@ __global__ void __launch_bounds__(NT) topk_merge_kernel(IndexArgs a, int q_begin
 constexpr int TK_PASS = 8192;                    // entries per CTA of a pass
 constexpr int TK_CAND = 8192;                    // boundary candidates kept per row
 constexpr int TK_MAXK = 4096;                    // larger k: single-CTA select
-constexpr int TK_HDR = 4096;                     // row header: hist1, hist2, counters
 
 struct TkRow {
   int* hist1;                                    // [256]

@@ -155,6 +155,24 @@ def test_index_decode_long_contexts(dsv4):
                    what="decode long")
 
 
+def test_index_decode_mixed_lengths_dynamic_units(dsv4):
+    """Decode batch with rows from no entries to ~50k: the score kernel's persistent CTAs draw
+    (row, 4096-entry chunk) units from a counter over the rows' dense unit list, so empty rows,
+    rows shorter than one chunk, exact multiples of a chunk and ragged last chunks all occur."""
+    rng = np.random.default_rng(5)
+    lens = [1, 3, 4, 7, 4 * 4096, 4 * 4096 + 3, 4 * 4097, 4 * 8192 + 2] + \
+        [int(x) for x in rng.integers(8, 4 * 50000, 16)]
+    shape = preset("flash_csa_prefill", B=len(lens))
+    rows = [L // 4 for L in lens]
+    offs = list(np.concatenate([[0], np.cumsum(rows)[:-1]]).astype(np.int64))
+    g = Generator(41)
+    qI, w = g.index_queries(shape, 1)
+    KI = g.index_keys(shape, int(sum(rows)) + 1)
+    pos0 = [L - 1 for L in lens]
+    _run_and_check(dsv4, qI, w, KI, offs, pos0, 4, 512, [(b, 0) for b in range(len(lens))],
+                   what="decode mixed")
+
+
 def test_index_many_long_rows(dsv4):
     """More than 1024 queries whose rows exceed 16384 entries: the workspace path selects per
     16384-entry segment and merges the candidates (the threshold pipeline serves requests with
