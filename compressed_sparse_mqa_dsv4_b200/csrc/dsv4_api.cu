@@ -246,7 +246,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     const int qn = total - q0 < chunk ? total - q0 : chunk;
     a.score_q0 = scores_out ? 0 : q0;
     ax.score_q0 = a.score_q0;
-    bool used = false;
+    bool used = false, hist1_built = false;
     int s = topk_prepare(a, q0, qn, st);
     if (s != DSV4_OK) return s;
     if (fp4x) {
@@ -257,9 +257,9 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
       if (s != DSV4_OK) return s;
       ax.q_map_q0 = q0;
       ax.q_map_rows = (long long)qn * H_I;
-      s = launch_index_scores_tc(ax, q0, qn, max_entries, st, &used);
+      s = launch_index_scores_tc(ax, q0, qn, max_entries, st, &used, &hist1_built);
     } else {
-      s = launch_index_scores_tc(a, q0, qn, max_entries, st, &used);
+      s = launch_index_scores_tc(a, q0, qn, max_entries, st, &used, &hist1_built);
     }
     if (s != DSV4_OK) return s;
     if (q0 == 0)
@@ -269,7 +269,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
       s = launch_index_scores_simt(a, q0, qn, max_entries, st);
       if (s != DSV4_OK) return s;
     }
-    a.hist1_done = used ? 1 : 0;                  // the tensor-core kernel built hist1
+    a.hist1_done = used && hist1_built ? 1 : 0;
     s = launch_topk(a, q0, qn, st);
     if (s != DSV4_OK) return s;
   }

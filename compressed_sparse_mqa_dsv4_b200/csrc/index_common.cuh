@@ -26,9 +26,8 @@ struct IndexArgs {
   int q_map_q0;
   long long q_map_rows;
   // top-k of long rows, one region of cand_row_bytes per score row:
-  //  * topk_pipe = 1 (few rows, decode): threshold pipeline; the region holds int hist1[256]
-  //    of key bits 31..24 at its start, then hist2, counters, the entries above the
-  //    threshold and the boundary candidates; hist1_done: the score kernel built hist1;
+  //  * topk_pipe = 1 (few rows, decode): threshold pipeline; the region holds hist1 of the
+  //    top TK_H1_BITS key bits (TK_HDR bytes); hist1_done: the score kernel built hist1;
   //  * nseg > 1 (many rows): per-segment selection then a merge; the region holds nseg * k
   //    candidate scores, then their nseg * k entry indices.
   int topk_pipe;
@@ -90,16 +89,21 @@ __device__ __forceinline__ float load_elem(const void* p, const uint8_t* scales,
   return e2m1_decode(nib) * e4m3_decode(scales[row * (cols / 16) + d / 16]);
 }
 
-// Row header of the threshold top-k's per-row region, zeroed before each score launch:
-// hist1 [256] at byte 0, hist2 [256] at byte 1024, the pipeline's counters at byte 2048. The
-// int at byte TK_WORK_BYTE of a launch's first row hands out the score kernel's work units.
-constexpr int TK_HDR = 4096;
-constexpr int TK_WORK_BYTE = 3072;
+// The threshold top-k's per-row region, zeroed before each score launch: hist1 [TK_H1_BINS]
+// at byte 0 (the row's scores binned by the top TK_H1_BITS bits of their order-preserving
+// keys). The int at byte TK_WORK_BYTE of a launch's first row hands out the score kernel's
+// work units.
+constexpr int TK_H1_BITS = 11;
+constexpr int TK_H1_BINS = 1 << TK_H1_BITS;
+constexpr int TK_HDR = 8448;
+constexpr int TK_WORK_BYTE = 8192;
 
 int launch_index_scores_simt(const IndexArgs& a, int q_begin, int q_count, int max_e,
                              cudaStream_t st);
+// *used: the tensor-core kernel took the request; *hist1_built: it also built the threshold
+// top-k's first histograms.
 int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max_e,
-                           cudaStream_t st, bool* used);
+                           cudaStream_t st, bool* used, bool* hist1_built);
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st);
 // Zeroes the threshold top-k headers of the score rows of queries [q_begin, q_begin +
 // q_count) (before the score kernel, which may build the first histogram).

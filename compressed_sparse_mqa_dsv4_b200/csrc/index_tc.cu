@@ -36,9 +36,10 @@ constexpr int IX_THREADS = 320;
 constexpr uint32_t IX_TM_COLS = 512;
 
 // QT queries per tile, NST key stages in flight. One-query tiles (decode) need a quarter of
-// the Q buffer and spend the room on a deeper key ring. HIST: the tile also histograms its
-// scores for the threshold top-k (kept out of the layout otherwise: a few KiB more shared
-// memory cost the prefill shape ~10 % through a smaller L1).
+// the Q buffer and spend the room on a deeper key ring. HIST (one-query tiles): the tile
+// also histograms its scores for the threshold top-k, by the top TK_H1_BITS bits of their
+// keys (kept out of the layout otherwise: a few KiB more shared memory cost the prefill
+// shape ~10 % through a smaller L1).
 // DYN: units come from a global counter through a shared-memory FIFO; pre[] holds the dense
 // unit list's per-tile offsets.
 constexpr int IX_DYN_TILES = 1024;     // tiles of one launch the dynamic scheduler indexes
@@ -50,7 +51,7 @@ struct IndexSmem {
   uint8_t q[2][QT * IX_HI * 128];           // K-major SW128: [QT*64 rows][64 ch] per K half
   uint8_t k[NST][2][IX_BLK * 128];          // [128 entries][64 ch] per K half
   float w[QT][IX_HI];
-  int hist[HIST ? QT : 1][HIST ? 256 : 1];  // key bits 31..24 of the tile's scores
+  int hist[HIST ? QT : 1][HIST ? TK_H1_BINS : 1];  // top key bits of the tile's scores
   int pre[DYN ? IX_DYN_TILES : 1];          // first dense unit of each tile
   int wsum[8];
   int n_dense;                              // units in the dense list
@@ -80,8 +81,11 @@ __device__ unsigned long long g_ix_trace[32][8];
 #endif
 
 template <int QT, int NST, bool HIST, bool DYN>
-constexpr size_t ix_smem() { return sizeof(IndexSmem<QT, NST, HIST, DYN>) + 1024; }
-static_assert(ix_smem<4, IX_STAGES, true, false>() <= 232448 && ix_smem<1, 6, true, true>() <= 232448,
+constexpr size_t ix_smem() {
+  static_assert(!HIST || QT == 1, "multi-query tiles leave the first histogram to a pass");
+  return sizeof(IndexSmem<QT, NST, HIST, DYN>) + 1024;
+}
+static_assert(ix_smem<4, IX_STAGES, false, false>() <= 232448 && ix_smem<1, 6, true, true>() <= 232448,
               "shared memory of the index score kernel");
 
 // Named-barrier OR-reduction over `threads` threads (all take the same decision).
@@ -187,7 +191,7 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
     tc::fence_barrier_init();
   }
   if constexpr (HIST)
-    for (int e = tid; e < QT * 256; e += blockDim.x) s.hist[e >> 8][e & 255] = 0;
+    for (int e = tid; e < QT * TK_H1_BINS; e += blockDim.x) s.hist[e / TK_H1_BINS][e % TK_H1_BINS] = 0;
   if constexpr (DYN) {
     // The dense unit list: every epilogue thread counts the chunks of four consecutive tiles,
     // then a block scan turns the counts into each tile's first unit.
@@ -454,21 +458,21 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
         }
         if (sidx < Et[0]) a.scores[srow[0] + sidx] = sc0;
         if constexpr (HIST) {                    // first histogram of the threshold top-k
-          hist_add(s.hist[QT > 1 ? 2 * qp : 0], score_key(sc0) >> 24, sidx < Et[0]);
-          if (QT > 1) hist_add(s.hist[QT > 1 ? 2 * qp + 1 : 0], score_key(sc1) >> 24, 2 * qp + 1 < w.nqt && sidx < Et[1]);
+          hist_add(s.hist[0], score_key(sc0) >> (32 - TK_H1_BITS), sidx < Et[0]);
         }
         if (tid == 0) IX_TRACE(6, (int)gb);
         if (QT > 1 && 2 * qp + 1 < w.nqt && sidx < Et[1]) a.scores[srow[1] + sidx] = sc1;
       }
       if constexpr (HIST) {
-        // add the unit's histograms to its rows' first histograms (int hist1[256] at the
-        // start of each row's top-k region) and clear them for the next unit
+        // add the unit's histogram to its row's first histogram (int hist1[TK_H1_BINS] at
+        // the start of the row's top-k region) and clear it for the next unit
         tc::named_barrier(1, 256);
-        for (int e = tid; e < QT * 256; e += 256) {
-          const int q = e >> 8, v = s.hist[q][e & 255];
+        int* h1 = reinterpret_cast<int*>(a.cand + (long long)(w.qlo - a.score_q0) * a.cand_row_bytes);
+        for (int e = tid; e < TK_H1_BINS; e += 256) {
+          const int v = s.hist[0][e];
           if (v) {
-            atomicAdd(reinterpret_cast<int*>(a.cand + (long long)(w.qlo + q - a.score_q0) * a.cand_row_bytes) + (e & 255), v);
-            s.hist[q][e & 255] = 0;
+            atomicAdd(h1 + e, v);
+            s.hist[0][e] = 0;
           }
         }
       }
@@ -493,14 +497,16 @@ __global__ void __launch_bounds__(IX_THREADS, 1)
 }  // namespace
 
 int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max_e,
-                           cudaStream_t st, bool* used) {
+                           cudaStream_t st, bool* used, bool* hist1_built) {
   *used = false;
+  *hist1_built = false;
   const char* force = std::getenv("DSV4_FORCE_SIMT");
   if (force && force[0] == '1') return DSV4_OK;
   if (a.qdtype != DSV4_BF16 || a.c_I != IX_CI || a.H_I != IX_HI) return DSV4_OK;
   if (!aligned16(a.qI) || !aligned16(a.KI)) return DSV4_OK;
   if (q_count <= 0 || max_e <= 0) {
     *used = true;
+    *hist1_built = true;
     return DSV4_OK;
   }
   const long long q_rows = a.q_map_rows > 0 ? a.q_map_rows : (long long)a.B * a.nq * IX_HI;
@@ -554,7 +560,6 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
       if (e == cudaSuccess) e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     };
     smem_attr((const void*)index_tc_kernel<IX_QT, IX_STAGES, false, false>, ix_smem<IX_QT, IX_STAGES, false, false>());
-    smem_attr((const void*)index_tc_kernel<IX_QT, IX_STAGES, true, false>, ix_smem<IX_QT, IX_STAGES, true, false>());
     smem_attr((const void*)index_tc_kernel<1, 6, false, false>, ix_smem<1, 6, false, false>());
     smem_attr((const void*)index_tc_kernel<1, 6, true, false>, ix_smem<1, 6, true, false>());
     smem_attr((const void*)index_tc_kernel<1, 6, true, true>, ix_smem<1, 6, true, true>());
@@ -570,11 +575,11 @@ int launch_index_scores_tc(const IndexArgs& a, int q_begin, int q_count, int max
     else if (a.topk_pipe) IX_LAUNCH(1, 6, true, false);
     else IX_LAUNCH(1, 6, false, false);
   } else {
-    if (a.topk_pipe) IX_LAUNCH(IX_QT, IX_STAGES, true, false);
-    else IX_LAUNCH(IX_QT, IX_STAGES, false, false);
+    IX_LAUNCH(IX_QT, IX_STAGES, false, false);
   }
 #undef IX_LAUNCH
   *used = true;
+  *hist1_built = qt == 1 && a.topk_pipe;
   return launch_status("index scores (tensor cores)");
 }
 

@@ -50,7 +50,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
 struct TopkShared {
   int hist[256];
   int warp_tot[32];
-  int sel, above;
+  int sel, above, cnt;
 };
 
 // Selects the keff (< n) largest of sc[0, n) under (score descending, position ascending) and
@@ -352,27 +352,40 @@ __global__ void __launch_bounds__(NT) topk_merge_kernel(IndexArgs a, int q_begin
 }
 
 // ---------------------------------------------------------------- threshold pipeline
-// Requests with few rows longer than TOPK_SEG entries (decode over long contexts). Each pass
-// is spread over
-// CTAs of TK_PASS entries and streams the row once:
-//   hist1  per-row histogram of key bits 31..24;
-//   hist2  the bin B1 holding the k_eff-th largest key -> histogram of bits 23..16 of the
-//          keys in B1;
-//   filter the bin B2 holding the k_eff-th largest key among those -> keys whose top 16 bits
-//          exceed (B1, B2) are selected; keys equal to it in their top 16 bits are boundary
-//          candidates, kept as (low 16 key bits, ~entry) so that a larger value means a larger
-//          score or, for equal scores, a lower entry;
-//   final  per row: the k_eff - (selected) largest boundary candidates by a radix select over
-//          those 48-bit values (all distinct), then the selected entries in ascending order.
-// A row whose boundary candidates exceed TK_CAND is selected by the single-CTA select over
-// the whole row instead (many scores sharing their top 16 bits).
-constexpr int TK_PASS = 8192;                    // entries per CTA of a pass
+// Requests with few rows longer than TOPK_SEG entries (decode over long contexts). Order-
+// preserving keys are binned by their top TK_H1_BITS bits (sign, exponent, two mantissa
+// bits: quarter-octave bins):
+//   hist1  per-row histogram of those 11 bits, built by the score kernel (else by a pass over
+//          CTAs of TK_PASS entries); the bin B1 holding the k_eff-th largest key and its
+//          population follow from it;
+//   filter CTAs of TK_FPASS entries of the rows whose bin B1 holds at most TK_CAND keys: keys
+//          above B1 are selected, keys in B1 are boundary candidates, kept as (low 21 key
+//          bits, ~entry) so that a larger value means a larger score or, for equal scores, a
+//          lower entry. Each CTA gathers them in shared memory and reserves room in the row's
+//          lists with one global atomic per list;
+//   final  one CTA per row: the k_eff - (selected) largest candidates by a radix select over
+//          those values (all distinct; 11-bit digits, stopping once a digit's bin is taken
+//          whole), then the selected entries in ascending order (a bitmap over the row). A row
+//          whose bin B1 is crowded takes a second level here -- a histogram of key bits 20..13
+//          of the keys in B1 and the filter against B1:B2, both in this CTA -- and a row whose
+//          boundary candidates still exceed TK_CAND (many equal scores) the whole-row select.
+// Keys are compared as the scores themselves: a bin's lowest key maps back to a float bound.
+constexpr int TK_PASS = 8192;                    // entries per CTA of the hist1 pass
+constexpr int TK_FPASS = 16384;                  // entries per CTA of the filter
 constexpr int TK_CAND = 8192;                    // boundary candidates kept per row
 constexpr int TK_MAXK = 4096;                    // larger k: single-CTA select
+constexpr int TK_LSEL = 1024;                    // shared-memory lists of a filter CTA
+constexpr int TK_LCAND = 1024;
+constexpr int TK_H1_SHIFT = 32 - TK_H1_BITS;     // first level: key bits 31..21
+constexpr int TK_H2_SHIFT = TK_H1_SHIFT - 8;     // second level: key bits 20..13
+constexpr int TK_BITMAP_MAX = 1 << 19;           // rows up to this many entries: bitmap order
+constexpr int TK_FINAL_NT = 512;
+constexpr int TK_FINAL_SMEM = TK_CAND * 8 + TK_MAXK * 4 + TK_BITMAP_MAX / 8;
+constexpr int TK_CNT_BYTE = TK_WORK_BYTE + 64;   // n_sel, n_cand of the row's lists
+static_assert(4 * TK_H1_BINS <= TK_WORK_BYTE && TK_CNT_BYTE + 8 <= TK_HDR, "top-k row header");
 
 struct TkRow {
-  int* hist1;                                    // [256]
-  int* hist2;                                    // [256]
+  int* hist1;                                    // [TK_H1_BINS]
   int* counters;                                 // n_sel, n_cand
   int32_t* sel;                                  // [k]
   unsigned long long* cand;                      // [TK_CAND]
@@ -382,51 +395,57 @@ __device__ __forceinline__ TkRow tk_row(const IndexArgs& a, long long row) {
   char* base = a.cand + row * a.cand_row_bytes;
   TkRow r;
   r.hist1 = reinterpret_cast<int*>(base);
-  r.hist2 = reinterpret_cast<int*>(base + 1024);
-  r.counters = reinterpret_cast<int*>(base + 2048);
+  r.counters = reinterpret_cast<int*>(base + TK_CNT_BYTE);
   r.sel = reinterpret_cast<int32_t*>(base + TK_HDR);
   r.cand = reinterpret_cast<unsigned long long*>(base + TK_HDR + (((long long)a.k * 4 + 255) & ~255ll));
   return r;
 }
 
-// The bin (by thread: thread t owns bin 255 - t) where the count from the top first reaches
-// `need`; returns the bin and the count strictly above it through shared memory.
-template <int NT>
-__device__ __forceinline__ void tk_find_bin(const int* hist_g, int need, TopkShared& sh) {
-  if (threadIdx.x == 0) {                         // (not found: an inconsistent row, which the
-    sh.sel = -1;                                  // final stage sends to the whole-row select)
+// The bin where the count from the top first reaches `need`, over `bins` <= P * NT bins read
+// through ld(bin); thread t owns bins bins-1-P*t .. bins-P*(t+1). Returns through shared
+// memory the bin (-1 if none: an inconsistent row, which goes to the whole-row select), the
+// count strictly above it and its own count.
+template <int NT, int P, typename Ld>
+__device__ __forceinline__ void tk_find_bin(Ld ld, int bins, int need, TopkShared& sh) {
+  if (threadIdx.x == 0) {
+    sh.sel = -1;
     sh.above = 0;
+    sh.cnt = 0;
   }
-  const int d = 255 - (int)threadIdx.x;
-  const int h = d >= 0 ? __ldcg(hist_g + d) : 0;
+  int h[P], sum = 0;
+#pragma unroll
+  for (int r = 0; r < P; ++r) {
+    const int d = bins - 1 - P * (int)threadIdx.x - r;
+    h[r] = d >= 0 ? ld(d) : 0;
+    sum += h[r];
+  }
   int tot;
-  const int above = block_exclusive_scan<NT>(h, sh.warp_tot, tot);
-  if (d >= 0 && above < need && need <= above + h) {
-    sh.sel = d;
-    sh.above = above;
+  int above = block_exclusive_scan<NT>(sum, sh.warp_tot, tot);
+#pragma unroll
+  for (int r = 0; r < P; ++r) {
+    const int d = bins - 1 - P * (int)threadIdx.x - r;
+    if (d >= 0 && above < need && need <= above + h[r]) {
+      sh.sel = d;
+      sh.above = above;
+      sh.cnt = h[r];
+    }
+    above += h[r];
   }
   __syncthreads();
 }
 
-// One pass over entries [lo, hi) of a score row: 32 keys per thread, loaded as float4s
-// (8 in flight per thread). f(j, key, valid) is called by whole warps.
+// One pass over entries [lo, hi) of a score row: 32 keys per thread, loaded as 8 float4s in
+// flight. The loads are unconditional: lo is a multiple of 4 and the row's stride a multiple
+// of 4 that covers its entries, so an index clamped to the row's last float4 (ld4) stays in
+// the row (what lies past hi is passed as invalid). f(j, key, valid) is called by whole warps.
 template <int NT, typename F>
-__device__ __forceinline__ void tk_scan(const float* sc, int lo, int hi, F f) {
+__device__ __forceinline__ void tk_scan(const float* sc, int ld4, int lo, int hi, F f) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   for (int j0 = lo + 128 * wid; j0 < hi; j0 += 128 * (NT / 32) * 8) {
     float4 v[8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int j = j0 + 128 * (NT / 32) * r + 4 * lane;
-      v[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j + 3 < hi) {
-        v[r] = __ldcg(reinterpret_cast<const float4*>(sc + j));
-      } else {
-        if (j < hi) v[r].x = __ldcg(sc + j);
-        if (j + 1 < hi) v[r].y = __ldcg(sc + j + 1);
-        if (j + 2 < hi) v[r].z = __ldcg(sc + j + 2);
-      }
-    }
+    for (int r = 0; r < 8; ++r)
+      v[r] = __ldcg(reinterpret_cast<const float4*>(sc + min(j0 + 128 * (NT / 32) * r + 4 * lane, ld4)));
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int j = j0 + 128 * (NT / 32) * r + 4 * lane;
@@ -437,16 +456,98 @@ __device__ __forceinline__ void tk_scan(const float* sc, int lo, int hi, F f) {
   }
 }
 
-// Warp-aggregated append of one value per flagged lane to list[*counter ...]; returns the
-// position of this lane's value (or -1).
-__device__ __forceinline__ int tk_append(int* counter, bool pred) {
-  const uint32_t m = __ballot_sync(0xffffffffu, pred);
-  if (m == 0) return -1;
-  const int lane = threadIdx.x & 31;
-  int base = 0;
-  if (lane == __ffs(m) - 1) base = atomicAdd(counter, __popc(m));
-  base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
-  return pred ? base + __popc(m & ((1u << lane) - 1u)) : -1;
+// Float bounds of bin `thr` of the keys' top 32 - shift bits: key >> shift > thr <=> score >= hi
+// (never for the top bin), key >> shift >= thr <=> score >= lo. (A bin of NaN keys gives NaN
+// bounds that nothing passes; the final stage then finds the lists inconsistent.)
+struct TkBounds {
+  float lo, hi;
+  bool has_hi;
+  uint32_t low;                                  // the key bits below the bin
+};
+
+__device__ __forceinline__ float tk_key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+__device__ __forceinline__ TkBounds tk_bounds(uint32_t thr, int shift) {
+  TkBounds b;
+  b.lo = tk_key_float(thr << shift);
+  const uint32_t next = (thr + 1u) << shift;     // 0: thr is the top bin
+  b.has_hi = next != 0u;
+  b.hi = b.has_hi ? tk_key_float(next) : 0.f;
+  b.low = (1u << shift) - 1u;
+  return b;
+}
+
+// Filters entries [lo, hi) of a row against the bounds: selected entries go to sel_list,
+// boundary candidates to cand_list; n[0], n[1] (shared) count them all. Every thread tests
+// its 32 keys on its own; a warp reserves room for its entries with one shared atomic per
+// list. Entries beyond sel_cap / cand_cap go to spill(is_selected, value).
+template <int NT, typename Spill>
+__device__ __forceinline__ void tk_filter_range(const float* sc, int ld4, int lo, int hi,
+                                                const TkBounds& b, int* n, int* sel_list,
+                                                int sel_cap, unsigned long long* cand_list,
+                                                int cand_cap, Spill spill) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (int j0 = lo + 128 * wid; j0 < hi; j0 += 128 * (NT / 32) * 8) {
+    float4 v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      v[q] = __ldcg(reinterpret_cast<const float4*>(sc + min(j0 + 128 * (NT / 32) * q + 4 * lane, ld4)));
+    uint32_t msel = 0, mcand = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int jb = j0 + 128 * (NT / 32) * q + 4 * lane;
+      const float fv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool in = jb + u < hi;
+        const bool s = in && b.has_hi && fv[u] >= b.hi;
+        const bool c = in && !s && fv[u] >= b.lo;
+        msel |= s ? 1u << (4 * q + u) : 0u;
+        mcand |= c ? 1u << (4 * q + u) : 0u;
+      }
+    }
+    const int ns = __popc(msel), nc = __popc(mcand);
+    if (!__any_sync(0xffffffffu, (ns | nc) != 0)) continue;
+    int ps = ns, pc = nc;                          // inclusive warp scans
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, ps, o), y = __shfl_up_sync(0xffffffffu, pc, o);
+      if (lane >= o) {
+        ps += x;
+        pc += y;
+      }
+    }
+    int bs = 0, bc = 0;
+    if (lane == 31) {
+      bs = ps ? atomicAdd(&n[0], ps) : 0;
+      bc = pc ? atomicAdd(&n[1], pc) : 0;
+    }
+    bs = __shfl_sync(0xffffffffu, bs, 31) + ps - ns;
+    bc = __shfl_sync(0xffffffffu, bc, 31) + pc - nc;
+    if ((msel | mcand) == 0) continue;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int jb = j0 + 128 * (NT / 32) * q + 4 * lane;
+      const float fv[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int bit = 4 * q + u;
+        if ((msel >> bit) & 1u) {
+          if (bs < sel_cap) sel_list[bs] = jb + u;
+          else spill(true, (unsigned long long)(jb + u));
+          ++bs;
+        } else if ((mcand >> bit) & 1u) {
+          const unsigned long long cv = ((unsigned long long)(score_key(fv[u]) & b.low) << 32) |
+                                        (unsigned long long)(0xFFFFFFFFu - (uint32_t)(jb + u));
+          if (bc < cand_cap) cand_list[bc] = cv;
+          else spill(false, cv);
+          ++bc;
+        }
+      }
+    }
+  }
 }
 
 struct TkCta {
@@ -455,81 +556,76 @@ struct TkCta {
   bool active;
 };
 
-__device__ __forceinline__ TkCta tk_cta(const IndexArgs& a, int q_begin) {
+__device__ __forceinline__ TkCta tk_cta(const IndexArgs& a, int q_begin, int pass) {
   TkCta c;
   c.qg = q_begin + blockIdx.y;
   const int b = c.qg / a.nq, i = c.qg % a.nq;
   c.Et = visible_entries(a, b, i);
   c.keff = min(a.k, c.Et);
   c.row = c.qg - a.score_q0;
-  c.lo = blockIdx.x * TK_PASS;
-  c.hi = min(c.Et, c.lo + TK_PASS);
+  c.lo = blockIdx.x * pass;
+  c.hi = min(c.Et, c.lo + pass);
   c.active = c.Et > a.k && c.lo < c.hi;          // shorter rows: the final kernel selects all
   return c;
 }
 
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_hist1_kernel(IndexArgs a, int q_begin) {
-  __shared__ TopkShared sh;
-  const TkCta c = tk_cta(a, q_begin);
+  __shared__ int h1[TK_H1_BINS];
+  const TkCta c = tk_cta(a, q_begin, TK_PASS);
   if (!c.active) return;
   const TkRow r = tk_row(a, c.row);
-  if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+  for (int e = threadIdx.x; e < TK_H1_BINS; e += NT) h1[e] = 0;
   __syncthreads();
-  tk_scan<NT>(a.scores + c.row * a.scores_ld, c.lo, c.hi,
-              [&](int, uint32_t key, bool valid) { hist_add(sh.hist, key >> 24, valid); });
+  tk_scan<NT>(a.scores + c.row * a.scores_ld, (int)a.scores_ld - 4, c.lo, c.hi,
+              [&](int, uint32_t key, bool valid) { hist_add(h1, key >> TK_H1_SHIFT, valid); });
   __syncthreads();
-  if (threadIdx.x < 256 && sh.hist[threadIdx.x]) atomicAdd(r.hist1 + threadIdx.x, sh.hist[threadIdx.x]);
+  for (int e = threadIdx.x; e < TK_H1_BINS; e += NT)
+    if (h1[e]) atomicAdd(r.hist1 + e, h1[e]);
 }
 
 template <int NT>
-__global__ void __launch_bounds__(NT) topk_hist2_kernel(IndexArgs a, int q_begin) {
+__global__ void __launch_bounds__(NT, 2) topk_filter_kernel(IndexArgs a, int q_begin) {
   __shared__ TopkShared sh;
-  const TkCta c = tk_cta(a, q_begin);
+  __shared__ int l_n[2], l_base[2];
+  __shared__ int l_sel[TK_LSEL];
+  __shared__ unsigned long long l_cand[TK_LCAND];
+  const TkCta c = tk_cta(a, q_begin, TK_FPASS);
   if (!c.active) return;
   const TkRow r = tk_row(a, c.row);
-  tk_find_bin<NT>(r.hist1, c.keff, sh);
-  const uint32_t b1 = (uint32_t)sh.sel;
-  if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+  if (threadIdx.x < 2) l_n[threadIdx.x] = 0;     // (ordered by the barriers below)
+  tk_find_bin<NT, TK_H1_BINS / NT>([&](int d) { return __ldcg(r.hist1 + d); }, TK_H1_BINS, c.keff, sh);
+  const int b1 = sh.sel, c1 = sh.cnt;
+  if (b1 < 0 || c1 > TK_CAND) return;            // the final kernel takes such rows whole
+  const TkBounds bd = tk_bounds((uint32_t)b1, TK_H1_SHIFT);
+  tk_filter_range<NT>(a.scores + c.row * a.scores_ld, (int)a.scores_ld - 4, c.lo, c.hi, bd, l_n,
+                      l_sel, TK_LSEL, l_cand, TK_LCAND, [&](bool is_sel, unsigned long long v) {
+                        const int pg = atomicAdd(r.counters + (is_sel ? 0 : 1), 1);
+                        if (is_sel && pg < a.k) r.sel[pg] = (int32_t)v;
+                        if (!is_sel && pg < TK_CAND) r.cand[pg] = v;
+                      });
   __syncthreads();
-  // few keys fall in bin B1 and they spread over the second byte: plain shared atomics
-  tk_scan<NT>(a.scores + c.row * a.scores_ld, c.lo, c.hi, [&](int, uint32_t key, bool valid) {
-    if (valid && (key >> 24) == b1) atomicAdd(&sh.hist[(key >> 16) & 255u], 1);
-  });
+  const int ns = min(l_n[0], TK_LSEL), nc = min(l_n[1], TK_LCAND);
+  if (threadIdx.x == 0) l_base[0] = ns ? atomicAdd(r.counters, ns) : 0;
+  if (threadIdx.x == 32) l_base[1] = nc ? atomicAdd(r.counters + 1, nc) : 0;
   __syncthreads();
-  if (threadIdx.x < 256 && sh.hist[threadIdx.x]) atomicAdd(r.hist2 + threadIdx.x, sh.hist[threadIdx.x]);
+  for (int e = threadIdx.x; e < ns; e += NT)
+    if (l_base[0] + e < a.k) r.sel[l_base[0] + e] = l_sel[e];
+  for (int e = threadIdx.x; e < nc; e += NT)
+    if (l_base[1] + e < TK_CAND) r.cand[l_base[1] + e] = l_cand[e];
 }
 
-template <int NT>
-__global__ void __launch_bounds__(NT) topk_filter_kernel(IndexArgs a, int q_begin) {
-  __shared__ TopkShared sh;
-  const TkCta c = tk_cta(a, q_begin);
-  if (!c.active) return;
-  const TkRow r = tk_row(a, c.row);
-  tk_find_bin<NT>(r.hist1, c.keff, sh);
-  const uint32_t b1 = (uint32_t)sh.sel;
-  const int above1 = sh.above;
-  __syncthreads();
-  tk_find_bin<NT>(r.hist2, c.keff - above1, sh);
-  const uint32_t t16 = (b1 << 8) | (uint32_t)sh.sel;
-  tk_scan<NT>(a.scores + c.row * a.scores_ld, c.lo, c.hi, [&](int j, uint32_t key, bool valid) {
-    const uint32_t top = key >> 16;
-    const int ps = tk_append(r.counters, valid && top > t16);
-    if (ps >= 0 && ps < a.k) r.sel[ps] = j;
-    const int pc = tk_append(r.counters + 1, valid && top == t16);
-    if (pc >= 0 && pc < TK_CAND)
-      r.cand[pc] = ((unsigned long long)(key & 0xFFFFu) << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)j);
-  });
-}
-
-// Final stage: one CTA per row. Dynamic shared memory: TK_CAND candidates + TK_MAXK outputs.
+// Final stage: one CTA per row. Dynamic shared memory: TK_CAND candidates, TK_MAXK outputs,
+// the bitmap of a row of up to TK_BITMAP_MAX entries.
 template <int NT>
 __global__ void __launch_bounds__(NT) topk_final_kernel(IndexArgs a, int q_begin) {
   __shared__ TopkShared sh;
-  __shared__ int n_out;
+  __shared__ int n_list[2], n_out;
+  __shared__ int rh[TK_H1_BINS];                 // radix digit histogram (<= 11 bits)
   extern __shared__ unsigned long long tk_smem[];
   unsigned long long* cv = tk_smem;                         // [TK_CAND]
   int* outl = reinterpret_cast<int*>(tk_smem + TK_CAND);    // [TK_MAXK]
+  uint32_t* bm = reinterpret_cast<uint32_t*>(outl + TK_MAXK);  // [TK_BITMAP_MAX / 32]
   const int qg = q_begin + blockIdx.x;
   const int b = qg / a.nq, i = qg % a.nq;
   const int Et = visible_entries(a, b, i);
@@ -545,56 +641,134 @@ __global__ void __launch_bounds__(NT) topk_final_kernel(IndexArgs a, int q_begin
   }
   const long long row = qg - a.score_q0;
   const TkRow r = tk_row(a, row);
-  const int n_sel = __ldcg(r.counters), n_cand = __ldcg(r.counters + 1);
-  const int need = keff - n_sel;
-  if (n_cand > TK_CAND || need < 0 || need > n_cand) {
-    // too many scores share the threshold's top 16 bits: select over the whole row
-    const float* sc = a.scores + row * a.scores_ld;
-    select_topk<NT, false>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; });
+  const float* sc = a.scores + row * a.scores_ld;
+  const int ld4 = (int)a.scores_ld - 4;
+  auto whole_row = [&]() { select_topk<NT, false>(sc, Et, keff, sh, [&](int p, int j) { out[p] = j; }); };
+
+  tk_find_bin<NT, TK_H1_BINS / NT>([&](int d) { return __ldcg(r.hist1 + d); }, TK_H1_BINS, keff, sh);
+  const int b1 = sh.sel, c1 = sh.cnt;
+  int above = sh.above;
+  if (threadIdx.x < 2) n_list[threadIdx.x] = 0;
+  __syncthreads();
+  if (b1 < 0) {                                   // inconsistent histogram (not expected)
+    whole_row();
     return;
   }
-  for (int e = threadIdx.x; e < n_cand; e += NT) cv[e] = __ldcg(r.cand + e);
-  for (int e = threadIdx.x; e < n_sel; e += NT) outl[e] = __ldcg(r.sel + e);
+  int n_sel, n_cand, shift;
+  if (c1 <= TK_CAND) {                            // the filter kernel gathered the row's lists
+    shift = TK_H1_SHIFT;
+    n_sel = __ldcg(r.counters);
+    n_cand = __ldcg(r.counters + 1);
+    if (n_sel == above && n_cand <= TK_CAND) {
+      for (int e = threadIdx.x; e < n_cand; e += NT) cv[e] = __ldcg(r.cand + e);
+      for (int e = threadIdx.x; e < n_sel; e += NT) outl[e] = __ldcg(r.sel + e);
+    }
+  } else {
+    // crowded bin B1: the second level (key bits 20..13 of the keys in B1) and the filter
+    // against B1:B2, both over the whole row in this CTA
+    if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+    __syncthreads();
+    const uint32_t ub1 = (uint32_t)b1;
+    tk_scan<NT>(sc, ld4, 0, Et, [&](int, uint32_t key, bool valid) {
+      if (valid && (key >> TK_H1_SHIFT) == ub1) atomicAdd(&sh.hist[(key >> TK_H2_SHIFT) & 255u], 1);
+    });
+    __syncthreads();
+    tk_find_bin<NT, 1>([&](int d) { return sh.hist[d]; }, 256, keff - above, sh);
+    const int b2 = sh.sel;
+    above += sh.above;
+    __syncthreads();
+    if (b2 < 0) {
+      whole_row();
+      return;
+    }
+    shift = TK_H2_SHIFT;
+    const TkBounds bd = tk_bounds((ub1 << 8) | (uint32_t)b2, TK_H2_SHIFT);
+    tk_filter_range<NT>(sc, ld4, 0, Et, bd, n_list, outl, TK_MAXK, cv, TK_CAND,
+                        [](bool, unsigned long long) {});
+    __syncthreads();
+    n_sel = n_list[0];
+    n_cand = n_list[1];
+  }
+  const int need = keff - n_sel;
+  if (n_sel != above || n_cand > TK_CAND || need < 0 || need > n_cand) {
+    // too many scores share the threshold's bits: select over the whole row
+    whole_row();
+    return;
+  }
   if (threadIdx.x == 0) n_out = n_sel;
   __syncthreads();
   if (need > 0) {
-    // radix select of the need-th largest 48-bit candidate value, 8 bits per pass
+    // radix select of the need-th largest candidate value over its 32 + shift bits, digits of
+    // up to 11 bits from the top; stops once the chosen digit's bin is taken whole
     unsigned long long prefix = 0, pmask = 0;
-    int remaining = need;
-    for (int pass = 0; pass < 6; ++pass) {
-      const int shift = 40 - 8 * pass;
-      if (threadIdx.x < 256) sh.hist[threadIdx.x] = 0;
+    int remaining = need, hi = 32 + shift;
+    bool bad = false;
+    while (hi > 0) {
+      const int nb = hi < 11 ? hi : 11, shift = hi - nb, bins = 1 << nb;
+      for (int e = threadIdx.x; e < bins; e += NT) rh[e] = 0;
       __syncthreads();
       for (int e = threadIdx.x; e < n_cand; e += NT) {
         const unsigned long long v = cv[e];
-        if ((v & pmask) == prefix) atomicAdd(&sh.hist[(v >> shift) & 255u], 1);
+        if ((v & pmask) == prefix) atomicAdd(&rh[(v >> shift) & (unsigned)(bins - 1)], 1);
       }
       __syncthreads();
-      const int d = 255 - (int)threadIdx.x;
-      const int h = d >= 0 ? sh.hist[d] : 0;
-      int tot;
-      const int above = block_exclusive_scan<NT>(h, sh.warp_tot, tot);
-      if (d >= 0 && above < remaining && remaining <= above + h) {
-        sh.sel = d;
-        sh.above = above;
+      tk_find_bin<NT, (TK_H1_BINS + NT - 1) / NT>([&](int d) { return rh[d]; }, bins, remaining, sh);
+      const int sel = sh.sel, above = sh.above, cnt = sh.cnt;
+      __syncthreads();
+      if (sel < 0) {
+        bad = true;
+        break;
       }
-      __syncthreads();
-      remaining -= sh.above;
-      prefix |= (unsigned long long)sh.sel << shift;
-      pmask |= 255ull << shift;
-      __syncthreads();
+      remaining -= above;
+      prefix |= (unsigned long long)sel << shift;
+      pmask |= (unsigned long long)(bins - 1) << shift;
+      hi = shift;
+      if (cnt == remaining) break;                 // the whole bin is selected
     }
-    // candidate values are distinct: exactly `need` of them are >= the threshold
+    if (bad || (hi == 0 && remaining != 1)) {      // inconsistent candidates (not expected)
+      whole_row();
+      return;
+    }
+    // exactly `need` candidates lie at or above the prefix in their masked bits
     for (int e = threadIdx.x; e < n_cand; e += NT) {
       const unsigned long long v = cv[e];
-      if (v >= prefix) {
+      if ((v & pmask) >= prefix) {
         const int p = atomicAdd(&n_out, 1);
         if (p < TK_MAXK) outl[p] = (int)(0xFFFFFFFFu - (uint32_t)(v & 0xFFFFFFFFull));
       }
     }
     __syncthreads();
   }
-  // ascending entry order: bitonic sort of the keff selected entries (padded to a power of 2)
+  if (Et <= TK_BITMAP_MAX) {
+    // ascending entry order: mark the selected entries in a bitmap of the row, then every
+    // thread emits the set bits of its words at its block-scan offset
+    const int nw = (Et + 31) >> 5, per = (nw + NT - 1) / NT;
+    for (int e = threadIdx.x; e < nw; e += NT) bm[e] = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < keff; e += NT) {
+      const int j = outl[e];
+      if (j >= 0 && j < Et) atomicOr(&bm[j >> 5], 1u << (j & 31));
+    }
+    __syncthreads();
+    const int w0 = threadIdx.x * per;
+    int cnt = 0;
+    for (int q = 0; q < per; ++q)
+      if (w0 + q < nw) cnt += __popc(bm[w0 + q]);
+    int tot;
+    int pos = block_exclusive_scan<NT>(cnt, sh.warp_tot, tot);
+    for (int q = 0; q < per; ++q) {
+      if (w0 + q >= nw) break;
+      uint32_t x = bm[w0 + q];
+      while (x) {
+        const int bit = __ffs(x) - 1;
+        if (pos < keff) out[pos] = 32 * (w0 + q) + bit;
+        ++pos;
+        x &= x - 1u;
+      }
+    }
+    return;
+  }
+  // longer rows: bitonic sort of the keff selected entries (padded to a power of 2)
   int n2 = 1;
   while (n2 < keff) n2 <<= 1;
   for (int e = keff + threadIdx.x; e < n2; e += NT) outl[e] = 0x7FFFFFFF;
@@ -620,20 +794,18 @@ __global__ void __launch_bounds__(NT) topk_final_kernel(IndexArgs a, int q_begin
 int launch_topk(const IndexArgs& a, int q_begin, int q_count, cudaStream_t st) {
   if (q_count <= 0) return DSV4_OK;
   if (a.topk_pipe) {
-    constexpr int kFinalSmem = TK_CAND * 8 + TK_MAXK * 4;
     static bool attr_set = false;
     if (!attr_set) {
-      const cudaError_t e = cudaFuncSetAttribute(topk_final_kernel<1024>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kFinalSmem);
+      const cudaError_t e = cudaFuncSetAttribute(topk_final_kernel<TK_FINAL_NT>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, TK_FINAL_SMEM);
       if (e != cudaSuccess) return fail(DSV4_ERR_CUDA, "top-k: %s", cudaGetErrorString(e));
       attr_set = true;
     }
     // (headers zeroed by topk_prepare; the score kernel may have built hist1 already)
-    const dim3 grid((a.max_e + TK_PASS - 1) / TK_PASS, q_count);
-    if (!a.hist1_done) topk_hist1_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
-    topk_hist2_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
-    topk_filter_kernel<256><<<grid, 256, 0, st>>>(a, q_begin);
-    topk_final_kernel<1024><<<q_count, 1024, kFinalSmem, st>>>(a, q_begin);
+    if (!a.hist1_done)
+      topk_hist1_kernel<256><<<dim3((a.max_e + TK_PASS - 1) / TK_PASS, q_count), 256, 0, st>>>(a, q_begin);
+    topk_filter_kernel<256><<<dim3((a.max_e + TK_FPASS - 1) / TK_FPASS, q_count), 256, 0, st>>>(a, q_begin);
+    topk_final_kernel<TK_FINAL_NT><<<q_count, TK_FINAL_NT, TK_FINAL_SMEM, st>>>(a, q_begin);
   } else if (a.nseg > 1) {
     topk_seg_kernel<256><<<dim3(a.nseg, q_count), 256, 0, st>>>(a, q_begin);
     if ((long long)a.nseg * a.k >= 4096)

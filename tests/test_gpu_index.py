@@ -173,6 +173,27 @@ def test_index_decode_mixed_lengths_dynamic_units(dsv4):
                    what="decode mixed")
 
 
+def test_index_decode_concentrated_scores_two_levels(dsv4):
+    """Long decode rows whose scores all lie within a few per cent of each other: the bin of
+    the top 11 key bits holding the k-th largest score holds nearly the whole row, so the
+    threshold takes the second histogram level (key bits 20..13)."""
+    shape = preset("flash_csa_prefill", B=2)
+    lens = [4 * 40000 + 1, 4 * 23000 + 2]
+    rows = [L // 4 for L in lens]
+    offs = list(np.concatenate([[0], np.cumsum(rows)[:-1]]).astype(np.int64))
+    g = Generator(43)
+    base = g.normal("base", (1, 128), 128 ** -0.5)
+    KI = (base + 0.05 * g.normal("KI", (int(sum(rows)) + 1, 128), 128 ** -0.5)).to(torch.bfloat16)
+    qI = (base.reshape(1, 1, 1, 128) + 0.05 * g.normal("qI", (2, 1, 64, 128), 128 ** -0.5))
+    qI = qI.to(torch.bfloat16)
+    w = g.uniform("wI", (2, 1, 64), 0.5, 1.0)
+    pos0 = [L - 1 for L in lens]
+    s64 = O.index_scores_query(O.as_f64(qI)[0, 0], O.as_f64(w)[0, 0], O.as_f64(KI), pos0[0], 4)
+    top = np.sort(s64)[::-1]
+    assert top[0] < 1.2 * top[-1]                      # one quarter-octave bin or two
+    _run_and_check(dsv4, qI, w, KI, offs, pos0, 4, 512, [(0, 0), (1, 0)], what="concentrated")
+
+
 def test_index_many_long_rows(dsv4):
     """More than 1024 queries whose rows exceed 16384 entries: the workspace path selects per
     16384-entry segment and merges the candidates (the threshold pipeline serves requests with
