@@ -144,8 +144,9 @@ int dsv4_quantize_fp4(const void* x, uint8_t* codes, uint8_t* scales, int64_t ro
 /* Bytes of workspace dsv4_index_topk needs for a bf16 / fp32 request: per chunk of queries
  * (at most 256 MiB of rows) the fp32 score rows (4 * round4(max_entries) bytes each) and,
  * for rows longer than 16384 entries, a top-k region per row: with at most 1024 rows in the
- * request and k <= 4096 the threshold top-k's (histograms, the entries above the threshold
- * and up to 8192 boundary candidates: 4 KiB + round256(4k) + 64 KiB), otherwise the
+ * request and k <= 4096 the threshold top-k's (a 2048-bin histogram and counters, the
+ * entries above the threshold and up to 8192 boundary candidates: 8448 bytes +
+ * round256(4k) + 64 KiB), otherwise the
  * per-segment candidates (8k bytes per 16384-entry segment). Each of the two regions is
  * rounded up to 256 bytes. A smaller workspace makes smaller chunks; a larger one is not
  * used.

@@ -88,13 +88,13 @@ def _r256(x):
 @pytest.mark.parametrize("B,nq,E,k", [(64, 1, 262144, 512), (1, 4, 16385, 512), (1, 1024, 40000, 4096)])
 def test_workspace_size_threshold_topk_rows(lib, B, nq, E, k):
     """Requests of at most 1024 rows longer than 16384 entries: score rows plus the threshold
-    top-k region of 4 KiB + round256(4k) + 64 KiB per row, as the header states."""
+    top-k region of 8448 bytes + round256(4k) + 64 KiB per row, as the header states."""
     f = lib.dsv4_index_topk_workspace_size
     f.restype = ctypes.c_size_t
     rows = B * nq
-    per = 4 * ((E + 3) // 4 * 4) + 4096 + _r256(4 * k) + 65536
+    per = 4 * ((E + 3) // 4 * 4) + 8448 + _r256(4 * k) + 65536
     rows = min(rows, (256 << 20) // per)
-    want = _r256(rows * 4 * ((E + 3) // 4 * 4)) + _r256(rows * (4096 + _r256(4 * k) + 65536))
+    want = _r256(rows * 4 * ((E + 3) // 4 * 4)) + _r256(rows * (8448 + _r256(4 * k) + 65536))
     assert f(B, nq, E, k) == want
 
 
