@@ -172,6 +172,7 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   a.cand = nullptr;
   a.cand_row_bytes = 0;
   a.hist1_done = 0;
+  a.k_fp4 = 0;
   a.q_map_q0 = 0;
   a.q_map_rows = 0;
   cudaStream_t st = (cudaStream_t)stream;
@@ -189,7 +190,10 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
   const long long wsb = ws_ok ? (long long)workspace_bytes : 0;
   bool fp4x = ws_ok && fp4_tensor_path(qdtype, H_I, c_I) && ki_rows > 0 &&
               !(reinterpret_cast<uintptr_t>(KI) & 7u) && !(reinterpret_cast<uintptr_t>(qI) & 7u);
-  const long long kx = fp4x ? ki_rows * c_I * 2 : 0;
+  // one query per sequence (decode) with 16-byte aligned key codes and scales: the score
+  // kernel expands K^I itself as it streams it, and only q^I goes through the workspace (f16)
+  const bool f4k = fp4x && nq == 1 && ki_rows >= 130 && aligned16(KI) && aligned16(KI_scales);
+  const long long kx = fp4x && !f4k ? ki_rows * c_I * 2 : 0;
   const long long qx = fp4x ? (long long)H_I * c_I * 2 : 0;
   long long rows;
   if (scores_out) {
@@ -232,14 +236,18 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     const IxLayout L = ix_layout(rows, ld, scores_out ? 0 : (a.cand ? cand : 0), kx, qx,
                                  !scores_out);
     char* base = static_cast<char*>(workspace);
-    __nv_bfloat16* kbuf = reinterpret_cast<__nv_bfloat16*>(base);
-    int s = launch_fp4_expand(static_cast<const uint8_t*>(KI), KI_scales, ki_rows, c_I, kbuf, st);
-    if (s != DSV4_OK) return s;
-    ax.qdtype = DSV4_BF16;
-    ax.KI = kbuf;
-    ax.KI_scales = nullptr;
+    ax.qdtype = DSV4_BF16;                         // a 16-bit query tile (f16 with FP4 keys)
     ax.qI = base + L.qx;
     ax.qI_scales = nullptr;
+    if (f4k) {
+      ax.k_fp4 = 1;                                // KI / KI_scales stay the FP4 pool
+    } else {
+      __nv_bfloat16* kbuf = reinterpret_cast<__nv_bfloat16*>(base);
+      int s = launch_fp4_expand(static_cast<const uint8_t*>(KI), KI_scales, ki_rows, c_I, kbuf, st);
+      if (s != DSV4_OK) return s;
+      ax.KI = kbuf;
+      ax.KI_scales = nullptr;
+    }
   }
   const int chunk = (int)rows;
   for (int q0 = 0; q0 < total; q0 += chunk) {
@@ -251,9 +259,11 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     if (s != DSV4_OK) return s;
     if (fp4x) {
       const long long qrow0 = (long long)q0 * H_I;
-      s = launch_fp4_expand(static_cast<const uint8_t*>(qI) + qrow0 * (c_I / 2),
-                            qI_scales + qrow0 * (c_I / 16), (long long)qn * H_I, c_I,
-                            static_cast<__nv_bfloat16*>(const_cast<void*>(ax.qI)), st);
+      const uint8_t* qc = static_cast<const uint8_t*>(qI) + qrow0 * (c_I / 2);
+      const uint8_t* qs = qI_scales + qrow0 * (c_I / 16);
+      void* qdst = const_cast<void*>(ax.qI);
+      s = f4k ? launch_fp4_expand_f16(qc, qs, (long long)qn * H_I, c_I, static_cast<__half*>(qdst), st)
+              : launch_fp4_expand(qc, qs, (long long)qn * H_I, c_I, static_cast<__nv_bfloat16*>(qdst), st);
       if (s != DSV4_OK) return s;
       ax.q_map_q0 = q0;
       ax.q_map_rows = (long long)qn * H_I;
@@ -263,7 +273,8 @@ extern "C" int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_sca
     }
     if (s != DSV4_OK) return s;
     if (q0 == 0)
-      trace_path(used ? (fp4x ? "index scores: tcgen05 (FP4 expanded to bf16)" : "index scores: tcgen05")
+      trace_path(used ? (f4k ? "index scores: tcgen05 (FP4 keys expanded in the kernel, f16)"
+                             : fp4x ? "index scores: tcgen05 (FP4 expanded to bf16)" : "index scores: tcgen05")
                       : "index scores: CUDA cores");
     if (!used) {
       s = launch_index_scores_simt(a, q0, qn, max_entries, st);

@@ -1,5 +1,7 @@
 // Shared declarations of the indexer / top-k kernels.
 #pragma once
+#include <cuda_fp16.h>
+
 #include "dsv4_common.cuh"
 
 namespace dsv4 {
@@ -30,6 +32,9 @@ struct IndexArgs {
   //    top TK_H1_BITS key bits (TK_HDR bytes); hist1_done: the score kernel built hist1;
   //  * nseg > 1 (many rows): per-segment selection then a merge; the region holds nseg * k
   //    candidate scores, then their nseg * k entry indices.
+  // k_fp4 = 1: K^I stays FP4 (KI = e2m1 codes [ki_rows, c_I/2], KI_scales = E4M3 [ki_rows,
+  // c_I/16]) and is expanded inside the tensor-core score kernel; qI is then f16
+  int k_fp4;
   int topk_pipe;
   int nseg;
   char* cand;
@@ -117,5 +122,7 @@ int topk_segments(int max_entries);
 // FP4 codes [rows, cols/2] + E4M3 scales [rows, cols/16] -> bf16 [rows, cols] (exact).
 int launch_fp4_expand(const uint8_t* codes, const uint8_t* scales, long long rows, int cols,
                       __nv_bfloat16* out, cudaStream_t st);
+int launch_fp4_expand_f16(const uint8_t* codes, const uint8_t* scales, long long rows, int cols,
+                          __half* out, cudaStream_t st);
 
 }  // namespace dsv4

@@ -122,6 +122,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
 // Add `bytes` to the expected transaction count of the current phase (no arrival).
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
@@ -308,6 +317,16 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t start, uint32_t lbo, ui
   return d;
 }
 
+// Instruction descriptor, kind::f16: f16 x f16 -> fp32, dense (A and B of the same type).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                       // D format: fp32
+         | (0u << 7)                     // A format: f16
+         | (0u << 10)                    // B format: f16
+         | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
+         | ((uint32_t)(N >> 3) << 17)    // N / 8
+         | ((uint32_t)(M >> 4) << 24);   // M / 16
+}
+
 // Instruction descriptor, kind::f16: bf16 x bf16 -> fp32, dense.
 // a_mn / b_mn: operand is MN-major (1) or K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
@@ -323,6 +342,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
 
 // Host: encode a 2D bf16/uint8 tensor map (row-major [rows, cols], 128-byte swizzle).
 // Returns DSV4_OK or a status with the reason recorded.
+// Host: a 3D tensor map with explicit byte strides of dimensions 1 and 2 (no swizzle); the box
+// lands in shared memory with dimension 0 innermost.
+int encode_tensor_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                         const uint64_t dims[3], const uint64_t strides[2], const uint32_t box[3]);
 int encode_tensor_map_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                          int elem_bytes, uint64_t cols, uint64_t rows, uint32_t box_cols,
                          uint32_t box_rows, CUtensorMapSwizzle swizzle);

@@ -233,6 +233,44 @@ def test_index_fp4(dsv4, index_path):
                    KI64=KI64, c_I=128, what=f"fp4 {index_path}")
 
 
+def _fp4_decode_case(lens, seed, k, pad_front=0):
+    """One query per sequence at its end; FP4 q^I and K^I (the oracle's quantiser), keys of
+    sequence b from row pad_front + sum(rows before b) of one pool."""
+    shape = preset("pro_csa_prefill", B=len(lens))
+    rows = [L // 4 for L in lens]
+    offs = list((pad_front + np.concatenate([[0], np.cumsum(rows)[:-1]])).astype(np.int64))
+    total = pad_front + int(sum(rows))
+    qI, w, KI = _inputs(shape, 1, total, seed)
+    qc, qs = O.quantize_fp4(qI.float().reshape(-1, 128))
+    kc, ks = O.quantize_fp4(KI.float())
+    qI64 = O.dequantize_fp4(qc, qs, 128).reshape(len(lens), 1, 64, 128)
+    KI64 = O.dequantize_fp4(kc, ks, 128)
+    qc_t = torch.from_numpy(qc).reshape(len(lens), 1, 64, 64)
+    return dict(qI=qc_t, w=w, KI=torch.from_numpy(kc), offs=offs, pos0=[L - 1 for L in lens],
+                m=4, k=k, positions=[(b, 0) for b in range(len(lens))],
+                qI_sc=torch.from_numpy(qs), KI_sc=torch.from_numpy(ks), qI64=qI64, KI64=KI64,
+                c_I=128)
+
+
+def test_index_fp4_decode_long_rows(dsv4):
+    """FP4 decode over long rows: the score kernel reads e2m1 codes and E4M3 scales of the key
+    pool and expands them itself (threshold top-k, dynamically scheduled units). The pool
+    starts two rows in, so most sequences start at odd rows (scale pairs straddle their
+    blocks), and has an odd row count (its last row's scales are read on their own)."""
+    lens = [4 * 20001 + 3, 4 * 17000, 4 * 3000 + 1, 4 * 40000 + 2]
+    case = _fp4_decode_case(lens, 51, 512, pad_front=2)
+    assert case["KI"].shape[0] % 2 == 1 and sum(o % 2 for o in case["offs"]) >= 2
+    _run_and_check(dsv4, what="fp4 decode long", **case)
+
+
+def test_index_fp4_decode_short_rows(dsv4):
+    """FP4 decode over rows shorter than the threshold top-k's (one CTA per unit), including
+    a row of one entry and the pool's last row."""
+    lens = [4 * 3 + 1, 4 * 129, 4 * 1000 + 2, 4 * 4097 + 3, 7]
+    case = _fp4_decode_case(lens, 52, 256)
+    _run_and_check(dsv4, what="fp4 decode short", **case)
+
+
 def test_index_k_zero_and_short(dsv4):
     shape = preset("tiny_csa")
     qI, w, KI = _inputs(shape, 10, 2, 4)
