@@ -431,6 +431,50 @@ def run_decode(args, dev, stream):
     b_csa8 = sum(e * cI * 2 for e in E4) + B * HI * (cI * 2 + 4) + B * k * 4 \
         + sum(min(k, e) for e in E4) * row8 + B * w * c * 2 + 2 * B * H * c * 2
     nbytes8 = sum(b_csa8 if kind == "csa" else b_hca for kind in D["layers"])
+    # and with the index keys in their production format too: FP4 (e2m1 + one E4M3 scale per
+    # 16, 72 bytes per key), expanded inside the score kernel
+    kc, ks = dsv4.dsv4_quantize_fp4(KI)
+    qc, qs = dsv4.dsv4_quantize_fp4(qI.reshape(-1, cI))
+    qc = qc.view(B, 1, HI, cI // 2)
+    ws4 = torch.empty(dsv4.dsv4_index_topk_workspace_size_ex(dsv4.FP4, B, 1, HI, cI, maxE, k, kc.shape[0]),
+                      dtype=torch.uint8, device=dev)
+
+    def layer_csa_prod():
+        dsv4.dsv4_index_topk(qc, wI, kc, off4, pos0, D["m_csa"], k, maxE, qI_scales=qs, KI_scales=ks,
+                             c_I=cI, idx=idx, counts=cnt, workspace=ws4)
+        dsv4.dsv4_hybrid_sparse_attn_fp8(Q, codes, scales, rope, off4, idx, cnt, local, pos0, D["m_csa"], w,
+                                         sink, O=O, lse=lse, workspace=fws)
+
+    def step_prod():
+        for kind in D["layers"]:
+            (layer_csa_prod if kind == "csa" else layer_hca)()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step_prod()
+    dsv4.dsv4_check_errors()
+    tsp = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step_prod()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        tsp.append(e0.elapsed_time(e1))
+    dsv4.dsv4_check_errors()
+    msp = statistics.median(tsp)
+    key4 = cI // 2 + cI // 16
+    b_csap = sum(e * key4 for e in E4) + B * HI * (cI // 2 + cI // 16 + 4) + B * k * 4 \
+        + sum(min(k, e) for e in E4) * row8 + B * w * c * 2 + 2 * B * H * c * 2
+    nbytesp = sum(b_csap if kind == "csa" else b_hca for kind in D["layers"])
+    production = {"what": "the same step with both CSA pools in their production formats: main entries "
+                          f"FP8 ({row8} bytes) and index keys FP4 (e2m1 + E4M3 per 16 = {key4} bytes, "
+                          "expanded to f16 inside the score kernel); HCA pools bf16",
+                  "ms_per_step": round(msp, 4), "bytes_per_step": nbytesp,
+                  "achieved_gbs": round(nbytesp / (msp / 1e3) / 1e9, 1),
+                  "frac": round(nbytesp / (msp / 1e3) / 1e9 / peak, 4), "steps": steps,
+                  "csa_index_key_bytes": {"bf16": int(sum(E4)) * cI * 2, "fp4": int(sum(E4)) * key4}}
     packed = {"what": "the same step with the CSA layers' compressed main pool stored as FP8 entries "
                       f"(448 FP8 + 64 bf16 channels + 7 fp32 scales = {row8} bytes per entry; index keys "
                       "and the HCA pools bf16)",
@@ -443,7 +487,8 @@ def run_decode(args, dev, stream):
                         f"{'/'.join(D['layers'])} (CSA m=4, HCA m'=128), bf16 pools in HBM",
             "ms_per_step": round(ms, 4), "bytes_per_step": nbytes, "achieved_gbs": round(gbps, 1),
             "peak_gbs": peak, "frac": round(gbps / peak, 4), "peak_source": f"{src} hbm_gbs",
-            "steps": steps, "l2": "flushed (256 MiB write) before every step", "packed_pools": packed}
+            "steps": steps, "l2": "flushed (256 MiB write) before every step", "packed_pools": packed,
+            "production_pools": production}
 
 
 def run_decode_state(args, dev, stream):

@@ -154,9 +154,12 @@ int dsv4_quantize_fp4(const void* x, uint8_t* codes, uint8_t* scales, int64_t ro
 size_t dsv4_index_topk_workspace_size(int B, int nq, int max_entries, int k);
 
 /* The same for any operand type. FP4 operands at H_I = 64, c_I = 128 are scored on the
- * tensor cores after an exact expansion to bf16 in the workspace (K^I: ki_rows x c_I, the
- * chunk's q^I rows); this size includes that room. With less room (or with scores_out and a
- * workspace too small for the expansion of every query) FP4 is scored on CUDA cores. */
+ * tensor cores after an exact expansion of the chunk's q^I rows in the workspace and, for
+ * requests with several queries per sequence, of K^I to bf16 (ki_rows x c_I) too; one query
+ * per sequence (decode) with 16-byte aligned KI and KI_scales and at least 130 key rows reads
+ * the FP4 key pool itself and expands it inside the score kernel. This size includes the room
+ * for the K^I expansion either way. With less room (or with scores_out and a workspace too
+ * small for the expansion of every query) FP4 is scored on CUDA cores. */
 size_t dsv4_index_topk_workspace_size_ex(int qdtype, int B, int nq, int H_I, int c_I,
                                          int max_entries, int k, int64_t ki_rows);
 
@@ -206,10 +209,12 @@ int dsv4_index_topk(int qdtype, const void* qI, const uint8_t* qI_scales, const 
  *     with DSV4_ERR_INVALID_ARG before anything is enqueued.
  *   - Queries are processed in chunks whose score rows fit in the scratch; long rows
  *     (more than 16384 entries) also need their top-k region there and get smaller chunks.
- *   - DSV4_FP4 operands are scored on the tensor cores only while the exact bf16 expansion
- *     of the whole key pool (256 bytes per key row at c_I = 128) fits in the scratch beside
- *     at least one score row: above roughly 32,000 key rows such requests are scored on
- *     CUDA cores instead (same results up to fp32 rounding order, lower throughput).
+ *   - DSV4_FP4 operands of requests with several queries per sequence are scored on the
+ *     tensor cores only while the exact bf16 expansion of the whole key pool (256 bytes per
+ *     key row at c_I = 128) fits in the scratch beside at least one score row: above roughly
+ *     32,000 key rows such requests are scored on CUDA cores instead (same results up to
+ *     fp32 rounding order, lower throughput). One query per sequence (decode) needs no such
+ *     room: the score kernel expands the FP4 keys it streams.
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
  *   - Every call on a device shares the one array. The scratch holds score rows that

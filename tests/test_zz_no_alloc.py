@@ -95,9 +95,9 @@ def test_noalloc_fp4_operands_match_workspace_entry_point(dsv4):
 
 def test_noalloc_long_rows_and_large_fp4_pool(dsv4):
     """Decode-length rows (one query per sequence over 40k-90k entries, beyond the one-CTA
-    top-k) and a FP4 key pool whose expansion does not fit in the fixed scratch (those
-    requests are scored on CUDA cores): checked against the fp64 oracle under the stated
-    tie rule, on two calls in a row."""
+    top-k) and a FP4 key pool far larger than a bf16 expansion in the fixed scratch could
+    hold (decode requests expand the FP4 keys inside the score kernel): checked against the
+    fp64 oracle under the stated tie rule, on two calls in a row."""
     import numpy as np
     import oracle as O
     from parity_util import check_topk_query
