@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "DSV4Error", "lib", "LIB_PATH", "F32", "BF16", "FP4",
     "dsv4_compress", "dsv4_compress_decode", "dsv4_ring_write", "decode_tail_shape",
+    "dsv4_decode_state", "decode_ring_job", "decode_compress_job",
     "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
     "dsv4_index_topk_workspace_size_ex",
     "dsv4_hybrid_sparse_attn", "dsv4_hybrid_sparse_attn_workspace_size", "dsv4_check_errors",
@@ -50,6 +51,20 @@ lib.dsv4_compress_decode.restype = _I
 lib.dsv4_compress_decode.argtypes = [_I, _P, _P, _P, _P, _P, _P, _L, _P, _I, _I, _I, _I, _P]
 lib.dsv4_ring_write.restype = _I
 lib.dsv4_ring_write.argtypes = [_I, _P, _P, _I, _P, _I, _I, _P]
+
+
+class _DecodeJob(ctypes.Structure):
+    """dsv4_decode_job of include/dsv4.h."""
+    _fields_ = [("kind", ctypes.c_int), ("c", ctypes.c_int), ("m", ctypes.c_int),
+                ("overlap", ctypes.c_int), ("R", ctypes.c_int), ("reserved", ctypes.c_int),
+                ("x_new", ctypes.c_void_p), ("z_new", ctypes.c_void_p), ("bias", ctypes.c_void_p),
+                ("tail", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("pool_row_off", ctypes.c_void_p), ("pool_rows", ctypes.c_int64)]
+
+
+DECODE_MAX_JOBS = 32
+lib.dsv4_decode_state.restype = _I
+lib.dsv4_decode_state.argtypes = [_I, ctypes.POINTER(_DecodeJob), _I, _P, _I, _P]
 lib.dsv4_quantize_fp4.restype = _I
 lib.dsv4_quantize_fp4.argtypes = [_P, _P, _P, _L, _I, _P]
 lib.dsv4_index_topk_workspace_size.restype = _S
@@ -176,6 +191,55 @@ def dsv4_ring_write(kv_new: torch.Tensor, local: torch.Tensor, pos: torch.Tensor
         raise ValueError(f"local must be [{B}, R, {c}]")
     _check(lib.dsv4_ring_write(_code(kv_new.dtype), _ptr(kv_new), _ptr(local), local.shape[1],
                                _ptr(pos), B, c, _stream(stream)), "dsv4_ring_write")
+
+
+def decode_ring_job(kv_new: torch.Tensor, local: torch.Tensor):
+    """A dsv4_decode_state job: the dsv4_ring_write of kv_new [B, c] into local [B, R, c]."""
+    _dev(kv_new, "kv_new"), _dev(local, "local", kv_new.dtype)
+    B, c = kv_new.shape
+    if local.shape[0] != B or local.shape[2] != c:
+        raise ValueError(f"local must be [{B}, R, {c}]")
+    job = _DecodeJob(kind=0, c=c, m=0, overlap=0, R=local.shape[1], reserved=0,
+                     x_new=kv_new.data_ptr(), z_new=None, bias=None, tail=None, out=local.data_ptr(),
+                     pool_row_off=None, pool_rows=0)
+    return job, kv_new.dtype, B, (kv_new, local)
+
+
+def decode_compress_job(C_new: torch.Tensor, Z_new: torch.Tensor, bias: torch.Tensor,
+                        tail: torch.Tensor, pool: torch.Tensor, pool_row_off: torch.Tensor,
+                        m: int, overlap: bool):
+    """A dsv4_decode_state job: the dsv4_compress_decode of one compressor (same arguments)."""
+    _dev(C_new, "C_new"), _dev(Z_new, "Z_new", C_new.dtype), _dev(bias, "bias", torch.float32)
+    B, width = C_new.shape
+    S = 2 if overlap else 1
+    c = width // S
+    _dev(tail, "tail", C_new.dtype), _dev(pool, "pool", C_new.dtype)
+    _dev(pool_row_off, "pool_row_off", torch.int64)
+    if tuple(tail.shape) != decode_tail_shape(B, c, m, overlap):
+        raise ValueError(f"tail must be {decode_tail_shape(B, c, m, overlap)}, got {tuple(tail.shape)}")
+    if pool.shape[-1] != c:
+        raise ValueError(f"pool rows must have {c} channels")
+    job = _DecodeJob(kind=1, c=c, m=m, overlap=1 if overlap else 0, R=0, reserved=0,
+                     x_new=C_new.data_ptr(), z_new=Z_new.data_ptr(), bias=bias.data_ptr(), tail=tail.data_ptr(),
+                     out=pool.data_ptr(), pool_row_off=pool_row_off.data_ptr(), pool_rows=pool.numel() // c)
+    return job, C_new.dtype, B, (C_new, Z_new, bias, tail, pool, pool_row_off)
+
+
+def dsv4_decode_state(jobs, pos: torch.Tensor, stream=None) -> None:
+    """One launch for a token's ring writes and compressor states: `jobs` from decode_ring_job
+    / decode_compress_job (same dtype and batch), pos int32 [B]."""
+    _dev(pos, "pos", torch.int32)
+    if not jobs:
+        return
+    if len(jobs) > DECODE_MAX_JOBS:
+        raise ValueError(f"at most {DECODE_MAX_JOBS} jobs per call")
+    dtypes = {j[1] for j in jobs}
+    batches = {j[2] for j in jobs}
+    if len(dtypes) != 1 or batches != {pos.shape[0]}:
+        raise ValueError("jobs must share one dtype and the batch of pos")
+    arr = (_DecodeJob * len(jobs))(*[j[0] for j in jobs])
+    _check(lib.dsv4_decode_state(_code(next(iter(dtypes))), arr, len(jobs), _ptr(pos), pos.shape[0],
+                                 _stream(stream)), "dsv4_decode_state")
 
 
 def dsv4_quantize_fp4(x: torch.Tensor, codes: Optional[torch.Tensor] = None,

@@ -18,15 +18,15 @@ namespace dsv4 {
 // The emitted entry goes to `pool` (dtype T), or -- FP8 -- through shared memory into the
 // production main-KV format (fp8_kv.cuh): the entry rounded to T, then quantised, so an FP8
 // pool holds exactly the quantisation of the T pool's row.
+// Sequence b's token (one CTA of 256 threads): its (C, Z) rows into the tail and, when t + 1
+// completes a block, the entry into the pool. FP8: `entry` is shared memory of c floats.
 template <typename T, bool FP8>
-__global__ void __launch_bounds__(256) compress_decode_kernel(
-    const T* __restrict__ C_new, const T* __restrict__ Z_new, const float* __restrict__ bias,
+__device__ __forceinline__ void compress_decode_seq(
+    int b, const T* __restrict__ C_new, const T* __restrict__ Z_new, const float* __restrict__ bias,
     T* __restrict__ tail, T* __restrict__ pool, const int64_t* __restrict__ pool_row_off,
     long long pool_rows, const int32_t* __restrict__ pos, int c, int m, int overlap,
     uint8_t* __restrict__ codes, float* __restrict__ scales, __nv_bfloat16* __restrict__ rope_out,
-    int rope) {
-  extern __shared__ float entry[];                          // FP8: the entry, c values
-  const int b = blockIdx.x;
+    int rope, float* entry) {
   const int S = overlap ? 2 : 1;
   const int T_slots = S * m;
   const long long width = (long long)S * c;
@@ -52,20 +52,37 @@ __global__ void __launch_bounds__(256) compress_decode_kernel(
     if (threadIdx.x == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
     return;
   }
+  constexpr int PF = 8;                                      // positions whose loads are in flight
   for (int ch = threadIdx.x; ch < c; ch += blockDim.x) {
     float mx = -INFINITY, den = 0.f, acc = 0.f;
     for (int half = (overlap && i > 0) ? 1 : 0; half >= 0; --half) {
       const long long tok0 = half ? m * (i - 1) : m * i;
-      for (int p = 0; p < m; ++p) {
-        const T* r = tail_b + ((tok0 + p) % T_slots) * 2 * width + half * c + ch;
-        float l = to_f32(r[width]) + bias[((long long)half * m + p) * c + ch];
-        float x = to_f32(r[0]);
-        if (l > mx) {
-          float e = expf(mx - l);
-          den = den * e + 1.f; acc = acc * e + x; mx = l;
-        } else {
-          float e = expf(l - mx);
-          den += e; acc = fmaf(e, x, acc);
+      for (int p0 = 0; p0 < m; p0 += PF) {
+        // the next PF positions' rows are loaded before any is used (a dependent load per
+        // position made an emission latency-bound); the online softmax then takes them in
+        // position order, as the prefill compressor does
+        float xs[PF], ls[PF];
+#pragma unroll
+        for (int u = 0; u < PF; ++u) {
+          xs[u] = 0.f;
+          ls[u] = -INFINITY;
+          if (p0 + u < m) {
+            const T* r = tail_b + ((tok0 + p0 + u) % T_slots) * 2 * width + half * c + ch;
+            xs[u] = to_f32(r[0]);
+            ls[u] = to_f32(r[width]) + bias[((long long)half * m + p0 + u) * c + ch];
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < PF; ++u) {
+          if (p0 + u >= m) break;
+          const float l = ls[u], x = xs[u];
+          if (l > mx) {
+            float e = expf(mx - l);
+            den = den * e + 1.f; acc = acc * e + x; mx = l;
+          } else {
+            float e = expf(l - mx);
+            den += e; acc = fmaf(e, x, acc);
+          }
         }
       }
     }
@@ -90,11 +107,22 @@ __global__ void __launch_bounds__(256) compress_decode_kernel(
   }
 }
 
+template <typename T, bool FP8>
+__global__ void __launch_bounds__(256) compress_decode_kernel(
+    const T* __restrict__ C_new, const T* __restrict__ Z_new, const float* __restrict__ bias,
+    T* __restrict__ tail, T* __restrict__ pool, const int64_t* __restrict__ pool_row_off,
+    long long pool_rows, const int32_t* __restrict__ pos, int c, int m, int overlap,
+    uint8_t* __restrict__ codes, float* __restrict__ scales, __nv_bfloat16* __restrict__ rope_out,
+    int rope) {
+  extern __shared__ float entry[];                          // FP8: the entry, c values
+  compress_decode_seq<T, FP8>(blockIdx.x, C_new, Z_new, bias, tail, pool, pool_row_off, pool_rows,
+                              pos, c, m, overlap, codes, scales, rope_out, rope, entry);
+}
+
 template <typename T>
-__global__ void __launch_bounds__(256) ring_write_kernel(const T* __restrict__ kv_new,
-                                                         T* __restrict__ local, int R,
-                                                         const int32_t* __restrict__ pos, int c) {
-  const int b = blockIdx.x;
+__device__ __forceinline__ void ring_write_seq(int b, const T* __restrict__ kv_new,
+                                               T* __restrict__ local, int R,
+                                               const int32_t* __restrict__ pos, int c) {
   const int t = pos[b];
   if (t < 0) {
     if (threadIdx.x == 0) flag_status(DSV4_ERR_DEVICE_BOUNDS);
@@ -102,6 +130,32 @@ __global__ void __launch_bounds__(256) ring_write_kernel(const T* __restrict__ k
   }
   T* dst = local + ((long long)b * R + t % R) * c;
   for (int j = threadIdx.x; j < c; j += blockDim.x) dst[j] = kv_new[(long long)b * c + j];
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) ring_write_kernel(const T* __restrict__ kv_new,
+                                                         T* __restrict__ local, int R,
+                                                         const int32_t* __restrict__ pos, int c) {
+  ring_write_seq<T>(blockIdx.x, kv_new, local, R, pos, c);
+}
+
+// Every job of a token's state update in one launch: CTA (b, j) performs job j for sequence b.
+struct DecodeJobs {
+  dsv4_decode_job j[DSV4_DECODE_MAX_JOBS];
+};
+
+template <typename T>
+__global__ void __launch_bounds__(256) decode_state_kernel(const __grid_constant__ DecodeJobs jobs,
+                                                           const int32_t* __restrict__ pos) {
+  const dsv4_decode_job& jb = jobs.j[blockIdx.y];
+  if (jb.kind == DSV4_JOB_RING)
+    ring_write_seq<T>(blockIdx.x, static_cast<const T*>(jb.x_new), static_cast<T*>(jb.out), jb.R, pos,
+                      jb.c);
+  else
+    compress_decode_seq<T, false>(blockIdx.x, static_cast<const T*>(jb.x_new),
+                                  static_cast<const T*>(jb.z_new), jb.bias, static_cast<T*>(jb.tail),
+                                  static_cast<T*>(jb.out), jb.pool_row_off, jb.pool_rows, pos, jb.c,
+                                  jb.m, jb.overlap, nullptr, nullptr, nullptr, 0, nullptr);
 }
 
 }  // namespace dsv4
@@ -150,6 +204,43 @@ extern "C" int dsv4_ring_write(int dtype, const void* kv_new, void* local, int R
   else
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_ring_write: dtype %d not F32/BF16", dtype);
   return launch_status("dsv4_ring_write");
+}
+
+extern "C" int dsv4_decode_state(int dtype, const dsv4_decode_job* jobs, int n_jobs,
+                                 const int32_t* pos, int B, void* stream) {
+  using namespace dsv4;
+  if (B < 0 || n_jobs < 0 || n_jobs > DSV4_DECODE_MAX_JOBS)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: bad sizes B=%d n_jobs=%d (at most %d)", B,
+                n_jobs, DSV4_DECODE_MAX_JOBS);
+  if (B == 0 || n_jobs == 0) return DSV4_OK;
+  if (!jobs || !pos) return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: NULL pointer");
+  if (dtype != DSV4_F32 && dtype != DSV4_BF16)
+    return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: dtype %d not F32/BF16", dtype);
+  DecodeJobs dj;
+  for (int i = 0; i < n_jobs; ++i) {
+    const dsv4_decode_job& j = jobs[i];
+    if (j.kind == DSV4_JOB_RING) {
+      if (j.c < 1 || j.R < 1 || !j.x_new || !j.out)
+        return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: ring job %d: c=%d R=%d or NULL pointer", i,
+                    j.c, j.R);
+    } else if (j.kind == DSV4_JOB_COMPRESS) {
+      if (j.c < 1 || j.m < 1 || (j.overlap != 0 && j.overlap != 1) || j.pool_rows < 0 || !j.x_new ||
+          !j.z_new || !j.bias || !j.tail || !j.out || !j.pool_row_off)
+        return fail(DSV4_ERR_INVALID_ARG,
+                    "dsv4_decode_state: compressor job %d: c=%d m=%d overlap=%d pool_rows=%lld or NULL "
+                    "pointer", i, j.c, j.m, j.overlap, (long long)j.pool_rows);
+    } else {
+      return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: job %d has kind %d", i, j.kind);
+    }
+    dj.j[i] = j;
+  }
+  cudaStream_t st = (cudaStream_t)stream;
+  const dim3 grid((unsigned)B, (unsigned)n_jobs);
+  if (dtype == DSV4_F32)
+    decode_state_kernel<float><<<grid, 256, 0, st>>>(dj, pos);
+  else
+    decode_state_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(dj, pos);
+  return launch_status("dsv4_decode_state");
 }
 
 extern "C" int dsv4_compress_decode_fp8(int dtype, const void* C_new, const void* Z_new,

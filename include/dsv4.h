@@ -128,6 +128,38 @@ int dsv4_ring_write(int dtype, const void* kv_new, void* local, int R, const int
                     int B, int c, void* stream);
 
 /*
+ * dsv4_decode_state -- a token's whole state update ([CSA-DEF] s7 steps 1-4 for every layer)
+ * in one launch: each job is a dsv4_ring_write or a dsv4_compress_decode of one layer for the
+ * same B sequences at positions pos, with the arguments, results, device-side errors and
+ * requirements of those calls (compressor jobs emit into a pool of dtype, not FP8). Jobs run
+ * concurrently, so two jobs must not write the same memory. At most DSV4_DECODE_MAX_JOBS jobs;
+ * the job array is read on the host before the call returns.
+ */
+#define DSV4_DECODE_MAX_JOBS 32
+typedef enum dsv4_job_kind {
+  DSV4_JOB_RING = 0,     /* x_new = kv_new [B, c], out = local ring [B, R, c] */
+  DSV4_JOB_COMPRESS = 1  /* x_new = C_new, z_new = Z_new [B, S*c], bias [S, m, c],
+                            tail [B, S*m, 2, S*c], out = pool [pool_rows, c] */
+} dsv4_job_kind;
+typedef struct dsv4_decode_job {
+  int kind;              /* dsv4_job_kind */
+  int c;                 /* channels of the entry */
+  int m;                 /* compressor: ratio */
+  int overlap;           /* compressor: 1 = CSA (two streams), 0 = HCA */
+  int R;                 /* ring: slots per sequence */
+  int reserved;          /* 0 */
+  const void* x_new;
+  const void* z_new;
+  const float* bias;
+  void* tail;
+  void* out;
+  const int64_t* pool_row_off;
+  int64_t pool_rows;
+} dsv4_decode_job;
+int dsv4_decode_state(int dtype, const dsv4_decode_job* jobs, int n_jobs, const int32_t* pos,
+                      int B, void* stream);
+
+/*
  * dsv4_quantize_fp4 -- FP4 indexer operands ([CSA-DEF] s3.1 and s8: the indexer Q/K are
  * multiplied in 4-bit floating point). Per group of 16 consecutive elements of a row:
  *   scale = RNE_E4M3(amax / 6) (fp32 quotient, saturating at 448);

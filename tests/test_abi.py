@@ -118,3 +118,19 @@ def test_workspace_size_short_rows_and_empty(lib):
     assert f(1, 8192, 16384, 512) == 256 << 20                    # chunks of 4096 rows
     assert f(0, 8, 100, 4) == 0 and f(2, 0, 100, 4) == 0
 
+
+
+def test_decode_job_layout_and_host_validation(lib):
+    """dsv4_decode_job as the binding builds it (80 bytes: six ints, six pointers, one
+    int64), and host validation of dsv4_decode_state before anything is enqueued."""
+    import compressed_sparse_mqa_dsv4_b200 as dsv4
+    J = dsv4._DecodeJob
+    assert ctypes.sizeof(J) == 80 and J.x_new.offset == 24 and J.pool_rows.offset == 72
+    bad = (J * 1)(J(kind=7, c=8))
+    assert lib.dsv4_decode_state(1, bad, 1, ctypes.c_void_p(16), 1, None) == 1
+    assert b"kind 7" in lib.dsv4_last_error_message()
+    too_many = (J * 33)()
+    assert lib.dsv4_decode_state(1, too_many, 33, ctypes.c_void_p(16), 1, None) == 1
+    ring_no_out = (J * 1)(J(kind=0, c=8, R=4, x_new=16))
+    assert lib.dsv4_decode_state(1, ring_no_out, 1, ctypes.c_void_p(16), 1, None) == 1
+    assert lib.dsv4_decode_state(1, bad, 1, ctypes.c_void_p(16), 0, None) == 0   # B == 0: no-op

@@ -116,6 +116,52 @@ def test_ring_write(dsv4, dtype, c):
     assert torch.equal(local, want)
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_decode_state_one_launch_equals_separate_calls(dsv4, dtype):
+    """A token's whole state update in one dsv4_decode_state launch (ring writes and the
+    compressors of a CSA layer -- main and index keys -- and of an HCA layer, over several
+    tokens crossing block boundaries) leaves rings, tails and pools bit-identical to the
+    separate dsv4_ring_write / dsv4_compress_decode calls."""
+    B, c, cI, R = 3, 128, 32, 8
+    n0 = [0, 4 * 33 + 1, 128 * 2 - 3]
+    steps = 9
+    g = Generator(61)
+    layers = [("csa", c, 4, True), ("csa_index", cI, 4, True), ("hca", c, 128, False)]
+    state = {}
+    for name, ch, m, ov in layers:
+        S = 2 if ov else 1
+        E = [(a + steps) // m + 1 for a in n0]
+        off = torch.tensor(np.concatenate([[0], np.cumsum(E)[:-1]]), dtype=torch.int64)
+        state[name] = dict(
+            ch=ch, m=m, ov=ov, S=S, off=off.cuda(),
+            bias=g.normal(f"bias_{name}", (S, m, ch), 0.1).cuda(),
+            tail=g.normal(f"tail_{name}", (B, S * m, 2, S * ch), 1.0, dtype).cuda(),
+            pool=g.normal(f"pool_{name}", (sum(E), ch), 1.0, dtype).cuda())
+    local = g.normal("local", (B, R, c), 1.0, dtype).cuda()
+    ref = {k: {x: v[x].clone() for x in ("tail", "pool")} for k, v in state.items()}
+    ref_local = local.clone()
+    for s in range(steps):
+        pos = torch.tensor([a + s for a in n0], dtype=torch.int32, device="cuda")
+        kv = g.normal(f"kv{s}", (B, c), 1.0, dtype).cuda()
+        news = {name: (g.normal(f"C{s}{name}", (B, st["S"] * st["ch"]), 1.0, dtype).cuda(),
+                       g.normal(f"Z{s}{name}", (B, st["S"] * st["ch"]), 1.0, dtype).cuda())
+                for name, st in state.items()}
+        jobs = [dsv4.decode_ring_job(kv, local)]
+        for name, st in state.items():
+            jobs.append(dsv4.decode_compress_job(*news[name], st["bias"], st["tail"], st["pool"],
+                                                 st["off"], st["m"], st["ov"]))
+        dsv4.dsv4_decode_state(jobs, pos)
+        dsv4.dsv4_ring_write(kv, ref_local, pos)
+        for name, st in state.items():
+            dsv4.dsv4_compress_decode(*news[name], st["bias"], ref[name]["tail"], ref[name]["pool"],
+                                      st["off"], pos, st["m"], st["ov"])
+    dsv4.dsv4_check_errors()
+    assert torch.equal(local, ref_local)
+    for name in state:
+        assert torch.equal(state[name]["tail"], ref[name]["tail"]), name
+        assert torch.equal(state[name]["pool"], ref[name]["pool"]), name
+
+
 def test_csa_decode_step_chain_fp32(dsv4):
     """Whole CSA decode steps of two sequences (prefixes of 37 and 64 tokens, 9 new tokens
     each): ring write, main and index compressor states, index top-k over the grown pools,
