@@ -32,6 +32,10 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "flash_csa_prefill"
 METRIC = "prefill tokens/s per CSA/HCA layer"
+# nominal B200 figures, reported beside the measured denominators: dense bf16 tensor rate and
+# the HGX HBM3e bandwidth
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 7700.0
 UNIT = "tokens/s"
 
 # DRAM traffic of the attention kernel per launch, from one ncu capture
@@ -294,7 +298,10 @@ def run_cuda(args, rank: int, world: int):
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "algorithmic_flops_per_launch": flops,
-                     "peak_source": f"{peak_src} bf16_tflops (burst)"},
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "frac_of_nominal": round(achieved / NOMINAL_BF16_TFLOPS, 4),
+                     "index_topk_tflops": round(index_flops(s.n, s.m, s.H_I, s.c_I) /
+                                                (statistics.mean(index_ms) / 1e3) / 1e12, 1)},
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "clocks": clk.summary(),
@@ -487,6 +494,7 @@ def run_decode(args, dev, stream):
                         f"{'/'.join(D['layers'])} (CSA m=4, HCA m'=128), bf16 pools in HBM",
             "ms_per_step": round(ms, 4), "bytes_per_step": nbytes, "achieved_gbs": round(gbps, 1),
             "peak_gbs": peak, "frac": round(gbps / peak, 4), "peak_source": f"{src} hbm_gbs",
+            "frac_of_nominal": round(gbps / NOMINAL_HBM_GBS, 4),
             "steps": steps, "l2": "flushed (256 MiB write) before every step", "packed_pools": packed,
             "production_pools": production}
 
