@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "DSV4Error", "lib", "LIB_PATH", "F32", "BF16", "FP4",
     "dsv4_compress", "dsv4_compress_decode", "dsv4_ring_write", "decode_tail_shape",
-    "dsv4_decode_state", "decode_ring_job", "decode_compress_job",
+    "dsv4_decode_state", "decode_ring_job", "decode_compress_job", "decode_compress_fp8_job",
+    "decode_compress_fp4_job",
     "dsv4_quantize_fp4", "dsv4_index_topk", "dsv4_index_topk_workspace_size",
     "dsv4_index_topk_workspace_size_ex",
     "dsv4_hybrid_sparse_attn", "dsv4_hybrid_sparse_attn_workspace_size", "dsv4_check_errors",
@@ -56,10 +57,11 @@ lib.dsv4_ring_write.argtypes = [_I, _P, _P, _I, _P, _I, _I, _P]
 class _DecodeJob(ctypes.Structure):
     """dsv4_decode_job of include/dsv4.h."""
     _fields_ = [("kind", ctypes.c_int), ("c", ctypes.c_int), ("m", ctypes.c_int),
-                ("overlap", ctypes.c_int), ("R", ctypes.c_int), ("reserved", ctypes.c_int),
+                ("overlap", ctypes.c_int), ("R", ctypes.c_int), ("rope_dims", ctypes.c_int),
                 ("x_new", ctypes.c_void_p), ("z_new", ctypes.c_void_p), ("bias", ctypes.c_void_p),
-                ("tail", ctypes.c_void_p), ("out", ctypes.c_void_p),
-                ("pool_row_off", ctypes.c_void_p), ("pool_rows", ctypes.c_int64)]
+                ("tail", ctypes.c_void_p), ("out", ctypes.c_void_p), ("out_scales", ctypes.c_void_p),
+                ("out_rope", ctypes.c_void_p), ("pool_row_off", ctypes.c_void_p),
+                ("pool_rows", ctypes.c_int64)]
 
 
 DECODE_MAX_JOBS = 32
@@ -199,7 +201,7 @@ def decode_ring_job(kv_new: torch.Tensor, local: torch.Tensor):
     B, c = kv_new.shape
     if local.shape[0] != B or local.shape[2] != c:
         raise ValueError(f"local must be [{B}, R, {c}]")
-    job = _DecodeJob(kind=0, c=c, m=0, overlap=0, R=local.shape[1], reserved=0,
+    job = _DecodeJob(kind=0, c=c, m=0, overlap=0, R=local.shape[1], rope_dims=0,
                      x_new=kv_new.data_ptr(), z_new=None, bias=None, tail=None, out=local.data_ptr(),
                      pool_row_off=None, pool_rows=0)
     return job, kv_new.dtype, B, (kv_new, local)
@@ -219,10 +221,58 @@ def decode_compress_job(C_new: torch.Tensor, Z_new: torch.Tensor, bias: torch.Te
         raise ValueError(f"tail must be {decode_tail_shape(B, c, m, overlap)}, got {tuple(tail.shape)}")
     if pool.shape[-1] != c:
         raise ValueError(f"pool rows must have {c} channels")
-    job = _DecodeJob(kind=1, c=c, m=m, overlap=1 if overlap else 0, R=0, reserved=0,
+    job = _DecodeJob(kind=1, c=c, m=m, overlap=1 if overlap else 0, R=0, rope_dims=0,
                      x_new=C_new.data_ptr(), z_new=Z_new.data_ptr(), bias=bias.data_ptr(), tail=tail.data_ptr(),
                      out=pool.data_ptr(), pool_row_off=pool_row_off.data_ptr(), pool_rows=pool.numel() // c)
     return job, C_new.dtype, B, (C_new, Z_new, bias, tail, pool, pool_row_off)
+
+
+def _compress_common(C_new, Z_new, bias, tail, pool_row_off, m, overlap):
+    _dev(C_new, "C_new"), _dev(Z_new, "Z_new", C_new.dtype), _dev(bias, "bias", torch.float32)
+    B, width = C_new.shape
+    c = width // (2 if overlap else 1)
+    _dev(tail, "tail", C_new.dtype), _dev(pool_row_off, "pool_row_off", torch.int64)
+    if tuple(tail.shape) != decode_tail_shape(B, c, m, overlap):
+        raise ValueError(f"tail must be {decode_tail_shape(B, c, m, overlap)}, got {tuple(tail.shape)}")
+    return B, c
+
+
+def decode_compress_fp8_job(C_new: torch.Tensor, Z_new: torch.Tensor, bias: torch.Tensor,
+                            tail: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                            rope: Optional[torch.Tensor], pool_row_off: torch.Tensor, m: int,
+                            overlap: bool, rope_dims: int = 64):
+    """A dsv4_decode_state job: the compressor token of dsv4_compress_decode_fp8 (the entry into
+    the FP8 main-KV pool: codes uint8 [rows, c - rope_dims], scales fp32 [rows, (c-rope)/64],
+    rope bf16 [rows, rope_dims])."""
+    B, c = _compress_common(C_new, Z_new, bias, tail, pool_row_off, m, overlap)
+    _dev(codes, "codes", torch.uint8), _dev(scales, "scales", torch.float32)
+    if rope_dims:
+        _dev(rope, "rope", torch.bfloat16)
+    if codes.shape[-1] != c - rope_dims:
+        raise ValueError(f"codes rows must have {c - rope_dims} bytes")
+    job = _DecodeJob(kind=2, c=c, m=m, overlap=1 if overlap else 0, R=0, rope_dims=rope_dims,
+                     x_new=C_new.data_ptr(), z_new=Z_new.data_ptr(), bias=bias.data_ptr(),
+                     tail=tail.data_ptr(), out=codes.data_ptr(), out_scales=scales.data_ptr(),
+                     out_rope=rope.data_ptr() if rope_dims else None,
+                     pool_row_off=pool_row_off.data_ptr(), pool_rows=codes.shape[0])
+    return job, C_new.dtype, B, (C_new, Z_new, bias, tail, codes, scales, rope, pool_row_off)
+
+
+def decode_compress_fp4_job(C_new: torch.Tensor, Z_new: torch.Tensor, bias: torch.Tensor,
+                            tail: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+                            pool_row_off: torch.Tensor, m: int, overlap: bool):
+    """A dsv4_decode_state job: the compressor token with the entry emitted into an FP4 pool
+    (the index keys: codes uint8 [rows, c/2], E4M3 scales uint8 [rows, c/16]), rounded to the
+    input dtype and quantised as dsv4_quantize_fp4 quantises that row."""
+    B, c = _compress_common(C_new, Z_new, bias, tail, pool_row_off, m, overlap)
+    _dev(codes, "codes", torch.uint8), _dev(scales, "scales", torch.uint8)
+    if codes.shape[-1] != c // 2 or scales.shape[-1] != c // 16:
+        raise ValueError(f"FP4 pool rows must be {c // 2} code bytes and {c // 16} scales")
+    job = _DecodeJob(kind=3, c=c, m=m, overlap=1 if overlap else 0, R=0, rope_dims=0,
+                     x_new=C_new.data_ptr(), z_new=Z_new.data_ptr(), bias=bias.data_ptr(),
+                     tail=tail.data_ptr(), out=codes.data_ptr(), out_scales=scales.data_ptr(),
+                     out_rope=None, pool_row_off=pool_row_off.data_ptr(), pool_rows=codes.shape[0])
+    return job, C_new.dtype, B, (C_new, Z_new, bias, tail, codes, scales, pool_row_off)
 
 
 def dsv4_decode_state(jobs, pos: torch.Tensor, stream=None) -> None:

@@ -11,22 +11,30 @@
 // the prefill compressor: an online softmax in fp32 over the preceding block's stream-b
 // positions, then the current block's stream-a positions, in position order.
 #include "dsv4_common.cuh"
+#include "fp4_quant.cuh"
 #include "fp8_kv.cuh"
 
 namespace dsv4 {
 
-// The emitted entry goes to `pool` (dtype T), or -- FP8 -- through shared memory into the
-// production main-KV format (fp8_kv.cuh): the entry rounded to T, then quantised, so an FP8
-// pool holds exactly the quantisation of the T pool's row.
+// Where the emitted entry goes: a pool of dtype T, or -- through shared memory -- the
+// production formats: the main-KV FP8 entry (fp8_kv.cuh) or the FP4 index key (fp4_quant.cuh).
+// Either way the entry is rounded to T first and then quantised, so a packed pool holds
+// exactly the quantisation of the T pool's row.
+enum EmitMode { kEmitPool = 0, kEmitFp8 = 1, kEmitFp4 = 2 };
+
 // Sequence b's token (one CTA of 256 threads): its (C, Z) rows into the tail and, when t + 1
-// completes a block, the entry into the pool. FP8: `entry` is shared memory of c floats.
-template <typename T, bool FP8>
+// completes a block, the entry into the pool. FP8 / FP4: `entry` is shared memory of c floats;
+// FP8: codes [rows, c - rope], scales fp32 [rows, (c - rope)/64], rope_out bf16 [rows, rope];
+// FP4: codes [rows, c/2], scales E4M3 bytes [rows, c/16].
+template <typename T, int MODE>
 __device__ __forceinline__ void compress_decode_seq(
     int b, const T* __restrict__ C_new, const T* __restrict__ Z_new, const float* __restrict__ bias,
     T* __restrict__ tail, T* __restrict__ pool, const int64_t* __restrict__ pool_row_off,
     long long pool_rows, const int32_t* __restrict__ pos, int c, int m, int overlap,
-    uint8_t* __restrict__ codes, float* __restrict__ scales, __nv_bfloat16* __restrict__ rope_out,
+    uint8_t* __restrict__ codes, void* __restrict__ scales_v, __nv_bfloat16* __restrict__ rope_out,
     int rope, float* entry) {
+  constexpr bool FP8 = MODE == kEmitFp8;
+  constexpr bool PACKED = MODE != kEmitPool;
   const int S = overlap ? 2 : 1;
   const int T_slots = S * m;
   const long long width = (long long)S * c;
@@ -86,12 +94,26 @@ __device__ __forceinline__ void compress_decode_seq(
         }
       }
     }
-    if constexpr (FP8)
+    if constexpr (PACKED)
       entry[ch] = to_f32(from_f32<T>(acc / den));
     else
       pool[row * c + ch] = from_f32<T>(acc / den);
   }
+  if constexpr (MODE == kEmitFp4) {
+    __syncthreads();
+    uint8_t* sc4 = static_cast<uint8_t*>(scales_v);
+    for (int g = threadIdx.x; g < c / 16; g += blockDim.x) {
+      float v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = entry[16 * g + j];
+      uint32_t w0, w1, sb;
+      fp4_quantize_group(v, w0, w1, sb);
+      *reinterpret_cast<uint2*>(codes + row * (c / 2) + 8 * g) = make_uint2(w0, w1);
+      sc4[row * (c / 16) + g] = (uint8_t)sb;
+    }
+  }
   if constexpr (FP8) {
+    float* scales = static_cast<float*>(scales_v);
     __syncthreads();
     const int lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int nf = c - rope, ng = nf / kFp8Group;
@@ -107,16 +129,16 @@ __device__ __forceinline__ void compress_decode_seq(
   }
 }
 
-template <typename T, bool FP8>
+template <typename T, int MODE>
 __global__ void __launch_bounds__(256) compress_decode_kernel(
     const T* __restrict__ C_new, const T* __restrict__ Z_new, const float* __restrict__ bias,
     T* __restrict__ tail, T* __restrict__ pool, const int64_t* __restrict__ pool_row_off,
     long long pool_rows, const int32_t* __restrict__ pos, int c, int m, int overlap,
     uint8_t* __restrict__ codes, float* __restrict__ scales, __nv_bfloat16* __restrict__ rope_out,
     int rope) {
-  extern __shared__ float entry[];                          // FP8: the entry, c values
-  compress_decode_seq<T, FP8>(blockIdx.x, C_new, Z_new, bias, tail, pool, pool_row_off, pool_rows,
-                              pos, c, m, overlap, codes, scales, rope_out, rope, entry);
+  extern __shared__ float entry[];                          // packed: the entry, c values
+  compress_decode_seq<T, MODE>(blockIdx.x, C_new, Z_new, bias, tail, pool, pool_row_off, pool_rows,
+                               pos, c, m, overlap, codes, scales, rope_out, rope, entry);
 }
 
 template <typename T>
@@ -147,15 +169,26 @@ struct DecodeJobs {
 template <typename T>
 __global__ void __launch_bounds__(256) decode_state_kernel(const __grid_constant__ DecodeJobs jobs,
                                                            const int32_t* __restrict__ pos) {
+  extern __shared__ float entry[];                          // packed emissions: c values
   const dsv4_decode_job& jb = jobs.j[blockIdx.y];
+  const T* x = static_cast<const T*>(jb.x_new);
+  const T* z = static_cast<const T*>(jb.z_new);
+  T* tail = static_cast<T*>(jb.tail);
   if (jb.kind == DSV4_JOB_RING)
-    ring_write_seq<T>(blockIdx.x, static_cast<const T*>(jb.x_new), static_cast<T*>(jb.out), jb.R, pos,
-                      jb.c);
+    ring_write_seq<T>(blockIdx.x, x, static_cast<T*>(jb.out), jb.R, pos, jb.c);
+  else if (jb.kind == DSV4_JOB_COMPRESS)
+    compress_decode_seq<T, kEmitPool>(blockIdx.x, x, z, jb.bias, tail, static_cast<T*>(jb.out),
+                                      jb.pool_row_off, jb.pool_rows, pos, jb.c, jb.m, jb.overlap,
+                                      nullptr, nullptr, nullptr, 0, entry);
+  else if (jb.kind == DSV4_JOB_COMPRESS_FP8)
+    compress_decode_seq<T, kEmitFp8>(blockIdx.x, x, z, jb.bias, tail, nullptr, jb.pool_row_off,
+                                     jb.pool_rows, pos, jb.c, jb.m, jb.overlap,
+                                     static_cast<uint8_t*>(jb.out), jb.out_scales,
+                                     static_cast<__nv_bfloat16*>(jb.out_rope), jb.rope_dims, entry);
   else
-    compress_decode_seq<T, false>(blockIdx.x, static_cast<const T*>(jb.x_new),
-                                  static_cast<const T*>(jb.z_new), jb.bias, static_cast<T*>(jb.tail),
-                                  static_cast<T*>(jb.out), jb.pool_row_off, jb.pool_rows, pos, jb.c,
-                                  jb.m, jb.overlap, nullptr, nullptr, nullptr, 0, nullptr);
+    compress_decode_seq<T, kEmitFp4>(blockIdx.x, x, z, jb.bias, tail, nullptr, jb.pool_row_off,
+                                     jb.pool_rows, pos, jb.c, jb.m, jb.overlap,
+                                     static_cast<uint8_t*>(jb.out), jb.out_scales, nullptr, 0, entry);
 }
 
 }  // namespace dsv4
@@ -175,11 +208,11 @@ extern "C" int dsv4_compress_decode(int dtype, const void* C_new, const void* Z_
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_compress_decode: NULL pointer");
   cudaStream_t st = (cudaStream_t)stream;
   if (dtype == DSV4_F32)
-    compress_decode_kernel<float, false><<<B, 256, 0, st>>>(
+    compress_decode_kernel<float, kEmitPool><<<B, 256, 0, st>>>(
         (const float*)C_new, (const float*)Z_new, bias, (float*)tail, (float*)pool, pool_row_off,
         pool_rows, pos, c, m, overlap, nullptr, nullptr, nullptr, 0);
   else if (dtype == DSV4_BF16)
-    compress_decode_kernel<__nv_bfloat16, false><<<B, 256, 0, st>>>(
+    compress_decode_kernel<__nv_bfloat16, kEmitPool><<<B, 256, 0, st>>>(
         (const __nv_bfloat16*)C_new, (const __nv_bfloat16*)Z_new, bias, (__nv_bfloat16*)tail,
         (__nv_bfloat16*)pool, pool_row_off, pool_rows, pos, c, m, overlap, nullptr, nullptr,
         nullptr, 0);
@@ -217,29 +250,43 @@ extern "C" int dsv4_decode_state(int dtype, const dsv4_decode_job* jobs, int n_j
   if (dtype != DSV4_F32 && dtype != DSV4_BF16)
     return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: dtype %d not F32/BF16", dtype);
   DecodeJobs dj;
+  int smem_c = 0;                                  // widest packed emission (floats)
   for (int i = 0; i < n_jobs; ++i) {
     const dsv4_decode_job& j = jobs[i];
     if (j.kind == DSV4_JOB_RING) {
       if (j.c < 1 || j.R < 1 || !j.x_new || !j.out)
         return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: ring job %d: c=%d R=%d or NULL pointer", i,
                     j.c, j.R);
-    } else if (j.kind == DSV4_JOB_COMPRESS) {
+    } else if (j.kind == DSV4_JOB_COMPRESS || j.kind == DSV4_JOB_COMPRESS_FP8 ||
+               j.kind == DSV4_JOB_COMPRESS_FP4) {
       if (j.c < 1 || j.m < 1 || (j.overlap != 0 && j.overlap != 1) || j.pool_rows < 0 || !j.x_new ||
           !j.z_new || !j.bias || !j.tail || !j.out || !j.pool_row_off)
         return fail(DSV4_ERR_INVALID_ARG,
                     "dsv4_decode_state: compressor job %d: c=%d m=%d overlap=%d pool_rows=%lld or NULL "
                     "pointer", i, j.c, j.m, j.overlap, (long long)j.pool_rows);
+      if (j.kind == DSV4_JOB_COMPRESS_FP8 &&
+          (j.rope_dims < 0 || j.rope_dims > j.c || (j.rope_dims & 1) || (j.c - j.rope_dims) % kFp8Group != 0 ||
+           j.c > 12 * 1024 || !j.out_scales || (j.rope_dims > 0 && !j.out_rope) ||
+           (reinterpret_cast<uintptr_t>(j.out) & 1u)))
+        return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: FP8 job %d: c=%d rope_dims=%d, scales/rope or "
+                    "2-byte aligned codes", i, j.c, j.rope_dims);
+      if (j.kind == DSV4_JOB_COMPRESS_FP4 &&
+          (j.c % 16 != 0 || j.c > 12 * 1024 || !j.out_scales || (reinterpret_cast<uintptr_t>(j.out) & 7u)))
+        return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: FP4 job %d: c=%d (c %% 16 == 0), scales or "
+                    "8-byte aligned codes", i, j.c);
+      if (j.kind != DSV4_JOB_COMPRESS && j.c > smem_c) smem_c = j.c;
     } else {
       return fail(DSV4_ERR_INVALID_ARG, "dsv4_decode_state: job %d has kind %d", i, j.kind);
     }
     dj.j[i] = j;
   }
+  const size_t smem = sizeof(float) * (size_t)smem_c;
   cudaStream_t st = (cudaStream_t)stream;
   const dim3 grid((unsigned)B, (unsigned)n_jobs);
   if (dtype == DSV4_F32)
-    decode_state_kernel<float><<<grid, 256, 0, st>>>(dj, pos);
+    decode_state_kernel<float><<<grid, 256, smem, st>>>(dj, pos);
   else
-    decode_state_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(dj, pos);
+    decode_state_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(dj, pos);
   return launch_status("dsv4_decode_state");
 }
 
@@ -264,11 +311,11 @@ extern "C" int dsv4_compress_decode_fp8(int dtype, const void* C_new, const void
   cudaStream_t st = (cudaStream_t)stream;
   const size_t smem = sizeof(float) * (size_t)c;
   if (dtype == DSV4_F32)
-    compress_decode_kernel<float, true><<<B, 256, smem, st>>>(
+    compress_decode_kernel<float, kEmitFp8><<<B, 256, smem, st>>>(
         (const float*)C_new, (const float*)Z_new, bias, (float*)tail, nullptr, pool_row_off,
         pool_rows, pos, c, m, overlap, codes, scales, (__nv_bfloat16*)rope_out, rope);
   else if (dtype == DSV4_BF16)
-    compress_decode_kernel<__nv_bfloat16, true><<<B, 256, smem, st>>>(
+    compress_decode_kernel<__nv_bfloat16, kEmitFp8><<<B, 256, smem, st>>>(
         (const __nv_bfloat16*)C_new, (const __nv_bfloat16*)Z_new, bias, (__nv_bfloat16*)tail,
         nullptr, pool_row_off, pool_rows, pos, c, m, overlap, codes, scales,
         (__nv_bfloat16*)rope_out, rope);

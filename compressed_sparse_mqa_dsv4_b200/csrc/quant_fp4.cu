@@ -9,29 +9,9 @@
 // scale byte. Rounding uses the sm_100a conversion instructions (round-to-nearest-even
 // with saturation) on fp32 quotients computed with IEEE division.
 #include "dsv4_common.cuh"
+#include "fp4_quant.cuh"
 
 namespace dsv4 {
-
-// e4m3 byte -> float (exact): exponent field 0 is subnormal (m * 2^-9).
-__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
-  const uint32_t e = (b >> 3) & 15u, mt = b & 7u;
-  float v = e == 0 ? (float)mt * 0x1p-9f : (float)(8u + mt) * exp2f((float)e - 10.f);
-  return (b & 0x80u) ? -v : v;
-}
-
-__device__ __forceinline__ uint32_t f32_to_e4m3_rn_sat(float x) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
-  return r & 0xFFu;  // second source operand lands in the low byte
-}
-
-// two fp32 -> one byte of e2m1 codes: `lo` in bits 0..3, `hi` in bits 4..7
-__device__ __forceinline__ uint32_t f32x2_to_e2m1_rn_sat(float lo, float hi) {
-  uint32_t r;
-  asm("{\n .reg .b8 t;\n cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n cvt.u32.u8 %0, t;\n}"
-      : "=r"(r) : "f"(hi), "f"(lo));
-  return r & 0xFFu;
-}
 
 __global__ void __launch_bounds__(256) quantize_fp4_kernel(
     const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ codes,
@@ -44,19 +24,8 @@ __global__ void __launch_bounds__(256) quantize_fp4_kernel(
     load16_f32(x + g * 16 + 8, b);
 #pragma unroll
     for (int j = 0; j < 8; ++j) { v[j] = a[j]; v[8 + j] = b[j]; }
-    float amax = 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    const uint32_t sb = f32_to_e4m3_rn_sat(__fdiv_rn(amax, 6.0f));
-    const float s = e4m3_to_float(sb);
-    uint32_t w0 = 0, w1 = 0;
-    if (s > 0.f) {
-#pragma unroll
-      for (int j = 0; j < 8; j += 2) {
-        w0 |= f32x2_to_e2m1_rn_sat(__fdiv_rn(v[j], s), __fdiv_rn(v[j + 1], s)) << (4 * j);
-        w1 |= f32x2_to_e2m1_rn_sat(__fdiv_rn(v[8 + j], s), __fdiv_rn(v[9 + j], s)) << (4 * j);
-      }
-    }
+    uint32_t w0, w1, sb;
+    fp4_quantize_group(v, w0, w1, sb);
     *reinterpret_cast<uint2*>(codes + g * 8) = make_uint2(w0, w1);
     scales[g] = (uint8_t)sb;
   }

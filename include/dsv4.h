@@ -129,17 +129,25 @@ int dsv4_ring_write(int dtype, const void* kv_new, void* local, int R, const int
 
 /*
  * dsv4_decode_state -- a token's whole state update ([CSA-DEF] s7 steps 1-4 for every layer)
- * in one launch: each job is a dsv4_ring_write or a dsv4_compress_decode of one layer for the
- * same B sequences at positions pos, with the arguments, results, device-side errors and
- * requirements of those calls (compressor jobs emit into a pool of dtype, not FP8). Jobs run
- * concurrently, so two jobs must not write the same memory. At most DSV4_DECODE_MAX_JOBS jobs;
- * the job array is read on the host before the call returns.
+ * in one launch: each job is a dsv4_ring_write or a compressor token of one layer for the same
+ * B sequences at positions pos, with the arguments, results, device-side errors and
+ * requirements of those calls: DSV4_JOB_COMPRESS as dsv4_compress_decode (entry into a pool of
+ * dtype), DSV4_JOB_COMPRESS_FP8 as dsv4_compress_decode_fp8 (the main-KV FP8 entry),
+ * DSV4_JOB_COMPRESS_FP4 emits the entry rounded to dtype and quantised exactly as
+ * dsv4_quantize_fp4 quantises that row (the FP4 index-key pool; c % 16 == 0, codes 8-byte
+ * aligned). Jobs run concurrently, so two jobs must not write the same memory. At most
+ * DSV4_DECODE_MAX_JOBS jobs; the job array is read on the host before the call returns.
  */
 #define DSV4_DECODE_MAX_JOBS 32
 typedef enum dsv4_job_kind {
-  DSV4_JOB_RING = 0,     /* x_new = kv_new [B, c], out = local ring [B, R, c] */
-  DSV4_JOB_COMPRESS = 1  /* x_new = C_new, z_new = Z_new [B, S*c], bias [S, m, c],
-                            tail [B, S*m, 2, S*c], out = pool [pool_rows, c] */
+  DSV4_JOB_RING = 0,          /* x_new = kv_new [B, c], out = local ring [B, R, c] */
+  DSV4_JOB_COMPRESS = 1,      /* x_new = C_new, z_new = Z_new [B, S*c], bias [S, m, c],
+                                 tail [B, S*m, 2, S*c], out = pool [pool_rows, c] */
+  DSV4_JOB_COMPRESS_FP8 = 2,  /* as 1; out = FP8 codes [pool_rows, c - rope_dims], out_scales =
+                                 fp32 [pool_rows, (c - rope_dims)/64], out_rope = bf16
+                                 [pool_rows, rope_dims] */
+  DSV4_JOB_COMPRESS_FP4 = 3   /* as 1; out = e2m1 codes [pool_rows, c/2], out_scales = E4M3
+                                 bytes [pool_rows, c/16] */
 } dsv4_job_kind;
 typedef struct dsv4_decode_job {
   int kind;              /* dsv4_job_kind */
@@ -147,12 +155,14 @@ typedef struct dsv4_decode_job {
   int m;                 /* compressor: ratio */
   int overlap;           /* compressor: 1 = CSA (two streams), 0 = HCA */
   int R;                 /* ring: slots per sequence */
-  int reserved;          /* 0 */
+  int rope_dims;         /* FP8: bf16 RoPE channels at the end of the entry */
   const void* x_new;
   const void* z_new;
   const float* bias;
   void* tail;
   void* out;
+  void* out_scales;
+  void* out_rope;
   const int64_t* pool_row_off;
   int64_t pool_rows;
 } dsv4_decode_job;

@@ -121,11 +121,11 @@ def test_workspace_size_short_rows_and_empty(lib):
 
 
 def test_decode_job_layout_and_host_validation(lib):
-    """dsv4_decode_job as the binding builds it (80 bytes: six ints, six pointers, one
+    """dsv4_decode_job as the binding builds it (96 bytes: six ints, eight pointers, one
     int64), and host validation of dsv4_decode_state before anything is enqueued."""
     import compressed_sparse_mqa_dsv4_b200 as dsv4
     J = dsv4._DecodeJob
-    assert ctypes.sizeof(J) == 80 and J.x_new.offset == 24 and J.pool_rows.offset == 72
+    assert ctypes.sizeof(J) == 96 and J.x_new.offset == 24 and J.pool_rows.offset == 88
     bad = (J * 1)(J(kind=7, c=8))
     assert lib.dsv4_decode_state(1, bad, 1, ctypes.c_void_p(16), 1, None) == 1
     assert b"kind 7" in lib.dsv4_last_error_message()
@@ -134,3 +134,9 @@ def test_decode_job_layout_and_host_validation(lib):
     ring_no_out = (J * 1)(J(kind=0, c=8, R=4, x_new=16))
     assert lib.dsv4_decode_state(1, ring_no_out, 1, ctypes.c_void_p(16), 1, None) == 1
     assert lib.dsv4_decode_state(1, bad, 1, ctypes.c_void_p(16), 0, None) == 0   # B == 0: no-op
+    fp4_odd = (J * 1)(J(kind=3, c=24, m=4, overlap=1, x_new=16, z_new=16, bias=16, tail=16, out=16,
+                        out_scales=16, pool_row_off=16, pool_rows=8))
+    assert lib.dsv4_decode_state(1, fp4_odd, 1, ctypes.c_void_p(16), 1, None) == 1     # c % 16
+    fp8_rope = (J * 1)(J(kind=2, c=512, m=4, overlap=1, rope_dims=63, x_new=16, z_new=16, bias=16,
+                         tail=16, out=16, out_scales=16, out_rope=16, pool_row_off=16, pool_rows=8))
+    assert lib.dsv4_decode_state(1, fp8_rope, 1, ctypes.c_void_p(16), 1, None) == 1    # odd rope

@@ -247,3 +247,53 @@ def test_csa_decode_step_chain_fp32(dsv4):
             assert_close(Lg[b, 0], l_ref, "f32", f"LSE b={b} t={t}")
             compared += 1
     assert compared >= 2 * steps - 2
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_decode_state_packed_emission(dsv4, dtype):
+    """The fused state update emitting straight into the production pools: the CSA main-KV
+    compressor into an FP8 pool (codes, scales, bf16 RoPE tail) and the index-key compressor
+    into an FP4 pool (e2m1 codes, E4M3 scales), beside an HCA compressor into a plain pool.
+    Over tokens crossing block boundaries, the FP8 pool is bit-identical to the one
+    dsv4_compress_decode_fp8 writes, and the FP4 pool holds exactly the oracle's FP4
+    quantisation of the entries dsv4_compress_decode emits (rounded to dtype first); rows not
+    completed stay untouched."""
+    B, c, cI, rd = 3, 576, 128, 64
+    n0 = [0, 4 * 21 + 2, 128 - 3]
+    steps = 11
+    g = Generator(67)
+    E = [(a + steps) // 4 + 1 for a in n0]
+    off = torch.tensor(np.concatenate([[0], np.cumsum(E)[:-1]]), dtype=torch.int64).cuda()
+    rows = sum(E)
+    b_main, b_idx = g.normal("b_main", (2, 4, c), 0.1).cuda(), g.normal("b_idx", (2, 4, cI), 0.1).cuda()
+    t_main = g.normal("t_main", (B, 8, 2, 2 * c), 1.0, dtype).cuda()
+    t_idx = g.normal("t_idx", (B, 8, 2, 2 * cI), 1.0, dtype).cuda()
+    codes8 = torch.full((rows, c - rd), 0x5A, dtype=torch.uint8, device="cuda")
+    scales8 = torch.full((rows, (c - rd) // 64), -1.0, device="cuda")
+    rope8 = torch.full((rows, rd), -7.0, dtype=torch.bfloat16, device="cuda")
+    codes4 = torch.full((rows, cI // 2), 0xA5, dtype=torch.uint8, device="cuda")
+    scales4 = torch.full((rows, cI // 16), 0x3C, dtype=torch.uint8, device="cuda")
+    ref8 = (codes8.clone(), scales8.clone(), rope8.clone())
+    ref_tmain, ref_tidx = t_main.clone(), t_idx.clone()
+    plain_idx = torch.full((rows, cI), 1024.0, dtype=dtype, device="cuda")  # sentinel rows
+    for s in range(steps):
+        pos = torch.tensor([a + s for a in n0], dtype=torch.int32, device="cuda")
+        Cm, Zm = (g.normal(f"{n}m{s}", (B, 2 * c), 1.0, dtype).cuda() for n in "CZ")
+        Ci, Zi = (g.normal(f"{n}i{s}", (B, 2 * cI), 1.0, dtype).cuda() for n in "CZ")
+        jobs = [dsv4.decode_compress_fp8_job(Cm, Zm, b_main, t_main, codes8, scales8, rope8, off, 4,
+                                             True, rd),
+                dsv4.decode_compress_fp4_job(Ci, Zi, b_idx, t_idx, codes4, scales4, off, 4, True)]
+        dsv4.dsv4_decode_state(jobs, pos)
+        dsv4.dsv4_compress_decode_fp8(Cm, Zm, b_main, ref_tmain, *ref8, off, pos, 4, True)
+        dsv4.dsv4_compress_decode(Ci, Zi, b_idx, ref_tidx, plain_idx, off, pos, 4, True)
+    dsv4.dsv4_check_errors()
+    assert torch.equal(t_main, ref_tmain) and torch.equal(t_idx, ref_tidx)
+    for got, want, name in zip((codes8, scales8, rope8), ref8, ("codes", "scales", "rope")):
+        assert torch.equal(got, want), f"FP8 {name}"
+    written = (plain_idx != 1024.0).any(dim=1).cpu().numpy()
+    assert written.sum() == sum((a + steps) // 4 - a // 4 for a in n0)
+    rc, rs = O.quantize_fp4(plain_idx.float().cpu()[written])
+    gc, gs = codes4.cpu().numpy(), scales4.cpu().numpy()
+    np.testing.assert_array_equal(gs[written], rs)
+    np.testing.assert_array_equal(gc[written], rc)
+    assert (gc[~written] == 0xA5).all() and (gs[~written] == 0x3C).all()
