@@ -567,6 +567,29 @@ def run_decode_state(args, dev, stream):
     def step_one_launch():
         dsv4.dsv4_decode_state(jobs, pos)
 
+    # the same launch emitting into the production pool formats: CSA main entries quantised to
+    # the FP8 entry format (448 FP8 channels + 7 scales + 64 bf16 RoPE channels), CSA index
+    # keys to FP4 (e2m1 + one E4M3 scale per 16); HCA entries stay bf16
+    rd = 64
+    jobs_q = []
+    for kind in D["layers"]:
+        jobs_q.append(dsv4.decode_ring_job(kv, torch.empty_like(local)))
+        if kind == "csa":
+            rows = int(sum(E4))
+            jobs_q.append(dsv4.decode_compress_fp8_job(
+                C4, Z4, b4, tail4.clone(), torch.empty(rows, c - rd, dtype=torch.uint8, device=dev),
+                torch.empty(rows, (c - rd) // 64, device=dev),
+                torch.empty(rows, rd, dtype=torch.bfloat16, device=dev), off4, m4, True, rd))
+            jobs_q.append(dsv4.decode_compress_fp4_job(
+                CI, ZI, bI, tailI.clone(), torch.empty(rows, cI // 2, dtype=torch.uint8, device=dev),
+                torch.empty(rows, cI // 16, dtype=torch.uint8, device=dev), off4, m4, True))
+        else:
+            jobs_q.append(dsv4.decode_compress_job(C128, Z128, b128, tail128.clone(),
+                                                   torch.empty_like(pool128), off128, m128, False))
+
+    def step_production():
+        dsv4.dsv4_decode_state(jobs_q, pos)
+
     def timed(step):
         for _ in range(3):
             step()
@@ -585,12 +608,16 @@ def run_decode_state(args, dev, stream):
 
     ms_one, n_one = timed(step_one_launch)
     ms_sep, _ = timed(step_separate)
+    ms_q, _ = timed(step_production)
     launches = sum(3 if kind == "csa" else 2 for kind in D["layers"])
     return {"what": "ring writes + compressor states of the 4 layers for one token of each of "
                     f"the {B} sequences (entries completing at this token appended), all "
                     f"{len(jobs)} jobs in one dsv4_decode_state launch",
             "ms_per_step": round(ms_one, 4), "launches_per_step": 1,
             "separate_calls": {"ms_per_step": round(ms_sep, 4), "launches_per_step": launches},
+            "production_pools": {"what": "the same single launch emitting CSA main entries as FP8 "
+                                         "entries and CSA index keys as FP4",
+                                 "ms_per_step": round(ms_q, 4), "launches_per_step": 1},
             "emitting_sequences": {"csa": int((L % m4 == 0).sum()), "hca": int((L % m128 == 0).sum())},
             "steps": n_one, "l2": "flushed (256 MiB write) before every step"}
 

@@ -153,6 +153,13 @@ __device__ __forceinline__ float xpose_reduce32(float (&v)[32]) {
   return v[0];
 }
 
+// 2^x by the PTX approximate base-2 exponential, results below 2^-126 flushed to zero (the
+// weights are rounded to bf16 next; one that small is zero beside the block's largest)
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
@@ -220,8 +227,7 @@ __device__ __forceinline__ ItemInfo item_info(const AttnArgs& a, int item, int h
 
 template <bool kSplit>
 __global__ void __maxnreg__(128)
-    attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q,
-                   const __grid_constant__ CUtensorMap map_o, int head_groups,
+    attn_tc_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap map_q, int head_groups,
                    int items, float scale_log2, uint32_t spin) {
   extern __shared__ uint8_t smem_raw[];
   AttnSmem& s = *reinterpret_cast<AttnSmem*>(
@@ -502,8 +508,6 @@ __global__ void __maxnreg__(128)
         float z[32];
         tc::tmem_ld32(tmem + lane_base + TM_S + hb, z);
         tc::tmem_wait_ld_dep(z);
-#pragma unroll
-        for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
         // GEMM1 of this block completing implies GEMM2 of the previous block completed (it
         // waited for the chunks that GEMM2 released), so P and O^T are free to touch.
         uint8_t* prow = s.p + slot * 128;
@@ -514,20 +518,28 @@ __global__ void __maxnreg__(128)
         // running max by more than TAU -- then the exact path below recomputes this block.
         bool exact = j == it.jb;
         if (!exact) {
+          // one FMA per weight: x = z * scale - m (log2 units); an invalid slot takes scale 0
+          // (its x is -m, finite or +inf) and its weights are zeroed after the exponential
           uint32_t pk[16];
           bool over = false;
+          const float sc = valid ? scale_log2 : 0.f;
 #pragma unroll
           for (int h = 0; h < 32; h += 4) {
             const float4 m4 = *reinterpret_cast<const float4*>(&s.mcur[hb + h]);
-            over |= !(z[h] <= m4.x + TAU) | !(z[h + 1] <= m4.y + TAU) |
-                    !(z[h + 2] <= m4.z + TAU) | !(z[h + 3] <= m4.w + TAU);
-            __nv_bfloat162 b0 = __floats2bfloat162_rn(exp2f(z[h] - m4.x), exp2f(z[h + 1] - m4.y));
-            __nv_bfloat162 b1 = __floats2bfloat162_rn(exp2f(z[h + 2] - m4.z), exp2f(z[h + 3] - m4.w));
+            const float x0 = fmaf(z[h], sc, -m4.x), x1 = fmaf(z[h + 1], sc, -m4.y);
+            const float x2 = fmaf(z[h + 2], sc, -m4.z), x3 = fmaf(z[h + 3], sc, -m4.w);
+            over |= !(x0 <= TAU) | !(x1 <= TAU) | !(x2 <= TAU) | !(x3 <= TAU);
+            __nv_bfloat162 b0 = __floats2bfloat162_rn(ex2_ftz(x0), ex2_ftz(x1));
+            __nv_bfloat162 b1 = __floats2bfloat162_rn(ex2_ftz(x2), ex2_ftz(x3));
             pk[h / 2] = *reinterpret_cast<uint32_t*>(&b0);
             pk[h / 2 + 1] = *reinterpret_cast<uint32_t*>(&b1);
           }
-          exact = bar_red_or(2, AT_SOFT, over);
+          exact = bar_red_or(2, AT_SOFT, over && valid);
           if (!exact) {
+            if (!valid) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = 0u;
+            }
 #pragma unroll
             for (int h = 0; h < 32; h += 2) {
               // the denominator sums the same bf16-rounded weights the PV product uses
@@ -542,6 +554,8 @@ __global__ void __maxnreg__(128)
           }
         }
         if (exact) {
+#pragma unroll
+          for (int h = 0; h < 32; ++h) z[h] = valid ? z[h] * scale_log2 : -INFINITY;
           // the butterfly consumes z; the scores are read from TMEM again (S^T is not
           // overwritten before this block's P is published) while the block max is combined
           s.red[quad][hb + lane] = xpose_reduce32<true>(z);
@@ -578,8 +592,8 @@ __global__ void __maxnreg__(128)
               const int h = 8 * c + 4 * v;
               const float4 mo = *reinterpret_cast<const float4*>(&s.moff[hb + h]);
               const float4 fa = *reinterpret_cast<const float4*>(&s.fac[hb + h]);
-              __nv_bfloat162 b0 = __floats2bfloat162_rn(exp2f(z[h] - mo.x), exp2f(z[h + 1] - mo.y));
-              __nv_bfloat162 b1 = __floats2bfloat162_rn(exp2f(z[h + 2] - mo.z), exp2f(z[h + 3] - mo.w));
+              __nv_bfloat162 b0 = __floats2bfloat162_rn(ex2_ftz(z[h] - mo.x), ex2_ftz(z[h + 1] - mo.y));
+              __nv_bfloat162 b1 = __floats2bfloat162_rn(ex2_ftz(z[h + 2] - mo.z), ex2_ftz(z[h + 3] - mo.w));
               // the denominator sums the same bf16-rounded weights the PV product uses
               const float2 r0 = __bfloat1622float2(b0), r1 = __bfloat1622float2(b1);
               lsum[h] = fmaf(lsum[h], fa.x, r0.x);
@@ -690,13 +704,21 @@ __global__ void __maxnreg__(128)
       // loads in the m8n8 fragment layout (thread t: channels c0 + t/4 and c0 + 8 + t/4, head
       // pairs 2(t%4) + 8k), scales and packs them to bf16 and writes them with transposing
       // 8x8 matrix stores, so each stored 16-byte row is 8 consecutive channels of one head.
-      // The rows land in the P buffer (free now) as two [64 heads x 64 channels] 128-byte
-      // swizzle boxes, which TMA stores to O.
+      // The rows land in the warp's own part of the P buffer (free now: 32 heads x 64 bytes
+      // of a 128-byte swizzled [64 heads x 64 channels] box), which the warp reads back as
+      // rows of one head and stores to O with 16-byte stores: no CTA barrier or bulk-copy
+      // wait between tiles.
       const int tq = lane & 3, mrow = lane & 7, mat = lane >> 3;
       float2 inv2[4];                                  // 1/denominator of this thread's heads
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) inv2[kk] = *reinterpret_cast<const float2*>(&s.inv[hb + 8 * kk + 2 * tq]);
       const uint32_t p0 = tc::smem_u32(s.p) + (uint32_t)((quad >> 1) * (AT_H * 128));
+      // read-back mapping: a phase of 8 lanes covers heads r and r + 4 (unit sets disjoint
+      // under the swizzle), 4 lanes per head row of 64 bytes
+      const int rb_u = 4 * (quad & 1) + (lane & 3);
+      const int rb_r = (lane >> 3) + 4 * ((lane >> 2) & 1);
+      __nv_bfloat16* const obase =
+          static_cast<__nv_bfloat16*>(a.O) + ((long long)it.qi * a.H + h0 + hb) * AT_C + 32 * quad + 8 * (lane & 3);
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[2][8];                             // [channel half][matrix slot]
 #pragma unroll
@@ -731,10 +753,7 @@ __global__ void __maxnreg__(128)
             pk[hh][2 * kk + 1] = pack_bf16(v[4 * kk + 2], v[4 * kk + 3]);
           }
         }
-        if (q > 0) {                                   // the previous tile's stores read P
-          if (tid == 0) tc::bulk_wait_read();
-          tc::named_barrier(1, AT_SOFT);
-        }
+        __syncwarp();                                  // the previous tile's read-back done
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
@@ -747,25 +766,27 @@ __global__ void __maxnreg__(128)
             tc::stmatrix_x4_trans(addr, pk[hh][4 * jx], pk[hh][4 * jx + 1], pk[hh][4 * jx + 2],
                                   pk[hh][4 * jx + 3]);
           }
-        tc::fence_proxy_async_smem();
-        tc::named_barrier(1, AT_SOFT);
-        if (tid == 0) {
-          const int orow = it.qi * a.H + h0;
-          tc::tma_store_2d(&map_o, s.p, 128 * q, orow);
-          tc::tma_store_2d(&map_o, s.p + AT_H * 128, 128 * q + 64, orow);
-          tc::bulk_commit();
-          A1_TRACE(24 + q, k, 0);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 8 * i + rb_r;                  // head hb + r
+          const int row = hb + r;
+          uint4 v;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                       : "r"(p0 + (uint32_t)(row * 128 + ((rb_u ^ (row & 7)) << 4)))
+                       : "memory");
+          *reinterpret_cast<uint4*>(obase + (long long)r * AT_C + 128 * q) = v;
         }
+        if (tid == 0) A1_TRACE(24 + q, k, 0);
       }
       // the next item's softmax writes P only after a barrier this thread reaches after here
-      if (tid == 0) tc::bulk_wait_read();
       tc::tc_fence_before();
       if (tid == 0) A1_TRACE(23, k, 0);
       ++k;
       it = nx;
       sink_h = nsink;
     }
-    if (tid == 0) tc::bulk_wait_all();                 // output stores complete before exit
   }
   tc::tc_fence_before();
   __syncthreads();
@@ -876,12 +897,9 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   }
   const long long nrows_local = (long long)a.B * a.R;
   if (nrows_local >= (1ll << 31) || !aligned16(a.O)) return DSV4_OK;
-  CUtensorMap mq, mo;
+  CUtensorMap mq;
   int s = encode_tensor_map_2d(&mq, a.Q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_q, 64,
                                AT_H, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (s != DSV4_OK) return s;
-  s = encode_tensor_map_2d(&mo, a.O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, AT_C, nrows_q, 64, AT_H,
-                           CU_TENSOR_MAP_SWIZZLE_128B);
   if (s != DSV4_OK) return s;
   // Few (query, head group) items: split each candidate list so that about one and a half
   // work items per SM exist, as far as the caller's workspace (a.nsplit = its capacity)
@@ -908,10 +926,10 @@ int launch_attn_tc(const AttnArgs& a_in, cudaStream_t st, bool* used) {
   const long long grid = (nsplit > 1 || work < sms) ? work : sms;
   if (nsplit > 1)
     attn_tc_kernel<true><<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(
-        a, mq, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
+        a, mq, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
   else
     attn_tc_kernel<false><<<(unsigned)grid, AT_THREADS, AT_SMEM, st>>>(
-        a, mq, mo, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
+        a, mq, a.H / AT_H, (int)work, a.scale * LOG2E, spin_limit());
   *used = true;
   int s2 = launch_status("hybrid attention (tensor cores)");
   if (s2 != DSV4_OK || nsplit == 1) return s2;
