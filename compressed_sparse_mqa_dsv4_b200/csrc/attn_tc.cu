@@ -160,6 +160,13 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// a0 += lo(v), a1 += hi(v) for a bf16 pair v, each widened exactly (sm_100 mixed-precision add)
+__device__ __forceinline__ void add_bf16x2_f32(float& a0, float& a1, uint32_t v) {
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %2;\n"
+      " add.rn.f32.bf16 %0, l, %0;\n add.rn.f32.bf16 %1, h, %1;\n}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(v));
+}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&p);
@@ -540,13 +547,9 @@ __global__ void __maxnreg__(128)
 #pragma unroll
               for (int i = 0; i < 16; ++i) pk[i] = 0u;
             }
+            // the denominator sums the same bf16-rounded weights the PV product uses
 #pragma unroll
-            for (int h = 0; h < 32; h += 2) {
-              // the denominator sums the same bf16-rounded weights the PV product uses
-              const float2 r = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pk[h / 2]));
-              lsum[h] += r.x;
-              lsum[h + 1] += r.y;
-            }
+            for (int h = 0; h < 32; h += 2) add_bf16x2_f32(lsum[h], lsum[h + 1], pk[h / 2]);
 #pragma unroll
             for (int c = 0; c < 4; ++c)
               *reinterpret_cast<uint4*>(prow + (((4 * half + c) ^ (slot & 7)) << 4)) =
