@@ -203,56 +203,96 @@ __device__ __forceinline__ void select_topk(const float* sc, int n, int keff, To
 }
 
 // Rows of at most R * NT entries: each thread holds its contiguous run of R keys in
-// registers for all four radix passes and the ordered compaction (the loop over global
-// loads re-read every key once per pass, one dependent load at a time).
+// registers for the radix passes and the ordered compaction (the loop over global loads
+// re-read every key once per pass, one dependent load at a time). A pass takes two barriers:
+// after the histogram updates, warp 0 alone scans the 256 digit counts (8 per lane) while the
+// other warps clear the second histogram for the next pass. The passes stop once the
+// selected bin is taken whole (its count is what is still needed): every key at or above the
+// digits fixed so far is selected and no tie needs breaking.
 template <int NT, int R, typename Emit>
 __device__ __forceinline__ void select_topk_regs(const float* sc, int n, int keff, TopkShared& sh,
                                                  Emit emit) {
-  int* hist = sh.hist;
+  static_assert(NT >= 64 && NT % 32 == 0, "one scanning warp and at least one clearing warp");
+  __shared__ __align__(16) int hist2[2][256];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int per = (n + NT - 1) / NT;              // <= R
   const int lo = threadIdx.x * per, hi = min(n, lo + per);
   uint32_t key[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) key[r] = (r < hi - lo) ? score_key(__ldg(sc + lo + r)) : 0u;
   const int cnt = max(0, hi - lo);
+  for (int t = threadIdx.x; t < 256; t += NT) hist2[0][t] = 0;
+  __syncthreads();
   uint32_t prefix = 0, pmask = 0;
   int remaining = keff;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    if (threadIdx.x < 256) hist[threadIdx.x] = 0;
-    __syncthreads();
+  bool whole = false;
+  int cur = 0;
+  for (int hi_bit = 31; hi_bit >= 0;) {
+    const int width = min(8, hi_bit + 1);
+    const int shift = hi_bit + 1 - width;
+    const uint32_t dmask = (1u << width) - 1u;
+    int* hist = hist2[cur];
 #pragma unroll
     for (int r = 0; r < R; ++r)
-      if (r < cnt && (key[r] & pmask) == prefix) atomicAdd(&hist[(key[r] >> shift) & 255u], 1);
+      if (r < cnt && (key[r] & pmask) == prefix) atomicAdd(&hist[(key[r] >> shift) & dmask], 1);
     __syncthreads();
-    const int d = 255 - (int)threadIdx.x;
-    const int h = d >= 0 ? hist[d] : 0;
-    int tot;
-    const int above = block_exclusive_scan<NT>(h, sh.warp_tot, tot);
-    if (d >= 0 && above < remaining && remaining <= above + h) {
-      sh.sel = d;
-      sh.above = above;
+    if (wid == 0) {
+      // lane l owns digits 255 - 8l - i, i = 0..7 (descending): lane-local sums, then a warp
+      // exclusive scan gives the count of keys in higher digits
+      const int4 h1 = *reinterpret_cast<const int4*>(&hist[248 - 8 * lane]);
+      const int4 h0 = *reinterpret_cast<const int4*>(&hist[252 - 8 * lane]);
+      const int v[8] = {h0.w, h0.z, h0.y, h0.x, h1.w, h1.z, h1.y, h1.x};
+      int tot = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) tot += v[i];
+      int incl = tot;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      int above = incl - tot;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (above < remaining && remaining <= above + v[i]) {
+          sh.sel = 255 - 8 * lane - i;
+          sh.above = above;
+          sh.cnt = v[i];
+        }
+        above += v[i];
+      }
+    } else {
+      for (int t = threadIdx.x - 32; t < 256; t += NT - 32) hist2[cur ^ 1][t] = 0;
     }
     __syncthreads();
     remaining -= sh.above;
     prefix |= (uint32_t)sh.sel << shift;
-    pmask |= 255u << shift;
-    __syncthreads();
+    pmask |= dmask << shift;
+    hi_bit -= width;
+    if (sh.cnt == remaining) {
+      whole = true;
+      break;
+    }
+    cur ^= 1;
   }
+  // selected: keys above T, and (unless the last bin was taken whole) the first `remaining`
+  // keys equal to T in entry order
   const uint32_t T = prefix;
   int n_gt = 0, n_eq = 0;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    n_gt += r < cnt && key[r] > T;
-    n_eq += r < cnt && key[r] == T;
+    n_gt += r < cnt && (whole ? key[r] >= T : key[r] > T);
+    n_eq += r < cnt && !whole && key[r] == T;
   }
-  int tot;
-  const int eq_before = block_exclusive_scan<NT>(n_eq, sh.warp_tot, tot);
-  const int take_eq = max(0, min(n_eq, remaining - eq_before));
+  int tot, take_eq = 0;
+  if (!whole) {
+    const int eq_before = block_exclusive_scan<NT>(n_eq, sh.warp_tot, tot);
+    take_eq = max(0, min(n_eq, remaining - eq_before));
+  }
   int pos = block_exclusive_scan<NT>(n_gt + take_eq, sh.warp_tot, tot), eq_seen = 0;
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    if (r < cnt && (key[r] > T || (key[r] == T && eq_seen++ < take_eq))) {
+    if (r < cnt && (whole ? key[r] >= T : (key[r] > T || (key[r] == T && eq_seen++ < take_eq)))) {
       if (pos < keff) emit(pos, lo + r);
       ++pos;
     }
