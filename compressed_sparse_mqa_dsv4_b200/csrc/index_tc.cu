@@ -61,6 +61,22 @@ constexpr int IX_SG_PAIRS = IX_BLK / 2 + 1;  // scale row pairs a block's stagin
 // a TMA tile's shared-memory destination must be 128-byte aligned: scale stages 1152 apart
 constexpr int IX_SG_STRIDE = (IX_SG_PAIRS * 16 + 127) / 128 * 128;
 
+// sum_h w[h] ReLU(d[h]) over 32 heads: four interleaved partial sums (heads h = j mod 4),
+// combined as (p0 + p1) + (p2 + p3). w: 16-byte aligned shared memory.
+__device__ __forceinline__ float ix_half_sum(const float (&d)[32], const float* w) {
+  const float4* wq = reinterpret_cast<const float4*>(w);
+  float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    const float4 wv = wq[h];
+    p0 = fmaf(wv.x, fmaxf(d[4 * h], 0.f), p0);
+    p1 = fmaf(wv.y, fmaxf(d[4 * h + 1], 0.f), p1);
+    p2 = fmaf(wv.z, fmaxf(d[4 * h + 2], 0.f), p2);
+    p3 = fmaf(wv.w, fmaxf(d[4 * h + 3], 0.f), p3);
+  }
+  return (p0 + p1) + (p2 + p3);
+}
+
 template <int QT, int NST, bool HIST, bool DYN, bool F4>
 struct IndexSmem {
   uint8_t q[2][QT * IX_HI * 128];           // K-major SW128: [QT*64 rows][64 ch] per K half
@@ -577,17 +593,7 @@ __global__ void __launch_bounds__(ix_threads<F4>(), 1)
           tc::tc_fence_before();
           tc::mbar_arrive(&s.d_empty[buf]);
           if (tid == 0) IX_TRACE(5, (int)gb);
-          const float4* wq = reinterpret_cast<const float4*>(&s.w[0][32 * hh]);
-          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
-#pragma unroll
-          for (int h = 0; h < 8; ++h) {
-            const float4 wv = wq[h];
-            p0 = fmaf(wv.x, fmaxf(d0[4 * h], 0.f), p0);
-            p1 = fmaf(wv.y, fmaxf(d0[4 * h + 1], 0.f), p1);
-            p2 = fmaf(wv.z, fmaxf(d0[4 * h + 2], 0.f), p2);
-            p3 = fmaf(wv.w, fmaxf(d0[4 * h + 3], 0.f), p3);
-          }
-          const float part = (p0 + p1) + (p2 + p3);
+          const float part = ix_half_sum(d0, &s.w[0][32 * hh]);
           const int e = 32 * quad + lane;
           if (hh == 1) s.part[buf][e] = part;
           tc::named_barrier(1, 256);
@@ -600,32 +606,28 @@ __global__ void __launch_bounds__(ix_threads<F4>(), 1)
           }
           if (tid == 0) IX_TRACE(6, (int)gb);
         } else {
-          float d0[32], d1[32], d2[32], d3[32];
           const uint32_t col = tmem + lane_base + buf * 256 + qp * 128;
           const bool two = 2 * qp < w.nqt;        // this warp has work in the tile
+          // per 32-head half four interleaved sums (short dependency chains), combined as the
+          // one-query tile combines them, so both tile shapes give the same scores; the
+          // second query's columns are read while the first query's are summed
+          float sc0 = 0.f, sc1 = 0.f;
           if (two) {
+            float d0[32], d1[32];
             tc::tmem_ld32(col, d0);
             tc::tmem_ld32(col + 32, d1);
-            tc::tmem_ld32(col + 64, d2);
-            tc::tmem_ld32(col + 96, d3);
             tc::tmem_wait_ld();
+            sc0 = ix_half_sum(d0, &s.w[2 * qp][0]) + ix_half_sum(d1, &s.w[2 * qp][32]);
+            tc::tmem_ld32(col + 64, d0);
+            tc::tmem_ld32(col + 96, d1);
+            tc::tmem_wait_ld();
+            sc1 = ix_half_sum(d0, &s.w[2 * qp + 1][0]) + ix_half_sum(d1, &s.w[2 * qp + 1][32]);
           }
           tc::tc_fence_before();
           tc::mbar_arrive(&s.d_empty[buf]);
           if (tid == 0) IX_TRACE(5, (int)gb);
           if (!two) continue;
           const int sidx = w.e0 + blk * IX_BLK + 32 * quad + lane;
-          float sc0 = 0.f, sc1 = 0.f;
-          const float* w0 = s.w[2 * qp];
-          const float* w1 = s.w[2 * qp + 1];
-#pragma unroll
-          for (int h = 0; h < 32; ++h) sc0 = fmaf(w0[h], fmaxf(d0[h], 0.f), sc0);
-#pragma unroll
-          for (int h = 0; h < 32; ++h) sc0 = fmaf(w0[32 + h], fmaxf(d1[h], 0.f), sc0);
-#pragma unroll
-          for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[h], fmaxf(d2[h], 0.f), sc1);
-#pragma unroll
-          for (int h = 0; h < 32; ++h) sc1 = fmaf(w1[32 + h], fmaxf(d3[h], 0.f), sc1);
           if (sidx < Et[0]) a.scores[srow[0] + sidx] = sc0;
           if (tid == 0) IX_TRACE(6, (int)gb);
           if (2 * qp + 1 < w.nqt && sidx < Et[1]) a.scores[srow[1] + sidx] = sc1;
