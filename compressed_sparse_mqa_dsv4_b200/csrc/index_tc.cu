@@ -608,9 +608,8 @@ __global__ void __launch_bounds__(ix_threads<F4>(), 1)
         } else {
           const uint32_t col = tmem + lane_base + buf * 256 + qp * 128;
           const bool two = 2 * qp < w.nqt;        // this warp has work in the tile
-          // per 32-head half four interleaved sums (short dependency chains), combined as the
-          // one-query tile combines them, so both tile shapes give the same scores; the
-          // second query's columns are read while the first query's are summed
+          // per 32-head half four interleaved sums (short dependency chains), combined in the
+          // one-query tile's order; one query's TMEM columns at a time (register budget)
           float sc0 = 0.f, sc1 = 0.f;
           if (two) {
             float d0[32], d1[32];
