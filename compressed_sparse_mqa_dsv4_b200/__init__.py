@@ -247,6 +247,8 @@ def decode_compress_fp8_job(C_new: torch.Tensor, Z_new: torch.Tensor, bias: torc
     B, c = _compress_common(C_new, Z_new, bias, tail, pool_row_off, m, overlap)
     _dev(codes, "codes", torch.uint8), _dev(scales, "scales", torch.float32)
     if rope_dims:
+        if rope is None:
+            raise ValueError(f"rope must be given for rope_dims={rope_dims}")
         _dev(rope, "rope", torch.bfloat16)
     if codes.shape[-1] != c - rope_dims:
         raise ValueError(f"codes rows must have {c - rope_dims} bytes")
@@ -276,8 +278,9 @@ def decode_compress_fp4_job(C_new: torch.Tensor, Z_new: torch.Tensor, bias: torc
 
 
 def dsv4_decode_state(jobs, pos: torch.Tensor, stream=None) -> None:
-    """One launch for a token's ring writes and compressor states: `jobs` from decode_ring_job
-    / decode_compress_job (same dtype and batch), pos int32 [B]."""
+    """One launch for a token's ring writes and compressor states: `jobs` from decode_ring_job,
+    decode_compress_job, decode_compress_fp8_job or decode_compress_fp4_job (same dtype and
+    batch; no two jobs writing the same memory), pos int32 [B]."""
     _dev(pos, "pos", torch.int32)
     if not jobs:
         return

@@ -134,3 +134,36 @@ def test_binding_argtypes_match_the_header():
             assert have in _ctype_for(p) or struct_ptr, f"{name} arg {i} ({p}): {have}"
         checked += 1
     assert checked >= 10
+
+
+def test_packed_decode_job_checks():
+    """The FP8 / FP4 compressor jobs of dsv4_decode_state check their pool shapes and dtypes
+    before any pointer is taken."""
+    B, c, cI, m, rd = 2, 576, 128, 4, 64
+    C = _FakeCuda(torch.zeros(B, 2 * c, dtype=torch.bfloat16))
+    bias = _FakeCuda(torch.zeros(2, m, c))
+    tail = _FakeCuda(torch.zeros(B, 2 * m, 2, 2 * c, dtype=torch.bfloat16))
+    off = _FakeCuda(torch.zeros(B, dtype=torch.int64))
+    codes = _FakeCuda(torch.zeros(8, c - rd, dtype=torch.uint8))
+    scales = _FakeCuda(torch.zeros(8, (c - rd) // 64))
+    rope = _FakeCuda(torch.zeros(8, rd, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="codes rows must have"):
+        dsv4.decode_compress_fp8_job(C, C, bias, tail, _FakeCuda(torch.zeros(8, c, dtype=torch.uint8)),
+                                     scales, rope, off, m, True, rd)
+    with pytest.raises(ValueError, match="rope must be given"):
+        dsv4.decode_compress_fp8_job(C, C, bias, tail, codes, scales, None, off, m, True, rd)
+    with pytest.raises(ValueError, match="scales must be"):
+        dsv4.decode_compress_fp8_job(C, C, bias, tail, codes, _FakeCuda(torch.zeros(8, 7, dtype=torch.uint8)),
+                                     rope, off, m, True, rd)
+    with pytest.raises(ValueError, match="tail must be"):
+        dsv4.decode_compress_fp8_job(C, C, bias, _FakeCuda(torch.zeros(B, m, 2, 2 * c, dtype=torch.bfloat16)),
+                                     codes, scales, rope, off, m, True, rd)
+    CI = _FakeCuda(torch.zeros(B, 2 * cI, dtype=torch.bfloat16))
+    biasI = _FakeCuda(torch.zeros(2, m, cI))
+    tailI = _FakeCuda(torch.zeros(B, 2 * m, 2, 2 * cI, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="FP4 pool rows"):
+        dsv4.decode_compress_fp4_job(CI, CI, biasI, tailI, _FakeCuda(torch.zeros(8, cI // 2, dtype=torch.uint8)),
+                                     _FakeCuda(torch.zeros(8, cI // 32, dtype=torch.uint8)), off, m, True)
+    with pytest.raises(ValueError, match="scales must be"):
+        dsv4.decode_compress_fp4_job(CI, CI, biasI, tailI, _FakeCuda(torch.zeros(8, cI // 2, dtype=torch.uint8)),
+                                     _FakeCuda(torch.zeros(8, cI // 16)), off, m, True)
