@@ -41,7 +41,7 @@ UNIT = "tokens/s"
 # DRAM traffic of the attention kernel per launch, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the attention
 # sources it was measured on; reported as null once those sources change.
-ATTN_TRAFFIC = {"sources_sha1": "45c8bb725b7d7eabe85219b3ac30e2d7d74379a0",
+ATTN_TRAFFIC = {"sources_sha1": "bf087f975892cb2814b868345dd23be8dc40e9c6",
                 "bytes_per_launch": 562_292_992 + 496_906_752}
 ATTN_SOURCES = ("attn_common.cuh", "attn_tc.cu", "dsv4_common.cuh", "rope.cuh", "tc_common.cuh")
 
