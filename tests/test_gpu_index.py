@@ -139,6 +139,30 @@ def test_index_long_rows_radix_path(dsv4):
     _run_and_check(dsv4, qI, w, KI, [0], pos0, 4, 1000, [(0, 0), (0, 1)], what="radix ties")
 
 
+@pytest.mark.parametrize("kind", ["few_values", "all_equal", "mostly_zero"])
+def test_index_short_rows_ties(dsv4, kind):
+    """Rows of at most 2048 entries (the select that keeps each thread's keys in registers and
+    stops its radix passes once a bin is taken whole) whose scores take a few distinct values,
+    a single value, or are zero for most entries (ReLU of negative dot products) with the k-th
+    place among the zeros. Integer-valued operands keep every score exact on both sides."""
+    g = Generator(13)
+    E = 1800
+    qI = (g.normal("qI", (1, 3, 4, 16), 1.0)).round().to(torch.bfloat16)
+    if kind == "few_values":
+        KI = (g.normal("KI", (E + 1, 16), 1.0) * 2).round().clamp(-3, 3).to(torch.bfloat16)
+    elif kind == "all_equal":
+        KI = torch.ones(E + 1, 16).to(torch.bfloat16)
+    else:
+        qI = qI.abs()
+        KI = -(g.normal("KI", (E + 1, 16), 1.0).abs() * 2).round().clamp(1, 3)
+        KI[::17] = -KI[::17]                       # about 106 entries with positive scores
+        KI = KI.to(torch.bfloat16)
+    w = torch.ones(1, 3, 4)
+    pos0 = [4 * E - 3]                             # E_t = E - 1, E - 1, E
+    _run_and_check(dsv4, qI, w, KI, [0], pos0, 4, 300, [(0, 0), (0, 1), (0, 2)],
+                   what=f"short-row {kind}")
+
+
 def test_index_decode_long_contexts(dsv4):
     """Decode over long contexts: one query per sequence, rows of 17.5k-75k entries (the
     workspace path: histograms of the top 16 key bits, a filter pass, then a select among
